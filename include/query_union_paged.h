@@ -1,0 +1,166 @@
+/*
+ * query_union_paged.h -- C ABI of the B200 (sm_100a) library for token-level
+ * sparse-attention prefill over a paged KV cache with page-affine query unions.
+ *
+ * Source of the operations: "PageWeaver: KV-Guided Query Unions for Sparse
+ * Attention" (Abstract; Figure 1; Figure 2; Figure 3).  Each query attends only
+ * to the tokens of its own TopK selected KV pages, causally inside a page.
+ * Queries that share pages are gathered into unions of up to max_group queries,
+ * so each union page is streamed once and fills tensor-core tiles, while every
+ * query keeps exactly its own support and writes its output row at its
+ * original query ID (no reordered Q tensor, no cross-page partial outputs).
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller; the
+ *    library never allocates or frees device memory.  Host pointers are read
+ *    during the call only.
+ *  - Calls are asynchronous on the given stream (cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and do not synchronize.
+ *  - The return value is QUP_OK or a synchronous error (bad argument, capacity,
+ *    launch failure).  Errors found on the device (a page ID out of range, a
+ *    bad group, a timed-out pipeline wait) are ORed into a per-device error
+ *    word, read and cleared by qup_get_error().  No call aborts or traps.
+ *
+ * Layouts (row-major, innermost last)
+ *   Q          [Nq][Hq][d]              bf16 or fp32
+ *   K, V cache [P_phys][Hkv][T][d]      bf16, fp32 or FP8 E4M3 (+ fp32 scale per KV head)
+ *   page_table [num_logical_pages]      int32, logical page -> physical page
+ *   topk       [Hq][Nq][Ksel]           int32 logical page IDs, -1 = padding
+ *   q_pos      [Nq]                     int32 token position of each query
+ *   O          [Nq][Hq][d]              dtype of Q
+ * Token t (logical position) lives in logical page t / T, slot t % T.  Query
+ * i with position q_pos[i] attends token t iff the page of t is in its row of
+ * topk, t <= q_pos[i] and t < kv_len.  KV head of Q head h' is h' / (Hq/Hkv).
+ */
+#ifndef QUERY_UNION_PAGED_H
+#define QUERY_UNION_PAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes and device error bits */
+#define QUP_OK 0
+#define QUP_ERR_ARG 1          /* null pointer, bad dimension, unsupported dtype or limit */
+#define QUP_ERR_CAPACITY 2     /* workspace or union capacity too small */
+#define QUP_ERR_CUDA 4         /* a CUDA runtime call or launch failed */
+#define QUP_ERR_PAGE_ID 8      /* device: a TopK or union page ID outside [0, num_logical_pages) */
+#define QUP_ERR_PHYS_PAGE 16   /* device: a page_table entry outside [0, P_phys) */
+#define QUP_ERR_GROUP 32       /* device: a group with no members, too many rows or a bad query ID */
+#define QUP_ERR_TIMEOUT 64     /* device: a pipeline wait exceeded its limit; the kernel exited cleanly */
+
+/* dtype codes */
+#define QUP_F32 0
+#define QUP_BF16 1
+#define QUP_E4M3 2
+
+/*
+ * Output of qup_sparse_group (every buffer is device memory, caller-allocated;
+ * sizes from qup_group_workspace).  For KV head h and group k:
+ *   members  [h*Nq + group_ptr[h*(Nq+1)+k] .. h*Nq + group_ptr[h*(Nq+1)+k+1])
+ *            query IDs of the group, ascending (at most max_group)
+ *   union    [union_ptr[h*(Nq+1)+k] .. union_ptr[h*(Nq+1)+k+1]) indexes
+ *            union_pages (sorted distinct logical pages of the group) and
+ *            row_mask (bit r = rank*g + j set iff that page is in row
+ *            topk[h*g+j][member of that rank]); offsets are absolute, the
+ *            regions of the KV heads follow each other in head order.
+ *   counters [h*4 + 0..3] = logical page visits (sum of union sizes), masked
+ *            row slots, masked query slots, page edges (sum of |S(i)|).
+ * (Figure 2: logical page visits and masked query-page slots.)
+ */
+typedef struct {
+    int32_t* n_groups;     /* [Hkv] */
+    int32_t* group_ptr;    /* [Hkv][Nq+1] */
+    int32_t* members;      /* [Hkv][Nq] */
+    int32_t* union_ptr;    /* [Hkv][Nq+1] */
+    int32_t* union_pages;  /* [cap_union] */
+    uint64_t* row_mask;    /* [cap_union] */
+    int64_t* counters;     /* [Hkv][4] */
+    int64_t cap_union;     /* entries available in union_pages and row_mask */
+} qup_groups;
+
+/*
+ * Sizes for qup_sparse_group.  Writes the scratch workspace bytes and the
+ * union capacity that is always sufficient (Hkv * Nq * min(g*Ksel, pages)).
+ * Returns QUP_ERR_ARG for unsupported sizes (window > 256, max_group*g > 32,
+ * too many pages for the shared-memory bitsets).
+ */
+int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int max_group,
+                        int window, size_t* ws_bytes, int64_t* cap_union);
+
+/*
+ * Bounded page-affinity grouping (Abstract: "a bounded GPU search produces
+ * query IDs" from selected-page affinity; Figure 2).  Per KV head h, S(i) is
+ * the set of distinct valid pages of the g rows topk[h*g+j][i]; inside fixed
+ * windows [w*window, (w+1)*window) of query IDs a group is seeded with the
+ * smallest unassigned ID and grown, up to max_group members, by the candidate
+ * that adds the fewest pages to the union (ties: smallest ID).  Output as in
+ * qup_groups; bit-exact with the CPU reference of the same rule.
+ *   topk       device int32 [Hq][Nq][Ksel]; -1 = padding, other IDs must lie
+ *              in [0, num_logical_pages) (else QUP_ERR_PAGE_ID, entry ignored)
+ *   max_group  1..8 and max_group*(Hq/Hkv) <= 32; window a multiple of
+ *              max_group, <= 256 (window == max_group gives fixed consecutive groups)
+ *   ws         device scratch of ws_bytes (from qup_group_workspace)
+ */
+int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages,
+                     int max_group, int window, const qup_groups* out, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * ID-aware union attention (Abstract; Figure 1; Figure 3).  One persistent
+ * kernel: per (KV head, group) it gathers the members' Q rows by original ID
+ * into shared memory, streams each union page's K and V once through a TMA
+ * ring, computes S^T = K Q^T and O^T += V^T P^T with tcgen05 MMAs into TMEM,
+ * applies each row's page mask and causal mask with an fp32 online softmax,
+ * and writes each row to O[qid][h'][:].
+ *   Q, q_dtype        device [Nq][Hq][d]; (QUP_F32 with kv QUP_F32) or
+ *                     (QUP_BF16 with kv QUP_BF16 or QUP_E4M3)
+ *   K_cache, V_cache  device [P_phys][Hkv][T][d], kv_dtype; 16-byte aligned
+ *   k_scale, v_scale  device fp32 [Hkv], required iff kv_dtype == QUP_E4M3
+ *   page_table        device int32 [num_logical_pages]
+ *   T                 page tokens: 16, 32, 64 or 128
+ *   topk, Ksel        accepted for the problem statement's signature; the
+ *                     groups' row masks carry each query's support and this
+ *                     call does not read topk (may be NULL)
+ *   groups            output of qup_sparse_group, or any partition with the
+ *                     same layout (at most 32 rows = members*g per group)
+ *   q_pos, kv_len     device int32 [Nq]; tokens >= kv_len are never attended
+ *   d                 must be 128; softmax_scale is applied to q.k
+ *   O                 device [Nq][Hq][d], dtype of Q; rows of queries that
+ *                     are in no group are not written
+ *   lse               device fp32 [Nq][Hq] natural-log sum of exponentials of
+ *                     the scaled scores, or NULL; empty support gives O = 0,
+ *                     lse = -inf
+ */
+int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache,
+                            int kv_dtype, const float* k_scale, const float* v_scale,
+                            const int32_t* page_table, int num_logical_pages, int P_phys, int T,
+                            const int32_t* topk, int Ksel, const qup_groups* groups,
+                            const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq, int d,
+                            float softmax_scale, void* O, float* lse, void* stream);
+
+/* Synchronizes `stream`, then reads and clears this device's error word. */
+int qup_get_error(int* code, void* stream);
+
+/* Static text for a return code or error bit. */
+const char* qup_error_string(int code);
+
+/*
+ * Pipeline-wait limit and host-side fault injection (for tests of the bounded
+ * waits; both reset with wait_limit_ms <= 0 and skip_stage < 0).  With
+ * skip_stage >= 0 the attention kernel's first CTA does not load that ring
+ * stage, so the consumer's wait runs out after wait_limit_ms, QUP_ERR_TIMEOUT
+ * is raised and every CTA exits cleanly.
+ */
+int qup_set_debug(int wait_limit_ms, int skip_stage);
+
+/* Number of SMs the persistent attention kernel is sized for on the current device. */
+int qup_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

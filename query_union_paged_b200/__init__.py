@@ -1,0 +1,220 @@
+"""B200 (sm_100a) paged sparse-attention prefill with page-affine query unions.
+
+Thin Python binding over the C ABI in ``include/query_union_paged.h`` (library
+``libqup.so`` built in-tree). Every step of the path runs in the library's
+CUDA kernels; this module only marshals arguments. PyTorch is used for device
+memory and streams. There is no CPU fallback: if the library is missing the
+calls raise.
+
+    groups = sparse_group(topk, Hq, Hkv, num_logical_pages, max_group=8, window=64)
+    O = sparse_prefill_attn(Q, K_cache, V_cache, page_table, groups, q_pos, kv_len, ...)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional
+
+__all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "get_error", "set_debug", "load",
+           "QupError", "F32", "BF16", "E4M3", "ERR"]
+
+F32, BF16, E4M3 = 0, 1, 2
+ERR = {"ARG": 1, "CAPACITY": 2, "CUDA": 4, "PAGE_ID": 8, "PHYS_PAGE": 16, "GROUP": 32, "TIMEOUT": 64}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqup.so")
+_lib = None
+
+
+class QupError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_strerror(code)} (code {code})")
+
+
+class _Groups(ctypes.Structure):
+    _fields_ = [("n_groups", ctypes.c_void_p), ("group_ptr", ctypes.c_void_p),
+                ("members", ctypes.c_void_p), ("union_ptr", ctypes.c_void_p),
+                ("union_pages", ctypes.c_void_p), ("row_mask", ctypes.c_void_p),
+                ("counters", ctypes.c_void_p), ("cap_union", ctypes.c_int64)]
+
+
+def load():
+    """Load libqup.so (in-tree). Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                           "`python -m query_union_paged_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.qup_group_workspace.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ), ctypes.POINTER(I64)]
+    lib.qup_sparse_group.argtypes = [P, I, I, I, I, I, I, I, ctypes.POINTER(_Groups), P, SZ, P]
+    lib.qup_sparse_prefill_attn.argtypes = [P, I, P, P, I, P, P, P, I, I, I, P, I,
+                                            ctypes.POINTER(_Groups), P, I, I, I, I, I,
+                                            ctypes.c_float, P, P, P]
+    lib.qup_get_error.argtypes = [ctypes.POINTER(I), P]
+    lib.qup_error_string.argtypes = [I]
+    lib.qup_error_string.restype = ctypes.c_char_p
+    lib.qup_set_debug.argtypes = [I, I]
+    lib.qup_num_sms.argtypes = []
+    for fn in ("qup_group_workspace", "qup_sparse_group", "qup_sparse_prefill_attn", "qup_get_error",
+               "qup_set_debug", "qup_num_sms"):
+        getattr(lib, fn).restype = I
+    _lib = lib
+    return lib
+
+
+def _strerror(code: int) -> str:
+    try:
+        return load().qup_error_string(code).decode()
+    except Exception:
+        return str(code)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise QupError(rc, where)
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+@dataclasses.dataclass
+class Groups:
+    """Device output of sparse_group (see qup_groups in the C header)."""
+    n_groups: "torch.Tensor"
+    group_ptr: "torch.Tensor"
+    members: "torch.Tensor"
+    union_ptr: "torch.Tensor"
+    union_pages: "torch.Tensor"
+    row_mask: "torch.Tensor"
+    counters: "torch.Tensor"
+    workspace: Optional["torch.Tensor"] = None
+
+    def c_struct(self) -> _Groups:
+        return _Groups(self.n_groups.data_ptr(), self.group_ptr.data_ptr(), self.members.data_ptr(),
+                       self.union_ptr.data_ptr(), self.union_pages.data_ptr(),
+                       self.row_mask.data_ptr(), self.counters.data_ptr(),
+                       self.union_pages.numel())
+
+    @staticmethod
+    def from_host(d: dict, device) -> "Groups":
+        """Upload a grouping held as numpy arrays (keys as the C struct)."""
+        import torch
+        t = {k: torch.from_numpy(d[k].view("int64") if k == "row_mask" else d[k]).to(device)
+             for k in ("n_groups", "group_ptr", "members", "union_ptr", "union_pages", "row_mask",
+                       "counters")}
+        if t["union_pages"].numel() == 0:
+            t["union_pages"] = torch.zeros(1, dtype=torch.int32, device=device)
+            t["row_mask"] = torch.zeros(1, dtype=torch.int64, device=device)
+        return Groups(**t)
+
+
+def group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group=8, window=64):
+    lib = load()
+    ws = ctypes.c_size_t(0)
+    cap = ctypes.c_int64(0)
+    _check(lib.qup_group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window,
+                                   ctypes.byref(ws), ctypes.byref(cap)), "qup_group_workspace")
+    return ws.value, cap.value
+
+
+def alloc_groups(Hkv, Nq, cap, ws_bytes, device) -> Groups:
+    import torch
+    i32 = dict(dtype=torch.int32, device=device)
+    return Groups(n_groups=torch.empty(Hkv, **i32), group_ptr=torch.empty(Hkv, Nq + 1, **i32),
+                  members=torch.empty(Hkv, Nq, **i32), union_ptr=torch.empty(Hkv, Nq + 1, **i32),
+                  union_pages=torch.empty(cap, **i32),
+                  row_mask=torch.empty(cap, dtype=torch.int64, device=device),
+                  counters=torch.empty(Hkv, 4, dtype=torch.int64, device=device),
+                  workspace=torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device))
+
+
+def sparse_group(topk, Hq: int, Hkv: int, num_logical_pages: int, max_group: int = 8,
+                 window: int = 64, out: Optional[Groups] = None, stream=None) -> Groups:
+    """Page-affinity grouping of the queries of every KV head (qup_sparse_group).
+
+    topk: int32 CUDA tensor [Hq][Nq][Ksel], -1 = padding. Returns Groups on the device.
+    """
+    lib = load()
+    Hq_, Nq, Ksel = topk.shape
+    assert Hq_ == Hq and topk.is_cuda and topk.is_contiguous()
+    ws_bytes, cap = group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window)
+    if out is None:
+        out = alloc_groups(Hkv, Nq, cap, ws_bytes, topk.device)
+    cs = out.c_struct()
+    _check(lib.qup_sparse_group(_p(topk), Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window,
+                                ctypes.byref(cs), _p(out.workspace), out.workspace.numel(),
+                                _stream_ptr(stream)), "qup_sparse_group")
+    return out
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return E4M3
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def sparse_prefill_attn(Q, K_cache, V_cache, page_table, groups: Groups, q_pos, kv_len: int,
+                        k_scale=None, v_scale=None, topk=None, softmax_scale: Optional[float] = None,
+                        out=None, lse=None, num_logical_pages: Optional[int] = None, stream=None):
+    """Union attention over the groups (qup_sparse_prefill_attn).
+
+    Q [Nq][Hq][d] bf16/fp32; K_cache, V_cache [P_phys][Hkv][T][d] bf16/fp32/E4M3 (uint8 or
+    float8_e4m3fn, with fp32 k_scale/v_scale [Hkv]); page_table int32 [pages]; q_pos int32 [Nq].
+    Returns O [Nq][Hq][d] in Q's dtype (and fills lse [Nq][Hq] fp32 if given).
+    """
+    import torch
+    lib = load()
+    Nq, Hq, d = Q.shape
+    P_phys, Hkv, T, d2 = K_cache.shape
+    assert d2 == d and V_cache.shape == K_cache.shape
+    for t in (Q, K_cache, V_cache, page_table, q_pos):
+        assert t.is_cuda and t.is_contiguous()
+    if out is None:
+        out = torch.empty_like(Q)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if num_logical_pages is None:
+        num_logical_pages = page_table.numel()
+    cs = groups.c_struct()
+    ksel = topk.shape[-1] if topk is not None else 0
+    _check(lib.qup_sparse_prefill_attn(_p(Q), _dtype_code(Q), _p(K_cache), _p(V_cache),
+                                       _dtype_code(K_cache), _p(k_scale), _p(v_scale), _p(page_table),
+                                       num_logical_pages, P_phys, T, _p(topk), ksel, ctypes.byref(cs),
+                                       _p(q_pos), kv_len, Hq, Hkv, Nq, d, float(softmax_scale),
+                                       _p(out), _p(lse), _stream_ptr(stream)),
+           "qup_sparse_prefill_attn")
+    return out
+
+
+def get_error(stream=None) -> int:
+    """Synchronize the stream, then read and clear the device error word."""
+    lib = load()
+    code = ctypes.c_int(0)
+    _check(lib.qup_get_error(ctypes.byref(code), _stream_ptr(stream)), "qup_get_error")
+    return code.value
+
+
+def set_debug(wait_limit_ms: int = 0, skip_stage: int = -1):
+    _check(load().qup_set_debug(wait_limit_ms, skip_stage), "qup_set_debug")
+
+
+def num_sms() -> int:
+    return load().qup_num_sms()

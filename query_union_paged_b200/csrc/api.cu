@@ -1,0 +1,305 @@
+// api.cu -- C ABI host layer: argument validation, workspace carving, TMA
+// tensor-map encoding, launches and the per-device error word.  Nothing here
+// allocates device memory; every buffer comes from the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "query_union_paged.h"
+
+namespace {
+
+__device__ unsigned g_err_word;  // ORed device error bits, read and cleared by qup_get_error
+
+constexpr int kMaxDevices = 64;
+
+struct DevState {
+    bool ready = false;
+    unsigned* err = nullptr;  // device address of g_err_word on this device
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+std::mutex g_mu;
+DevState g_dev[kMaxDevices];
+int g_wait_limit_ms = 0;   // 0: default
+int g_skip_stage = -1;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int device_state(DevState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QUP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevState& s = g_dev[dev];
+    if (!s.ready) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return QUP_ERR_CUDA;
+        s.err = static_cast<unsigned*>(p);
+        if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return QUP_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&s.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return QUP_ERR_CUDA;
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return QUP_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        s.ready = true;
+    }
+    *out = &s;
+    return QUP_OK;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct GroupWs {
+    size_t rowbits, usize, wtot, wcnt, total;
+};
+
+GroupWs group_ws_layout(int Hq, int Hkv, int Nq, int NW, int nwin) {
+    GroupWs w;
+    size_t off = 0;
+    w.rowbits = off;
+    off = align256(off + sizeof(uint32_t) * (size_t)Hq * Nq * NW);
+    w.usize = off;
+    off = align256(off + sizeof(int32_t) * (size_t)Hkv * Nq);
+    w.wtot = off;
+    off = align256(off + sizeof(int32_t) * (size_t)Hkv * nwin);
+    w.wcnt = off;
+    off = align256(off + sizeof(int32_t) * 3 * (size_t)Hkv * nwin);
+    w.total = off;
+    return w;
+}
+
+int check_group_args(int Hq, int Hkv, int Nq, int K, int P, int max_group, int window) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || K < 0 || P <= 0) return QUP_ERR_ARG;
+    const int g = Hq / Hkv;
+    if (max_group < 1 || max_group > 8 || max_group * g > 32) return QUP_ERR_ARG;
+    if (window < max_group || window % max_group != 0 || window > 256) return QUP_ERR_ARG;
+    return QUP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int max_group, int window,
+                        size_t* ws_bytes, int64_t* cap_union) {
+    int rc = check_group_args(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window);
+    if (rc) return rc;
+    const int NW = (num_logical_pages + 31) / 32;
+    const int nwin = (Nq + window - 1) / window;
+    // the greedy keeps the window's bitsets in shared memory (227 KB per CTA)
+    if (qup::group_greedy_smem(window, NW) > 227u * 1024u || 8u * 4u * (size_t)NW > 227u * 1024u) return QUP_ERR_ARG;
+    const int g = Hq / Hkv;
+    const int64_t cap = (int64_t)Hkv * Nq * std::min<int64_t>((int64_t)g * Ksel, num_logical_pages);
+    if (cap >= ((int64_t)1 << 31)) return QUP_ERR_ARG;  // union offsets are int32
+    if (ws_bytes) *ws_bytes = group_ws_layout(Hq, Hkv, Nq, NW, nwin).total;
+    if (cap_union) *cap_union = std::max<int64_t>(cap, 1);
+    return QUP_OK;
+}
+
+int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int max_group,
+                     int window, const qup_groups* out, void* ws, size_t ws_bytes, void* stream) {
+    size_t need = 0;
+    int64_t cap = 0;
+    int rc = qup_group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window, &need, &cap);
+    if (rc) return rc;
+    if (!out || !out->n_groups || !out->group_ptr || !out->members || !out->union_ptr || !out->union_pages ||
+        !out->row_mask || !out->counters)
+        return QUP_ERR_ARG;
+    if ((Nq > 0 && Ksel > 0 && !topk) || (!ws && need > 0)) return QUP_ERR_ARG;
+    if (ws_bytes < need) return QUP_ERR_CAPACITY;
+    if (out->cap_union < cap) return QUP_ERR_CAPACITY;
+    DevState* ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (Nq == 0) {  // nothing to group: zero groups, empty unions, zero counters
+        if (cudaMemsetAsync(out->n_groups, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(out->group_ptr, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(out->union_ptr, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(out->counters, 0, sizeof(int64_t) * 4 * Hkv, st) != cudaSuccess)
+            return QUP_ERR_CUDA;
+        return QUP_OK;
+    }
+    const int NW = (num_logical_pages + 31) / 32;
+    const int nwin = (Nq + window - 1) / window;
+    const GroupWs L = group_ws_layout(Hq, Hkv, Nq, NW, nwin);
+    char* base = static_cast<char*>(ws);
+    qup::GroupLaunch a;
+    a.topk = topk;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Nq = Nq;
+    a.K = Ksel;
+    a.P = num_logical_pages;
+    a.NW = NW;
+    a.max_group = max_group;
+    a.W = window;
+    a.nwin = nwin;
+    a.rowbits = reinterpret_cast<uint32_t*>(base + L.rowbits);
+    a.ws_usize = reinterpret_cast<int32_t*>(base + L.usize);
+    a.ws_wtot = reinterpret_cast<int32_t*>(base + L.wtot);
+    a.ws_wcnt = reinterpret_cast<int32_t*>(base + L.wcnt);
+    a.n_groups = out->n_groups;
+    a.group_ptr = out->group_ptr;
+    a.members = out->members;
+    a.union_ptr = out->union_ptr;
+    a.union_pages = out->union_pages;
+    a.row_mask = out->row_mask;
+    a.cap = out->cap_union;
+    a.counters = out->counters;
+    a.err = ds->err;
+    a.sms = ds->sms;
+    if (Ksel == 0) a.topk = nullptr;
+    return qup::launch_group(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+}
+
+int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
+                            const float* k_scale, const float* v_scale, const int32_t* page_table,
+                            int num_logical_pages, int P_phys, int T, const int32_t* topk, int Ksel,
+                            const qup_groups* groups, const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq,
+                            int d, float softmax_scale, void* O, float* lse, void* stream) {
+    (void)topk;
+    (void)Ksel;
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || d != qup::kHeadDim) return QUP_ERR_ARG;
+    if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
+    if (num_logical_pages <= 0 || P_phys <= 0 || kv_len < 0) return QUP_ERR_ARG;
+    if (!(std::isfinite(softmax_scale))) return QUP_ERR_ARG;
+    int es;
+    if (q_dtype == QUP_F32 && kv_dtype == QUP_F32) es = 4;
+    else if (q_dtype == QUP_BF16 && kv_dtype == QUP_BF16) es = 2;
+    else if (q_dtype == QUP_BF16 && kv_dtype == QUP_E4M3) es = 1;
+    else return QUP_ERR_ARG;
+    if (es == 1 && (!k_scale || !v_scale)) return QUP_ERR_ARG;
+    if (!groups || !groups->n_groups || !groups->group_ptr || !groups->members || !groups->union_ptr ||
+        !groups->union_pages || !groups->row_mask)
+        return QUP_ERR_ARG;
+    if (Nq == 0) return QUP_OK;
+    if (!Q || !K_cache || !V_cache || !page_table || !q_pos || !O) return QUP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(K_cache) | reinterpret_cast<uintptr_t>(V_cache)) & 15) return QUP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(Q) & 15)) return QUP_ERR_ARG;
+    const int g = Hq / Hkv;
+    // rows per group: members * g <= 32; one row tile of 16 or 32 columns
+    const int max_members = 32 / g;
+    if (max_members < 1) return QUP_ERR_ARG;
+    int r_pad = (std::min(8, max_members) * g <= 16) ? 16 : 32;
+    if (es != 2) r_pad = 32;  // E4M3 and tf32 P tiles need 32-byte / 128-byte rows
+    DevState* ds = nullptr;
+    int rc = device_state(&ds);
+    if (rc) return rc;
+
+    // K / V cache tensor maps: dims (d, T, Hkv, P_phys), box (128 bytes of d, T, 1, 1), 128B swizzle
+    CUtensorMap tm[2];
+    const CUtensorMapDataType dt = es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                           : (es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)Hkv, (cuuint64_t)P_phys};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)T * d * es, (cuuint64_t)Hkv * T * d * es};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)T, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const void* srcs[2] = {K_cache, V_cache};
+    for (int i = 0; i < 2; ++i) {
+        if (g_encode(&tm[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     // V^T is an MN-major operand; for tf32 its only layout uses 32-byte swizzle atoms
+                     (es == 4 && i == 1) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QUP_ERR_ARG;
+    }
+    // ring depth: as many K+V stages as shared memory allows
+    const size_t stage = 2u * qup::kStepTok * qup::kHeadDim * es;
+    const size_t fixed = qup::attn_smem_bytes(es, r_pad, 0, Hkv);
+    int ns = (int)std::min<size_t>(qup::kMaxStages, ((size_t)ds->smem_optin - fixed) / stage);
+    if (ns < 1) return QUP_ERR_ARG;
+    const size_t smem = qup::attn_smem_bytes(es, r_pad, ns, Hkv);
+    if (smem > (size_t)ds->smem_optin) return QUP_ERR_ARG;
+
+    qup::AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.Q = Q;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.page_table = page_table;
+    p.n_groups = groups->n_groups;
+    p.group_ptr = groups->group_ptr;
+    p.members = groups->members;
+    p.union_ptr = groups->union_ptr;
+    p.union_pages = groups->union_pages;
+    p.row_mask = groups->row_mask;
+    p.q_pos = q_pos;
+    p.O = O;
+    p.lse = lse;
+    p.err = ds->err;
+    p.cap_union = groups->cap_union;
+    p.num_logical_pages = num_logical_pages;
+    p.P_phys = P_phys;
+    p.T = T;
+    p.kv_len = kv_len;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.g = g;
+    p.max_members = std::min(8, max_members);
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.n_stages = ns;
+    p.wait_limit_ns = (unsigned long long)(g_wait_limit_ms > 0 ? g_wait_limit_ms : 2000) * 1000000ull;
+    p.dbg_skip_stage = g_skip_stage;
+    const cudaError_t e =
+        qup::launch_union_attn(es, r_pad, tm[0], tm[1], p, ds->sms, smem, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+}
+
+int qup_get_error(int* code, void* stream) {
+    if (!code) return QUP_ERR_ARG;
+    DevState* ds = nullptr;
+    int rc = device_state(&ds);
+    if (rc) return rc;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QUP_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(v)) != cudaSuccess) return QUP_ERR_CUDA;
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero)) != cudaSuccess) return QUP_ERR_CUDA;
+    *code = (int)v;
+    return QUP_OK;
+}
+
+const char* qup_error_string(int code) {
+    switch (code) {
+        case QUP_OK: return "ok";
+        case QUP_ERR_ARG: return "invalid argument";
+        case QUP_ERR_CAPACITY: return "workspace or union capacity too small";
+        case QUP_ERR_CUDA: return "CUDA runtime or launch failure";
+        case QUP_ERR_PAGE_ID: return "page ID out of range";
+        case QUP_ERR_PHYS_PAGE: return "page_table entry out of range";
+        case QUP_ERR_GROUP: return "malformed group";
+        case QUP_ERR_TIMEOUT: return "pipeline wait timed out";
+        default: return "multiple errors (bitwise OR of codes)";
+    }
+}
+
+int qup_set_debug(int wait_limit_ms, int skip_stage) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_wait_limit_ms = wait_limit_ms > 0 ? wait_limit_ms : 0;
+    g_skip_stage = skip_stage >= 0 ? skip_stage : -1;
+    return QUP_OK;
+}
+
+int qup_num_sms(void) {
+    DevState* ds = nullptr;
+    return device_state(&ds) == QUP_OK ? ds->sms : 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,316 @@
+// group.cu -- bounded page-affinity grouping (PageWeaver, Abstract: "a bounded
+// GPU search produces query IDs" from selected-page affinity; Figure 2:
+// logical page visits and masked query-page slots).
+//
+// Three kernels, all deterministic:
+//   1. rowbits: one warp per TopK row builds the row's page bitset (duplicates
+//      and -1 padding vanish; out-of-range IDs raise QUP_ERR_PAGE_ID).
+//   2. greedy:  one CTA per (window, KV head).  The g rows of each query are
+//      ORed into S(i) in shared memory; warp 0 then runs the greedy: seed =
+//      smallest unassigned query, add the candidate with the fewest pages
+//      outside the union (ties to the smallest ID) until max_group members or
+//      the window is exhausted.  The argmin is one warp reduction of the
+//      packed key (new_pages << 9 | local_id).
+//   3. emit:    one CTA per (window, KV head) sums the union sizes of all
+//      earlier windows for its absolute offset, then one warp per group
+//      writes the sorted union pages and per-page row masks from the bitsets.
+#include <algorithm>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "internal.h"
+#include "query_union_paged.h"
+
+namespace qup {
+
+__global__ void __launch_bounds__(256) grp_rowbits_kernel(const int32_t* __restrict__ topk, int Hq,
+                                                           int Hkv, int Nq, int K, int P, int NW,
+                                                           uint32_t* __restrict__ rowbits,
+                                                           int64_t* __restrict__ counters,
+                                                           unsigned* err) {
+    extern __shared__ uint32_t sm_rb[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* bits = sm_rb + warp * NW;
+    if (blockIdx.x == 0)
+        for (int x = threadIdx.x; x < Hkv * 4; x += blockDim.x) counters[x] = 0;
+    const int g = Hq / Hkv;
+    const long long nrows = (long long)Hq * Nq;
+    for (long long row = (long long)blockIdx.x * 8 + warp; row < nrows; row += (long long)gridDim.x * 8) {
+        const int hq = (int)(row / Nq), i = (int)(row % Nq);
+        for (int w = lane; w < NW; w += 32) bits[w] = 0;
+        __syncwarp();
+        const int32_t* tr = topk + row * K;
+        for (int k = lane; k < K; k += 32) {
+            const int p = tr[k];
+            if (p == -1) continue;
+            if (p < 0 || p >= P) {
+                atomicOr(err, QUP_ERR_PAGE_ID);
+                continue;
+            }
+            atomicOr(&bits[p >> 5], 1u << (p & 31));
+        }
+        __syncwarp();
+        const int h = hq / g, j = hq % g;
+        uint32_t* dst = rowbits + (((size_t)h * Nq + i) * g + j) * NW;
+        for (int w = lane; w < NW; w += 32) dst[w] = bits[w];
+        __syncwarp();
+    }
+}
+
+__global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restrict__ rowbits, int Hq,
+                                                          int Hkv, int Nq, int NW, int max_group, int W,
+                                                          int nwin, int32_t* __restrict__ group_ptr,
+                                                          int32_t* __restrict__ members,
+                                                          int32_t* __restrict__ n_groups,
+                                                          int32_t* __restrict__ ws_usize,
+                                                          int32_t* __restrict__ ws_wtot,
+                                                          int32_t* __restrict__ ws_wcnt) {
+    extern __shared__ uint32_t sm_gr[];
+    const int NWp = NW | 1;  // odd row pitch: lanes reading different queries hit different banks
+    uint32_t* S = sm_gr;
+    uint32_t* U = S + (size_t)W * NWp;
+    int* ssize = reinterpret_cast<int*>(U + NWp);
+    const int w = blockIdx.x, h = blockIdx.y, g = Hq / Hkv;
+    const int w0 = w * W, nw = min(W, Nq - w0);
+
+    for (int idx = threadIdx.x; idx < nw * NW; idx += blockDim.x) {
+        const int a = idx / NW, wd = idx % NW;
+        const uint32_t* src = rowbits + ((size_t)h * Nq + w0 + a) * g * NW + wd;
+        uint32_t v = 0;
+        for (int j = 0; j < g; ++j) v |= src[(size_t)j * NW];
+        S[a * NWp + wd] = v;
+    }
+    __syncthreads();
+    for (int a = threadIdx.x; a < nw; a += blockDim.x) {
+        int c = 0;
+        for (int wd = 0; wd < NW; ++wd) c += __popc(S[a * NWp + wd]);
+        ssize[a] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+
+    const int lane = threadIdx.x;
+    const int CPL = (W + 31) >> 5;  // candidates per lane: lane + 32k
+    uint32_t taken = 0;
+    for (int k = 0; k < CPL; ++k)
+        if (lane + 32 * k >= nw) taken |= 1u << k;
+    const int gbase = w * (W / max_group);
+    int ngw = 0, mpos = 0, visits = 0, masked_q = 0, edges = 0;
+    for (int a = lane; a < nw; a += 32) edges += ssize[a];
+    edges = __reduce_add_sync(0xffffffffu, edges);
+
+    while (true) {
+        unsigned my = 0xffffffffu;
+        for (int k = 0; k < CPL; ++k)
+            if (!((taken >> k) & 1u)) my = min(my, (unsigned)(lane + 32 * k));
+        const unsigned seed = __reduce_min_sync(0xffffffffu, my);
+        if (seed == 0xffffffffu) break;
+        if ((int)(seed & 31u) == lane) taken |= 1u << (seed >> 5);
+        for (int wd = lane; wd < NW; wd += 32) U[wd] = S[seed * NWp + wd];
+        __syncwarp();
+        int grp[8];
+        grp[0] = (int)seed;
+        int cnt = 1, sum_s = ssize[seed];
+        while (cnt < max_group) {
+            unsigned key = 0xffffffffu;
+            for (int k = 0; k < CPL; ++k) {
+                if ((taken >> k) & 1u) continue;
+                const int a = lane + 32 * k;
+                const uint32_t* sa = S + a * NWp;
+                int nc = 0;
+                for (int wd = 0; wd < NW; ++wd) nc += __popc(sa[wd] & ~U[wd]);
+                key = min(key, ((unsigned)nc << 9) | (unsigned)a);
+            }
+            const unsigned best = __reduce_min_sync(0xffffffffu, key);
+            if (best == 0xffffffffu) break;
+            const int c = (int)(best & 511u);
+            if ((c & 31) == lane) taken |= 1u << (c >> 5);
+            __syncwarp();
+            for (int wd = lane; wd < NW; wd += 32) U[wd] |= S[c * NWp + wd];
+            __syncwarp();
+            grp[cnt++] = c;
+            sum_s += ssize[c];
+        }
+        int us = 0;
+        for (int wd = lane; wd < NW; wd += 32) us += __popc(U[wd]);
+        us = __reduce_add_sync(0xffffffffu, us);
+        for (int a = 1; a < cnt; ++a) {  // ascending members
+            const int v = grp[a];
+            int b = a - 1;
+            while (b >= 0 && grp[b] > v) {
+                grp[b + 1] = grp[b];
+                --b;
+            }
+            grp[b + 1] = v;
+        }
+        if (lane == 0) {
+            for (int m = 0; m < cnt; ++m) members[(size_t)h * Nq + w0 + mpos + m] = w0 + grp[m];
+            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = w0 + mpos;
+            ws_usize[(size_t)h * Nq + gbase + ngw] = us;
+        }
+        mpos += cnt;
+        ++ngw;
+        visits += us;
+        masked_q += cnt * us - sum_s;
+        __syncwarp();
+    }
+    if (lane == 0) {
+        const int f = h * nwin + w;
+        ws_wtot[f] = visits;
+        ws_wcnt[f * 3 + 0] = visits;
+        ws_wcnt[f * 3 + 1] = masked_q;
+        ws_wcnt[f * 3 + 2] = edges;
+        if (w == nwin - 1) {
+            n_groups[h] = gbase + ngw;
+            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = Nq;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) grp_emit_kernel(
+    const uint32_t* __restrict__ rowbits, int Hq, int Hkv, int Nq, int NW, int max_group, int W,
+    int nwin, const int32_t* __restrict__ group_ptr, const int32_t* __restrict__ members,
+    const int32_t* __restrict__ ws_usize, const int32_t* __restrict__ ws_wtot,
+    const int32_t* __restrict__ ws_wcnt, int32_t* __restrict__ union_ptr,
+    int32_t* __restrict__ union_pages, uint64_t* __restrict__ row_mask, long long cap,
+    int64_t* __restrict__ counters, unsigned* err) {
+    extern __shared__ uint32_t sm_em[];
+    __shared__ long long red[8];
+    __shared__ long long s_base;
+    __shared__ int goff[257];
+    __shared__ int s_mem[8][8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w = blockIdx.x, h = blockIdx.y, g = Hq / Hkv;
+    const int f = h * nwin + w;
+
+    long long s = 0;
+    for (int x = threadIdx.x; x < f; x += blockDim.x) s += ws_wtot[x];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[warp] = s;
+    __syncthreads();
+    const int w0 = w * W, nw = min(W, Nq - w0);
+    const int ngw = (nw + max_group - 1) / max_group;
+    const int gbase = w * (W / max_group);
+    if (threadIdx.x == 0) {
+        long long b = 0;
+        for (int x = 0; x < 8; ++x) b += red[x];
+        s_base = b;
+        int o = 0;
+        for (int k = 0; k < ngw; ++k) {
+            goff[k] = o;
+            union_ptr[(size_t)h * (Nq + 1) + gbase + k] = (int32_t)(b + o);
+            o += ws_usize[(size_t)h * Nq + gbase + k];
+        }
+        goff[ngw] = o;
+        if (w == nwin - 1) union_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = (int32_t)(b + o);
+        if (b + o > cap) atomicOr(err, QUP_ERR_CAPACITY);
+    }
+    __syncthreads();
+    const long long base = s_base;
+    if (base + goff[ngw] > cap) return;
+
+    uint32_t* Uw = sm_em + warp * NW;
+    int masked_row = 0;
+    for (int k = warp; k < ngw; k += 8) {
+        const int gi = gbase + k;
+        const int p0 = group_ptr[(size_t)h * (Nq + 1) + gi];
+        const int nm = group_ptr[(size_t)h * (Nq + 1) + gi + 1] - p0;
+        const int R = nm * g;
+        if (lane < nm) s_mem[warp][lane] = members[(size_t)h * Nq + p0 + lane];
+        __syncwarp();
+        for (int wd = lane; wd < NW; wd += 32) {
+            uint32_t u = 0;
+            for (int m = 0; m < nm; ++m) {
+                const uint32_t* src = rowbits + ((size_t)h * Nq + s_mem[warp][m]) * g * NW + wd;
+                for (int j = 0; j < g; ++j) u |= src[(size_t)j * NW];
+            }
+            Uw[wd] = u;
+        }
+        __syncwarp();
+        const int wpl = (NW + 31) >> 5;
+        const int wb = min(NW, lane * wpl), we = min(NW, wb + wpl);
+        int c = 0;
+        for (int wd = wb; wd < we; ++wd) c += __popc(Uw[wd]);
+        int incl = c;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int rank = incl - c;
+        const long long out0 = base + goff[k];
+        int pop = 0;
+        for (int wd = wb; wd < we; ++wd) {
+            uint32_t word = Uw[wd];
+            if (!word) continue;
+            uint32_t rw[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r)
+                rw[r] = (r < R) ? rowbits[((size_t)h * Nq + s_mem[warp][r / g]) * g * NW +
+                                          (size_t)(r % g) * NW + wd]
+                                : 0u;
+            while (word) {
+                const int b = __ffs(word) - 1;
+                word &= word - 1;
+                uint64_t mk = 0;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) mk |= (uint64_t)((rw[r] >> b) & 1u) << r;
+                union_pages[out0 + rank] = wd * 32 + b;
+                row_mask[out0 + rank] = mk;
+                pop += __popcll(mk);
+                ++rank;
+            }
+        }
+        pop = __reduce_add_sync(0xffffffffu, pop);
+        masked_row += ws_usize[(size_t)h * Nq + gi] * R - pop;
+        __syncwarp();
+    }
+    __syncthreads();
+    if (lane == 0) red[warp] = masked_row;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long mr = 0;
+        for (int x = 0; x < 8; ++x) mr += red[x];
+        atomicAdd(reinterpret_cast<unsigned long long*>(&counters[h * 4 + 0]),
+                  (unsigned long long)ws_wcnt[f * 3 + 0]);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&counters[h * 4 + 1]), (unsigned long long)mr);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&counters[h * 4 + 2]),
+                  (unsigned long long)ws_wcnt[f * 3 + 1]);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&counters[h * 4 + 3]),
+                  (unsigned long long)ws_wcnt[f * 3 + 2]);
+    }
+}
+
+size_t group_greedy_smem(int W, int NW) {
+    const int NWp = NW | 1;
+    return sizeof(uint32_t) * ((size_t)W * NWp + NWp + W);
+}
+
+cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
+    const size_t sm1 = sizeof(uint32_t) * 8 * (size_t)a.NW;
+    const size_t sm2 = group_greedy_smem(a.W, a.NW);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(grp_rowbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm1)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(grp_greedy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm2)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(grp_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm1)) != cudaSuccess)
+        return e;
+    const long long rows = (long long)a.Hq * a.Nq;
+    const int grid1 = (int)std::min<long long>((rows + 7) / 8, (long long)a.sms * 8);
+    grp_rowbits_kernel<<<grid1, 256, sm1, stream>>>(a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW,
+                                                   a.rowbits, a.counters, a.err);
+    const dim3 grid2(a.nwin, a.Hkv);
+    grp_greedy_kernel<<<grid2, 128, sm2, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
+                                                   a.nwin, a.group_ptr, a.members, a.n_groups, a.ws_usize,
+                                                   a.ws_wtot, a.ws_wcnt);
+    grp_emit_kernel<<<grid2, 256, sm1, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
+                                                 a.nwin, a.group_ptr, a.members, a.ws_usize, a.ws_wtot,
+                                                 a.ws_wcnt, a.union_ptr, a.union_pages, a.row_mask, a.cap,
+                                                 a.counters, a.err);
+    return cudaGetLastError();
+}
+
+}  // namespace qup

@@ -1,0 +1,68 @@
+"""Shared test utilities: move a seeded workload to the GPU and compare results."""
+import numpy as np
+
+from query_union_paged_b200 import workloads as W
+
+
+def to_device(w, device="cuda"):
+    import torch
+    d = {}
+    Q = torch.from_numpy(np.ascontiguousarray(w.Q)).to(device)
+    d["Q"] = Q.view(torch.bfloat16) if w.q_dtype == W.DT_BF16 else Q
+    for name, arr in (("K", w.Kc), ("V", w.Vc)):
+        t = torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+        if w.kv_dtype == W.DT_BF16:
+            t = t.view(torch.bfloat16)
+        d[name] = t
+    d["k_scale"] = None if w.k_scale is None else torch.from_numpy(w.k_scale).to(device)
+    d["v_scale"] = None if w.v_scale is None else torch.from_numpy(w.v_scale).to(device)
+    d["page_table"] = torch.from_numpy(w.page_table).to(device)
+    d["topk"] = torch.from_numpy(w.topk).to(device)
+    d["q_pos"] = torch.from_numpy(w.q_pos).to(device)
+    return d
+
+
+def groups_to_host(gr):
+    """Device Groups -> dict of numpy arrays trimmed to the used union entries."""
+    n_groups = gr.n_groups.cpu().numpy()
+    union_ptr = gr.union_ptr.cpu().numpy()
+    Hkv = n_groups.size
+    total = int(union_ptr[Hkv - 1, n_groups[Hkv - 1]]) if Hkv else 0
+    return dict(n_groups=n_groups, group_ptr=gr.group_ptr.cpu().numpy(),
+                members=gr.members.cpu().numpy(), union_ptr=union_ptr,
+                union_pages=gr.union_pages[:total].cpu().numpy(),
+                row_mask=gr.row_mask[:total].cpu().numpy().view(np.uint64),
+                counters=gr.counters.cpu().numpy())
+
+
+def assert_groups_equal(got, ref):
+    Hkv = ref["n_groups"].size
+    assert np.array_equal(got["n_groups"], ref["n_groups"])
+    assert np.array_equal(got["counters"], ref["counters"])
+    for h in range(Hkv):
+        n = int(ref["n_groups"][h])
+        assert np.array_equal(got["group_ptr"][h, :n + 1], ref["group_ptr"][h, :n + 1])
+        m = int(ref["group_ptr"][h, n])
+        assert np.array_equal(got["members"][h, :m], ref["members"][h, :m])
+        assert np.array_equal(got["union_ptr"][h, :n + 1], ref["union_ptr"][h, :n + 1])
+    assert np.array_equal(got["union_pages"], ref["union_pages"])
+    assert np.array_equal(got["row_mask"], ref["row_mask"])
+
+
+def out_to_f64(O):
+    import torch
+    return O.float().cpu().numpy().astype(np.float64) if O.dtype != torch.float32 else \
+        O.cpu().numpy().astype(np.float64)
+
+
+# bounds from the arithmetic of each storage type (max abs, mean abs)
+TOL = {W.DT_F32: (2e-2, 2e-3), W.DT_BF16: (2e-2, 2e-3), W.DT_E4M3: (6e-2, 6e-3)}
+
+
+def check_close(got, ref, kv_dtype, what=""):
+    err = np.abs(got - ref)
+    mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
+    tmax, tmean = TOL[kv_dtype]
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert mx <= tmax and mean <= tmean, f"{what}: max abs {mx:.3e} (<= {tmax}), mean abs {mean:.3e} (<= {tmean})"
+    return mx, mean
