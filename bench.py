@@ -225,7 +225,7 @@ def main():
     vs = t(w.v_scale) if w.v_scale is not None else None
     topk, page_table, q_pos = t(w.topk), t(w.page_table), t(w.q_pos)
     ws_bytes, cap = qup.group_workspace(w.Hq, w.Hkv, w.Nq, w.K, w.num_logical_pages, max_group, window)
-    groups = qup.alloc_groups(w.Hkv, w.Nq, cap, ws_bytes, dev["Q"].device)
+    groups = qup.alloc_groups(w.Hq, w.Hkv, w.Nq, cap, ws_bytes, dev["Q"].device)
     O = torch.empty_like(dev["Q"])
     stream = torch.cuda.current_stream()
 
@@ -279,6 +279,7 @@ def main():
     n_uniq = unique_kv_pages(w)
     uniq_bytes = n_uniq * w.kv_page_bytes()
     ctr = groups.counters.cpu().numpy().sum(axis=0)
+    bctr = groups.bcounters.cpu().numpy().sum(axis=0)
     ms_per_step = total_ms / args.steps
     value = world * flop / (ms_per_step * 1e-3) / 1e12
     attn_ms = statistics.mean(t_attn)
@@ -308,7 +309,9 @@ def main():
         "work": {"selected_edges": E, "flop": flop, "unique_kv_pages": n_uniq,
                  "unique_kv_bytes": uniq_bytes, "logical_page_visits": int(ctr[0]),
                  "masked_row_slots": int(ctr[1]), "masked_query_slots": int(ctr[2]),
-                 "page_edges": int(ctr[3])},
+                 "page_edges": int(ctr[3]), "bundles": int(bctr[1]),
+                 "bundle_page_visits": int(bctr[0]),
+                 "streamed_kv_bytes": int(bctr[0]) * w.kv_page_bytes()},
         "roofline": {"kernel": "union_attn_kernel", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": round(mma_peak, 1), "unit": "TFLOP/s",
                      "frac": round(attn_tflops / mma_peak, 4),

@@ -70,6 +70,24 @@ extern "C" {
  *   counters [h*4 + 0..3] = logical page visits (sum of union sizes), masked
  *            row slots, masked query slots, page edges (sum of |S(i)|).
  * (Figure 2: logical page visits and masked query-page slots.)
+ *
+ * Bundles (the attention kernel's work items; no counterpart on the pages,
+ * which share a page between the two CTAs of one Union8 group instead):
+ * the groups of one KV head are packed, by the same greedy page-affinity
+ * rule applied to group unions inside windows of bundle_window groups, into
+ * bundles of up to 128 / rows_per_group groups.  A bundle's query rows are
+ * laid out slot by slot: row = slot*rows_per_group + rank*g + j, with
+ * rows_per_group = max_group*g rounded up to a power of two (<= 32).
+ *   bundle_ptr[h*(Nq+1)+b] .. [+b+1]  indexes bundle_groups[h*Nq + ...]
+ *            (group indices within head h, ascending = slot order)
+ *   bunion   [bunion_ptr[h*(Nq+1)+b] .. [+b+1]) indexes bunion_pages (sorted
+ *            union of the bundle's groups) and bunion_mask[4*entry + w]:
+ *            bit (row % 32) of word row/32 set iff the page is in that row's
+ *            own TopK row.
+ *   bundle_qid[(h*Nq + b)*(128/g) + row/g] = query ID of the row, -1 if the
+ *            slot or rank is empty.
+ *   bcounters[h*2 + 0..1] = bundle page visits (sum of bundle union sizes:
+ *            the pages the attention kernel streams), number of bundles.
  */
 typedef struct {
     int32_t* n_groups;     /* [Hkv] */
@@ -79,7 +97,17 @@ typedef struct {
     int32_t* union_pages;  /* [cap_union] */
     uint64_t* row_mask;    /* [cap_union] */
     int64_t* counters;     /* [Hkv][4] */
-    int64_t cap_union;     /* entries available in union_pages and row_mask */
+    int64_t cap_union;     /* entries available in union_pages/row_mask and in bunion_pages */
+    int32_t* n_bundles;    /* [Hkv] */
+    int32_t* bundle_ptr;   /* [Hkv][Nq+1] */
+    int32_t* bundle_groups;/* [Hkv][Nq] */
+    int32_t* bunion_ptr;   /* [Hkv][Nq+1] */
+    int32_t* bunion_pages; /* [cap_union] */
+    uint32_t* bunion_mask; /* [cap_union][4] */
+    int32_t* bundle_qid;   /* [Hkv][Nq][128/g] */
+    int64_t* bcounters;    /* [Hkv][2] */
+    int32_t rows_per_group;/* set by qup_sparse_group / qup_build_bundles */
+    int32_t bundle_window; /* groups per bundling window (0: default 64) */
 } qup_groups;
 
 /*
@@ -106,16 +134,27 @@ int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages
  *   ws         device scratch of ws_bytes (from qup_group_workspace)
  */
 int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages,
-                     int max_group, int window, const qup_groups* out, void* ws, size_t ws_bytes,
+                     int max_group, int window, qup_groups* out, void* ws, size_t ws_bytes,
                      void* stream);
 
 /*
+ * Pack the groups in `g` (n_groups .. row_mask filled, for instance by a
+ * caller's own partition) into bundles: fills n_bundles .. bcounters and
+ * rows_per_group.  max_group bounds the members of every group (1..8,
+ * max_group*(Hq/Hkv) <= 32).  qup_sparse_group calls this itself.
+ *   ws  device scratch of at least the size qup_group_workspace reports
+ */
+int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * ID-aware union attention (Abstract; Figure 1; Figure 3).  One persistent
- * kernel: per (KV head, group) it gathers the members' Q rows by original ID
- * into shared memory, streams each union page's K and V once through a TMA
- * ring, computes S^T = K Q^T and O^T += V^T P^T with tcgen05 MMAs into TMEM,
- * applies each row's page mask and causal mask with an fp32 online softmax,
- * and writes each row to O[qid][h'][:].
+ * kernel: per bundle (up to 128 query rows of one KV head) it gathers the
+ * rows of Q by original ID into shared memory, streams each page of the
+ * bundle union once through a TMA ring, computes S = Q K^T and O += P V with
+ * tcgen05 MMAs into TMEM (P written back to TMEM as the A operand), applies
+ * each row's page mask and causal mask with an fp32 online softmax, and
+ * writes each row to O[qid][h'][:].
  *   Q, q_dtype        device [Nq][Hq][d]; (QUP_F32 with kv QUP_F32) or
  *                     (QUP_BF16 with kv QUP_BF16 or QUP_E4M3)
  *   K_cache, V_cache  device [P_phys][Hkv][T][d], kv_dtype; 16-byte aligned
@@ -125,8 +164,8 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
  *   topk, Ksel        accepted for the problem statement's signature; the
  *                     groups' row masks carry each query's support and this
  *                     call does not read topk (may be NULL)
- *   groups            output of qup_sparse_group, or any partition with the
- *                     same layout (at most 32 rows = members*g per group)
+ *   groups            output of qup_sparse_group (or qup_build_bundles on
+ *                     any partition); the kernel walks its bundles
  *   q_pos, kv_len     device int32 [Nq]; tokens >= kv_len are never attended
  *   d                 must be 128; softmax_scale is applied to q.k
  *   O                 device [Nq][Hq][d], dtype of Q; rows of queries that

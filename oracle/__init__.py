@@ -54,6 +54,8 @@ def _load():
             lib.oracle_group.restype = I
             lib.oracle_build_unions.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, I64, P]
             lib.oracle_build_unions.restype = I
+            lib.oracle_bundle.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, I64, P]
+            lib.oracle_bundle.restype = I
             lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
             lib.oracle_e4m3_decode.restype = D
             lib.oracle_bf16_decode.argtypes = [ctypes.c_uint16]
@@ -189,3 +191,33 @@ def build_unions(topk, Hq, Hkv, Nq, num_logical_pages, partition):
     if rc:
         raise ValueError(f"oracle_build_unions: {ERRORS.get(rc, rc)}")
     return _trim(out)
+
+
+def bundle(groups, Hq, Hkv, Nq, max_group=8, bundle_window=64):
+    """Bundles of the groups (dict as returned by group/build_unions); adds bundle keys."""
+    lib = _load()
+    g = Hq // Hkv
+    cap = max(1, int(groups["union_pages"].size))
+    out = dict(n_bundles=np.zeros(Hkv, np.int32), bundle_ptr=np.zeros((Hkv, Nq + 1), np.int32),
+               bundle_groups=np.zeros((Hkv, Nq), np.int32), bunion_ptr=np.zeros((Hkv, Nq + 1), np.int32),
+               bunion_pages=np.zeros(cap, np.int32), bunion_mask=np.zeros((cap, 4), np.uint32),
+               bundle_qid=np.full((Hkv, Nq, 128 // g), -1, np.int32), bcounters=np.zeros((Hkv, 2), np.int64))
+    gr = {k: np.ascontiguousarray(groups[k]) for k in ("n_groups", "group_ptr", "members", "union_ptr",
+                                                      "union_pages", "row_mask")}
+    if gr["union_pages"].size == 0:
+        gr["union_pages"] = np.zeros(1, np.int32)
+        gr["row_mask"] = np.zeros(1, np.uint64)
+    rc = lib.oracle_bundle(Hq, Hkv, Nq, max_group, bundle_window,
+                           *(_ptr(gr[k]) for k in ("n_groups", "group_ptr", "members", "union_ptr",
+                                                   "union_pages", "row_mask")),
+                           *(_ptr(out[k]) for k in ("n_bundles", "bundle_ptr", "bundle_groups", "bunion_ptr",
+                                                    "bunion_pages", "bunion_mask", "bundle_qid")),
+                           cap, _ptr(out["bcounters"]))
+    if rc:
+        raise ValueError(f"oracle_bundle: {ERRORS.get(rc, rc)}")
+    total = int(out["bunion_ptr"][Hkv - 1, out["n_bundles"][Hkv - 1]]) if Hkv else 0
+    out["bunion_pages"] = out["bunion_pages"][:total].copy()
+    out["bunion_mask"] = out["bunion_mask"][:total].copy()
+    res = dict(groups)
+    res.update(out)
+    return res

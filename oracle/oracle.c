@@ -392,3 +392,127 @@ int oracle_group(const int32_t* topk, int Hq, int Hkv, int Nq, int K, int P,
     return oracle_build_unions(topk, Hq, Hkv, Nq, K, P, n_groups, group_ptr, members,
                                union_ptr, union_pages, row_mask, cap, counters);
 }
+
+/*
+ * Bundles (an execution-level packing with no counterpart on the pages): per
+ * KV head, the groups in order are cut into windows of wb groups; inside a
+ * window a bundle is seeded with the first unbundled group and grown, up to
+ * `slots` groups, by the group whose union adds the fewest pages to the
+ * bundle union (ties: smallest index).  Groups of a bundle are listed
+ * ascending (slot order).  Row of slot j, member rank m, head offset jj:
+ * j*rs + m*g + jj.  The 128-bit mask of a bundle page has the group's row
+ * mask of that page at bit offset j*rs.
+ *   rs = smallest power of two >= max_group*g; slots = 128/rs;
+ *   wb = max(slots, (bundle_window/slots)*slots).
+ * Inputs are the group arrays (as produced by oracle_group or
+ * oracle_build_unions).  bmask holds 4 uint32 per entry; bqid has 128/g
+ * entries per bundle slot of [Hkv][Nq].
+ */
+int oracle_bundle(int Hq, int Hkv, int Nq, int max_group, int bundle_window,
+                  const int32_t* n_groups, const int32_t* group_ptr, const int32_t* members,
+                  const int32_t* union_ptr, const int32_t* union_pages, const uint64_t* row_mask,
+                  int32_t* n_bundles, int32_t* bundle_ptr, int32_t* bundle_groups,
+                  int32_t* bunion_ptr, int32_t* bunion_pages, uint32_t* bmask, int32_t* bqid,
+                  int64_t cap, int64_t* bcounters) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq < 0 || max_group < 1) return ORC_EARG;
+    const int g = Hq / Hkv;
+    int rs = 1;
+    while (rs < max_group * g) rs <<= 1;
+    if (rs > 32) return ORC_EARG;
+    const int slots = 128 / rs;
+    int wb = bundle_window > 0 ? bundle_window : 64;
+    wb = (wb / slots) * slots;
+    if (wb < slots) wb = slots;
+    const int mq = 128 / g;
+    int64_t off = 0;
+    int rc = ORC_OK;
+    int pmax = 1;
+    for (int64_t e = 0; e < (Hkv > 0 ? union_ptr[(size_t)(Hkv - 1) * (Nq + 1) + n_groups[Hkv - 1]] : 0); ++e)
+        if (union_pages[e] + 1 > pmax) pmax = union_pages[e] + 1;
+    int32_t* U = (int32_t*)malloc(sizeof(int32_t) * (size_t)pmax);
+    int32_t* tmp = (int32_t*)malloc(sizeof(int32_t) * (size_t)pmax * 2 + 8);
+    char* taken = (char*)malloc((size_t)(wb > 0 ? wb : 1));
+    int32_t grp[128];
+    if (!U || !tmp || !taken) { free(U); free(tmp); free(taken); return ORC_EMEM; }
+    for (int h = 0; h < Hkv && rc == ORC_OK; ++h) {
+        const int32_t* gp = group_ptr + (size_t)h * (Nq + 1);
+        const int32_t* up = union_ptr + (size_t)h * (Nq + 1);
+        int32_t* bp = bundle_ptr + (size_t)h * (Nq + 1);
+        int32_t* bu = bunion_ptr + (size_t)h * (Nq + 1);
+        int nb = 0, nbg = 0;
+        int64_t visits = 0;
+        bp[0] = 0;
+        const int ng = n_groups[h];
+        for (int w0 = 0; w0 < ng && rc == ORC_OK; w0 += wb) {
+            const int nw = (ng - w0 < wb) ? ng - w0 : wb;
+            for (int a = 0; a < nw; ++a) taken[a] = 0;
+            for (int seed = 0; seed < nw; ++seed) {
+                if (taken[seed]) continue;
+                iset u = { U, up[w0 + seed + 1] - up[w0 + seed] };
+                memcpy(U, union_pages + up[w0 + seed], sizeof(int32_t) * (size_t)u.n);
+                taken[seed] = 1;
+                int cnt = 1;
+                grp[0] = seed;
+                while (cnt < slots) {
+                    int best = -1, bestc = 0;
+                    for (int c = seed + 1; c < nw; ++c) {
+                        if (taken[c]) continue;
+                        iset sc = { (int32_t*)union_pages + up[w0 + c], up[w0 + c + 1] - up[w0 + c] };
+                        int nc = set_minus_count(&sc, &u);
+                        if (best < 0 || nc < bestc) { best = c; bestc = nc; }
+                    }
+                    if (best < 0) break;
+                    taken[best] = 1;
+                    iset sb = { (int32_t*)union_pages + up[w0 + best], up[w0 + best + 1] - up[w0 + best] };
+                    set_union_into(&u, &sb, tmp);
+                    grp[cnt++] = best;
+                }
+                qsort(grp, (size_t)cnt, sizeof(int32_t), cmp_i32);
+                /* emit */
+                bu[nb] = (int32_t)off;
+                if (off + u.n > cap) { rc = ORC_ECAP; break; }
+                int32_t* q = bqid + ((size_t)h * Nq + nb) * mq;
+                for (int k = 0; k < mq; ++k) q[k] = -1;
+                for (int j = 0; j < cnt; ++j) {
+                    const int gi = w0 + grp[j];
+                    bundle_groups[(size_t)h * Nq + nbg + j] = gi;
+                    for (int m = 0; m < gp[gi + 1] - gp[gi]; ++m)
+                        q[j * (rs / g) + m] = members[(size_t)h * Nq + gp[gi] + m];
+                }
+                for (int a = 0; a < u.n; ++a) {
+                    uint32_t mk[4] = {0, 0, 0, 0};
+                    for (int j = 0; j < cnt; ++j) {
+                        const int gi = w0 + grp[j];
+                        /* the group's entry for this page, if any */
+                        int lo = up[gi], hi = up[gi + 1] - 1, at = -1;
+                        while (lo <= hi) {
+                            int mid = (lo + hi) / 2;
+                            if (union_pages[mid] == u.v[a]) { at = mid; break; }
+                            if (union_pages[mid] < u.v[a]) lo = mid + 1; else hi = mid - 1;
+                        }
+                        if (at < 0) continue;
+                        const uint64_t rm = row_mask[at];
+                        for (int r = 0; r < rs; ++r)
+                            if ((rm >> r) & 1) {
+                                const int row = j * rs + r;
+                                mk[row >> 5] |= 1u << (row & 31);
+                            }
+                    }
+                    bunion_pages[off + a] = u.v[a];
+                    for (int k = 0; k < 4; ++k) bmask[(off + a) * 4 + k] = mk[k];
+                }
+                off += u.n;
+                visits += u.n;
+                nbg += cnt;
+                bp[++nb] = nbg;
+            }
+        }
+        if (rc) break;
+        bu[nb] = (int32_t)off;
+        n_bundles[h] = nb;
+        bcounters[2 * h] = visits;
+        bcounters[2 * h + 1] = nb;
+    }
+    free(U); free(tmp); free(taken);
+    return rc;
+}

@@ -17,7 +17,10 @@ import math
 import os
 from typing import Optional
 
-__all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "get_error", "set_debug", "load",
+import numpy as np
+
+__all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host",
+           "get_error", "set_debug", "load",
            "QupError", "F32", "BF16", "E4M3", "ERR"]
 
 F32, BF16, E4M3 = 0, 1, 2
@@ -34,11 +37,15 @@ class QupError(RuntimeError):
         super().__init__(f"{where}: {_strerror(code)} (code {code})")
 
 
+_GROUP_KEYS = ("n_groups", "group_ptr", "members", "union_ptr", "union_pages", "row_mask", "counters")
+_BUNDLE_KEYS = ("n_bundles", "bundle_ptr", "bundle_groups", "bunion_ptr", "bunion_pages", "bunion_mask",
+                "bundle_qid", "bcounters")
+
+
 class _Groups(ctypes.Structure):
-    _fields_ = [("n_groups", ctypes.c_void_p), ("group_ptr", ctypes.c_void_p),
-                ("members", ctypes.c_void_p), ("union_ptr", ctypes.c_void_p),
-                ("union_pages", ctypes.c_void_p), ("row_mask", ctypes.c_void_p),
-                ("counters", ctypes.c_void_p), ("cap_union", ctypes.c_int64)]
+    _fields_ = ([(k, ctypes.c_void_p) for k in _GROUP_KEYS] + [("cap_union", ctypes.c_int64)] +
+                [(k, ctypes.c_void_p) for k in _BUNDLE_KEYS] +
+                [("rows_per_group", ctypes.c_int32), ("bundle_window", ctypes.c_int32)])
 
 
 def load():
@@ -53,6 +60,7 @@ def load():
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     lib.qup_group_workspace.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ), ctypes.POINTER(I64)]
     lib.qup_sparse_group.argtypes = [P, I, I, I, I, I, I, I, ctypes.POINTER(_Groups), P, SZ, P]
+    lib.qup_build_bundles.argtypes = [ctypes.POINTER(_Groups), I, I, I, I, I, P, SZ, P]
     lib.qup_sparse_prefill_attn.argtypes = [P, I, P, P, I, P, P, P, I, I, I, P, I,
                                             ctypes.POINTER(_Groups), P, I, I, I, I, I,
                                             ctypes.c_float, P, P, P]
@@ -61,8 +69,8 @@ def load():
     lib.qup_error_string.restype = ctypes.c_char_p
     lib.qup_set_debug.argtypes = [I, I]
     lib.qup_num_sms.argtypes = []
-    for fn in ("qup_group_workspace", "qup_sparse_group", "qup_sparse_prefill_attn", "qup_get_error",
-               "qup_set_debug", "qup_num_sms"):
+    for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
+               "qup_get_error", "qup_set_debug", "qup_num_sms"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -92,7 +100,8 @@ def _p(t):
 
 @dataclasses.dataclass
 class Groups:
-    """Device output of sparse_group (see qup_groups in the C header)."""
+    """Device output of sparse_group (see qup_groups in the C header): the groups and the
+    bundles the attention kernel walks."""
     n_groups: "torch.Tensor"
     group_ptr: "torch.Tensor"
     members: "torch.Tensor"
@@ -100,25 +109,26 @@ class Groups:
     union_pages: "torch.Tensor"
     row_mask: "torch.Tensor"
     counters: "torch.Tensor"
+    n_bundles: "torch.Tensor" = None
+    bundle_ptr: "torch.Tensor" = None
+    bundle_groups: "torch.Tensor" = None
+    bunion_ptr: "torch.Tensor" = None
+    bunion_pages: "torch.Tensor" = None
+    bunion_mask: "torch.Tensor" = None
+    bundle_qid: "torch.Tensor" = None
+    bcounters: "torch.Tensor" = None
     workspace: Optional["torch.Tensor"] = None
+    rows_per_group: int = 0
+    bundle_window: int = 0
 
     def c_struct(self) -> _Groups:
-        return _Groups(self.n_groups.data_ptr(), self.group_ptr.data_ptr(), self.members.data_ptr(),
-                       self.union_ptr.data_ptr(), self.union_pages.data_ptr(),
-                       self.row_mask.data_ptr(), self.counters.data_ptr(),
-                       self.union_pages.numel())
+        cs = _Groups(*[getattr(self, k).data_ptr() for k in _GROUP_KEYS], self.union_pages.numel(),
+                     *[getattr(self, k).data_ptr() for k in _BUNDLE_KEYS], self.rows_per_group,
+                     self.bundle_window)
+        return cs
 
-    @staticmethod
-    def from_host(d: dict, device) -> "Groups":
-        """Upload a grouping held as numpy arrays (keys as the C struct)."""
-        import torch
-        t = {k: torch.from_numpy(d[k].view("int64") if k == "row_mask" else d[k]).to(device)
-             for k in ("n_groups", "group_ptr", "members", "union_ptr", "union_pages", "row_mask",
-                       "counters")}
-        if t["union_pages"].numel() == 0:
-            t["union_pages"] = torch.zeros(1, dtype=torch.int32, device=device)
-            t["row_mask"] = torch.zeros(1, dtype=torch.int64, device=device)
-        return Groups(**t)
+    def _after(self, cs: _Groups):
+        self.rows_per_group = cs.rows_per_group
 
 
 def group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group=8, window=64):
@@ -130,20 +140,59 @@ def group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group=8, window=64
     return ws.value, cap.value
 
 
-def alloc_groups(Hkv, Nq, cap, ws_bytes, device) -> Groups:
+def alloc_groups(Hq, Hkv, Nq, cap, ws_bytes, device) -> Groups:
     import torch
     i32 = dict(dtype=torch.int32, device=device)
+    g = Hq // Hkv
+    cap = max(int(cap), 1)
     return Groups(n_groups=torch.empty(Hkv, **i32), group_ptr=torch.empty(Hkv, Nq + 1, **i32),
                   members=torch.empty(Hkv, Nq, **i32), union_ptr=torch.empty(Hkv, Nq + 1, **i32),
                   union_pages=torch.empty(cap, **i32),
                   row_mask=torch.empty(cap, dtype=torch.int64, device=device),
                   counters=torch.empty(Hkv, 4, dtype=torch.int64, device=device),
+                  n_bundles=torch.empty(Hkv, **i32), bundle_ptr=torch.empty(Hkv, Nq + 1, **i32),
+                  bundle_groups=torch.empty(Hkv, Nq, **i32), bunion_ptr=torch.empty(Hkv, Nq + 1, **i32),
+                  bunion_pages=torch.empty(cap, **i32), bunion_mask=torch.empty(cap, 4, **i32),
+                  bundle_qid=torch.empty(Hkv, max(Nq, 1), 128 // g, **i32),
+                  bcounters=torch.empty(Hkv, 2, dtype=torch.int64, device=device),
                   workspace=torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device))
+
+
+def groups_from_host(d: dict, Hq: int, Hkv: int, num_logical_pages: int, max_group: int = 8,
+                     device="cuda", stream=None) -> Groups:
+    """Upload a partition held as numpy arrays (keys as the C struct: n_groups .. counters)
+    and build its bundles on the device (qup_build_bundles)."""
+    import torch
+    Hkv_, Np1 = d["group_ptr"].shape
+    Nq = Np1 - 1
+    ws_bytes, cap = group_workspace(Hq, Hkv, Nq, 1, num_logical_pages, max_group, max_group)
+    cap = max(cap, int(d["union_pages"].size), 1)
+    gr = alloc_groups(Hq, Hkv, Nq, cap, ws_bytes, device)
+    for k in _GROUP_KEYS:
+        src = d[k].view("int64") if k == "row_mask" else d[k]
+        dst = getattr(gr, k)
+        if k in ("union_pages", "row_mask"):
+            dst[:src.size].copy_(torch.from_numpy(np.ascontiguousarray(src)))
+        else:
+            dst.copy_(torch.from_numpy(np.ascontiguousarray(src)))
+    build_bundles(gr, Hq, Hkv, Nq, num_logical_pages, max_group, stream=stream)
+    return gr
+
+
+def build_bundles(gr: Groups, Hq: int, Hkv: int, Nq: int, num_logical_pages: int, max_group: int = 8,
+                  stream=None) -> Groups:
+    lib = load()
+    cs = gr.c_struct()
+    _check(lib.qup_build_bundles(ctypes.byref(cs), Hq, Hkv, Nq, num_logical_pages, max_group,
+                                 _p(gr.workspace), gr.workspace.numel(), _stream_ptr(stream)),
+           "qup_build_bundles")
+    gr._after(cs)
+    return gr
 
 
 def sparse_group(topk, Hq: int, Hkv: int, num_logical_pages: int, max_group: int = 8,
                  window: int = 64, out: Optional[Groups] = None, stream=None) -> Groups:
-    """Page-affinity grouping of the queries of every KV head (qup_sparse_group).
+    """Page-affinity grouping of the queries of every KV head, then bundling (qup_sparse_group).
 
     topk: int32 CUDA tensor [Hq][Nq][Ksel], -1 = padding. Returns Groups on the device.
     """
@@ -152,11 +201,12 @@ def sparse_group(topk, Hq: int, Hkv: int, num_logical_pages: int, max_group: int
     assert Hq_ == Hq and topk.is_cuda and topk.is_contiguous()
     ws_bytes, cap = group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window)
     if out is None:
-        out = alloc_groups(Hkv, Nq, cap, ws_bytes, topk.device)
+        out = alloc_groups(Hq, Hkv, Nq, cap, ws_bytes, topk.device)
     cs = out.c_struct()
     _check(lib.qup_sparse_group(_p(topk), Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window,
                                 ctypes.byref(cs), _p(out.workspace), out.workspace.numel(),
                                 _stream_ptr(stream)), "qup_sparse_group")
+    out._after(cs)
     return out
 
 

@@ -83,6 +83,18 @@ GroupWs group_ws_layout(int Hq, int Hkv, int Nq, int NW, int nwin) {
     return w;
 }
 
+// Bundle geometry: rows per group slot (power of two >= max_group*g), slots
+// per 128-row bundle, and the bundling window (a multiple of the slots).
+void bundle_geometry(int g, int max_group, int bundle_window, int* RS, int* slots, int* WB) {
+    int rs = 1;
+    while (rs < max_group * g) rs <<= 1;
+    *RS = rs;
+    *slots = 128 / rs;
+    int wb = bundle_window > 0 ? bundle_window : 64;
+    wb = (wb / *slots) * *slots;
+    *WB = wb < *slots ? *slots : wb;
+}
+
 int check_group_args(int Hq, int Hkv, int Nq, int K, int P, int max_group, int window) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || K < 0 || P <= 0) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
@@ -100,25 +112,109 @@ int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages
     int rc = check_group_args(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window);
     if (rc) return rc;
     const int NW = (num_logical_pages + 31) / 32;
-    const int nwin = (Nq + window - 1) / window;
-    // the greedy keeps the window's bitsets in shared memory (227 KB per CTA)
-    if (qup::group_greedy_smem(window, NW) > 227u * 1024u || 8u * 4u * (size_t)NW > 227u * 1024u) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
+    int RS, slots, WB;
+    bundle_geometry(g, max_group, 0, &RS, &slots, &WB);
+    const int nwin = std::max((Nq + window - 1) / window, (Nq + slots - 1) / slots);
+    // the greedy kernels keep a window's bitsets in shared memory (227 KB per CTA)
+    if (qup::group_greedy_smem(window, NW) > 227u * 1024u || qup::group_greedy_smem(std::max(WB, 256), NW) > 227u * 1024u ||
+        8u * 4u * (size_t)NW > 227u * 1024u)
+        return QUP_ERR_ARG;
     const int64_t cap = (int64_t)Hkv * Nq * std::min<int64_t>((int64_t)g * Ksel, num_logical_pages);
     if (cap >= ((int64_t)1 << 31)) return QUP_ERR_ARG;  // union offsets are int32
-    if (ws_bytes) *ws_bytes = group_ws_layout(Hq, Hkv, Nq, NW, nwin).total;
+    (void)nwin;
+    if (ws_bytes) *ws_bytes = group_ws_layout(Hq, Hkv, Nq, NW, std::max(Nq, 1)).total;
     if (cap_union) *cap_union = std::max<int64_t>(cap, 1);
     return QUP_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group, void* ws,
+                DevState* ds, cudaStream_t st) {
+    const int gq = Hq / Hkv;
+    int RS, slots, WB;
+    bundle_geometry(gq, max_group, g->bundle_window, &RS, &slots, &WB);
+    g->rows_per_group = RS;
+    if (Nq == 0) {
+        if (cudaMemsetAsync(g->n_bundles, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(g->bundle_ptr, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(g->bunion_ptr, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
+            cudaMemsetAsync(g->bcounters, 0, sizeof(int64_t) * 2 * Hkv, st) != cudaSuccess)
+            return QUP_ERR_CUDA;
+        return QUP_OK;
+    }
+    const int NW = (num_logical_pages + 31) / 32;
+    const GroupWs L = group_ws_layout(Hq, Hkv, Nq, NW, std::max(Nq, 1));
+    char* base = static_cast<char*>(ws);
+    qup::BundleLaunch a;
+    a.Hkv = Hkv;
+    a.Nq = Nq;
+    a.P = num_logical_pages;
+    a.NW = NW;
+    a.g = gq;
+    a.RS = RS;
+    a.slots = slots;
+    a.WB = WB;
+    a.nwin = (Nq + WB - 1) / WB;
+    a.n_groups = g->n_groups;
+    a.group_ptr = g->group_ptr;
+    a.members = g->members;
+    a.union_ptr = g->union_ptr;
+    a.union_pages = g->union_pages;
+    a.row_mask = g->row_mask;
+    a.gbits = reinterpret_cast<uint32_t*>(base + L.rowbits);
+    a.ws_usize = reinterpret_cast<int32_t*>(base + L.usize);
+    a.ws_wtot = reinterpret_cast<int32_t*>(base + L.wtot);
+    a.ws_wcnt = reinterpret_cast<int32_t*>(base + L.wcnt);
+    a.n_bundles = g->n_bundles;
+    a.bundle_ptr = g->bundle_ptr;
+    a.bundle_groups = g->bundle_groups;
+    a.bunion_ptr = g->bunion_ptr;
+    a.bunion_pages = g->bunion_pages;
+    a.bunion_mask = g->bunion_mask;
+    a.bundle_qid = g->bundle_qid;
+    a.cap = g->cap_union;
+    a.bcounters = g->bcounters;
+    a.err = ds->err;
+    a.sms = ds->sms;
+    return qup::launch_bundles(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+}
+
+bool bundle_fields_ok(const qup_groups* g) {
+    return g->n_bundles && g->bundle_ptr && g->bundle_groups && g->bunion_ptr && g->bunion_pages && g->bunion_mask &&
+           g->bundle_qid && g->bcounters;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group, void* ws,
+                      size_t ws_bytes, void* stream) {
+    size_t need = 0;
+    int64_t cap = 0;
+    int rc = qup_group_workspace(Hq, Hkv, Nq, 1, num_logical_pages, max_group, max_group, &need, &cap);
+    if (rc) return rc;
+    if (!g || !g->n_groups || !g->group_ptr || !g->members || !g->union_ptr || !g->union_pages || !g->row_mask ||
+        !bundle_fields_ok(g))
+        return QUP_ERR_ARG;
+    if (!ws || ws_bytes < need) return QUP_ERR_CAPACITY;
+    DevState* ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    return run_bundles(g, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, static_cast<cudaStream_t>(stream));
+}
+
 int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int max_group,
-                     int window, const qup_groups* out, void* ws, size_t ws_bytes, void* stream) {
+                     int window, qup_groups* out, void* ws, size_t ws_bytes, void* stream) {
     size_t need = 0;
     int64_t cap = 0;
     int rc = qup_group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window, &need, &cap);
     if (rc) return rc;
     if (!out || !out->n_groups || !out->group_ptr || !out->members || !out->union_ptr || !out->union_pages ||
-        !out->row_mask || !out->counters)
+        !out->row_mask || !out->counters || !bundle_fields_ok(out))
         return QUP_ERR_ARG;
     if ((Nq > 0 && Ksel > 0 && !topk) || (!ws && need > 0)) return QUP_ERR_ARG;
     if (ws_bytes < need) return QUP_ERR_CAPACITY;
@@ -132,11 +228,11 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
             cudaMemsetAsync(out->union_ptr, 0, sizeof(int32_t) * Hkv, st) != cudaSuccess ||
             cudaMemsetAsync(out->counters, 0, sizeof(int64_t) * 4 * Hkv, st) != cudaSuccess)
             return QUP_ERR_CUDA;
-        return QUP_OK;
+        return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st);
     }
     const int NW = (num_logical_pages + 31) / 32;
     const int nwin = (Nq + window - 1) / window;
-    const GroupWs L = group_ws_layout(Hq, Hkv, Nq, NW, nwin);
+    const GroupWs L = group_ws_layout(Hq, Hkv, Nq, NW, std::max(Nq, 1));
     char* base = static_cast<char*>(ws);
     qup::GroupLaunch a;
     a.topk = topk;
@@ -164,7 +260,8 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
     a.err = ds->err;
     a.sms = ds->sms;
     if (Ksel == 0) a.topk = nullptr;
-    return qup::launch_group(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+    if (qup::launch_group(a, st) != cudaSuccess) return QUP_ERR_CUDA;
+    return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st);
 }
 
 int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
@@ -176,6 +273,7 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     (void)Ksel;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || d != qup::kHeadDim) return QUP_ERR_ARG;
     if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
+    // supported (dtype, page size) pairs: bf16 16/32/64/128, E4M3 64/128, fp32 32/64
     if (num_logical_pages <= 0 || P_phys <= 0 || kv_len < 0) return QUP_ERR_ARG;
     if (!(std::isfinite(softmax_scale))) return QUP_ERR_ARG;
     int es;
@@ -184,19 +282,14 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     else if (q_dtype == QUP_BF16 && kv_dtype == QUP_E4M3) es = 1;
     else return QUP_ERR_ARG;
     if (es == 1 && (!k_scale || !v_scale)) return QUP_ERR_ARG;
-    if (!groups || !groups->n_groups || !groups->group_ptr || !groups->members || !groups->union_ptr ||
-        !groups->union_pages || !groups->row_mask)
-        return QUP_ERR_ARG;
+    if ((es == 1 && T < 64) || (es == 4 && (T < 32 || T > 64))) return QUP_ERR_ARG;
+    if (!groups || !bundle_fields_ok(groups) || groups->rows_per_group < 1) return QUP_ERR_ARG;
     if (Nq == 0) return QUP_OK;
     if (!Q || !K_cache || !V_cache || !page_table || !q_pos || !O) return QUP_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(K_cache) | reinterpret_cast<uintptr_t>(V_cache)) & 15) return QUP_ERR_ARG;
-    if ((reinterpret_cast<uintptr_t>(Q) & 15)) return QUP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(groups->bunion_mask)) & 15) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
-    // rows per group: members * g <= 32; one row tile of 16 or 32 columns
-    const int max_members = 32 / g;
-    if (max_members < 1) return QUP_ERR_ARG;
-    int r_pad = (std::min(8, max_members) * g <= 16) ? 16 : 32;
-    if (es != 2) r_pad = 32;  // E4M3 and tf32 P tiles need 32-byte / 128-byte rows
+    if (128 % g != 0 || groups->rows_per_group % g != 0) return QUP_ERR_ARG;
     DevState* ds = nullptr;
     int rc = device_state(&ds);
     if (rc) return rc;
@@ -213,19 +306,18 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     for (int i = 0; i < 2; ++i) {
         if (g_encode(&tm[i], dt, 4, const_cast<void*>(srcs[i]), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     // V^T is an MN-major operand; for tf32 its only layout uses 32-byte swizzle atoms
+                     // V is an MN-major operand; for tf32 its only layout uses 32-byte swizzle atoms
                      (es == 4 && i == 1) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QUP_ERR_ARG;
     }
-    // ring depth: as many K+V stages as shared memory allows
-    const size_t stage = 2u * qup::kStepTok * qup::kHeadDim * es;
-    const size_t fixed = qup::attn_smem_bytes(es, r_pad, 0, Hkv);
-    int ns = (int)std::min<size_t>(qup::kMaxStages, ((size_t)ds->smem_optin - fixed) / stage);
-    if (ns < 1) return QUP_ERR_ARG;
-    const size_t smem = qup::attn_smem_bytes(es, r_pad, ns, Hkv);
-    if (smem > (size_t)ds->smem_optin) return QUP_ERR_ARG;
+    // a pipeline step covers one page (T >= 64) or 64 tokens of smaller pages
+    const int st = T >= 64 ? T : 64;
+    const size_t stage = 2u * st * qup::kHeadDim * es;
+    const size_t fixed = qup::attn_smem_bytes(es, st, 0, Hkv);
+    if ((size_t)ds->smem_optin < fixed + stage) return QUP_ERR_ARG;
+    const int ns = (int)std::min<size_t>(qup::kMaxStages, ((size_t)ds->smem_optin - fixed) / stage);
+    const size_t smem = qup::attn_smem_bytes(es, st, ns, Hkv);
 
     qup::AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -233,12 +325,11 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.page_table = page_table;
-    p.n_groups = groups->n_groups;
-    p.group_ptr = groups->group_ptr;
-    p.members = groups->members;
-    p.union_ptr = groups->union_ptr;
-    p.union_pages = groups->union_pages;
-    p.row_mask = groups->row_mask;
+    p.n_bundles = groups->n_bundles;
+    p.union_ptr = groups->bunion_ptr;
+    p.union_pages = groups->bunion_pages;
+    p.row_mask = groups->bunion_mask;
+    p.bundle_qid = groups->bundle_qid;
     p.q_pos = q_pos;
     p.O = O;
     p.lse = lse;
@@ -252,13 +343,12 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.Hkv = Hkv;
     p.Nq = Nq;
     p.g = g;
-    p.max_members = std::min(8, max_members);
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.n_stages = ns;
     p.wait_limit_ns = (unsigned long long)(g_wait_limit_ms > 0 ? g_wait_limit_ms : 2000) * 1000000ull;
     p.dbg_skip_stage = g_skip_stage;
     const cudaError_t e =
-        qup::launch_union_attn(es, r_pad, tm[0], tm[1], p, ds->sms, smem, static_cast<cudaStream_t>(stream));
+        qup::launch_union_attn(es, T, tm[0], tm[1], p, ds->sms, smem, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
 }
 

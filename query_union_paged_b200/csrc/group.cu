@@ -57,21 +57,40 @@ __global__ void __launch_bounds__(256) grp_rowbits_kernel(const int32_t* __restr
     }
 }
 
-__global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restrict__ rowbits, int Hq,
-                                                          int Hkv, int Nq, int NW, int max_group, int W,
+// Greedy packing of the items of one KV head inside one window.  Items are
+// queries (sets = the g TopK rows of the query, ORed) or groups (sets = the
+// group union bitset); n_items_dev == nullptr means Nq items per head.
+__global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restrict__ rowbits, int sets_per_item,
+                                                          int Hkv, int Nq, const int32_t* __restrict__ n_items_dev,
+                                                          int NW, int max_group, int W,
                                                           int nwin, int32_t* __restrict__ group_ptr,
                                                           int32_t* __restrict__ members,
                                                           int32_t* __restrict__ n_groups,
                                                           int32_t* __restrict__ ws_usize,
                                                           int32_t* __restrict__ ws_wtot,
-                                                          int32_t* __restrict__ ws_wcnt) {
+                                                          int32_t* __restrict__ ws_wcnt,
+                                                          int64_t* __restrict__ out_count) {
     extern __shared__ uint32_t sm_gr[];
     const int NWp = NW | 1;  // odd row pitch: lanes reading different queries hit different banks
     uint32_t* S = sm_gr;
     uint32_t* U = S + (size_t)W * NWp;
     int* ssize = reinterpret_cast<int*>(U + NWp);
-    const int w = blockIdx.x, h = blockIdx.y, g = Hq / Hkv;
-    const int w0 = w * W, nw = min(W, Nq - w0);
+    const int w = blockIdx.x, h = blockIdx.y, g = sets_per_item;
+    const int n_items = n_items_dev ? n_items_dev[h] : Nq;
+    const int w0 = w * W, nw = max(0, min(W, n_items - w0));
+    if (nw == 0) {  // window past the head's last item: contributes nothing
+        if (threadIdx.x == 0) {
+            const int f = h * nwin + w;
+            ws_wtot[f] = 0;
+            ws_wcnt[f * 3 + 0] = ws_wcnt[f * 3 + 1] = ws_wcnt[f * 3 + 2] = 0;
+            if (w == 0) {
+                n_groups[h] = 0;
+                group_ptr[(size_t)h * (Nq + 1)] = 0;
+                if (out_count) out_count[h * 2 + 1] = 0;
+            }
+        }
+        return;
+    }
 
     for (int idx = threadIdx.x; idx < nw * NW; idx += blockDim.x) {
         const int a = idx / NW, wd = idx % NW;
@@ -160,9 +179,10 @@ __global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restr
         ws_wcnt[f * 3 + 0] = visits;
         ws_wcnt[f * 3 + 1] = masked_q;
         ws_wcnt[f * 3 + 2] = edges;
-        if (w == nwin - 1) {
+        if (w0 + nw == n_items) {  // the window holding the head's last item
             n_groups[h] = gbase + ngw;
-            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = Nq;
+            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = w0 + mpos;
+            if (out_count) out_count[h * 2 + 1] = gbase + ngw;
         }
     }
 }
@@ -280,6 +300,167 @@ __global__ void __launch_bounds__(256) grp_emit_kernel(
     }
 }
 
+// ------------------------------------------------------------------ bundles
+
+// One warp per group: the group's union list -> its page bitset.
+__global__ void __launch_bounds__(256) bnd_gbits_kernel(const int32_t* __restrict__ n_groups,
+                                                         const int32_t* __restrict__ union_ptr,
+                                                         const int32_t* __restrict__ union_pages, int Hkv,
+                                                         int Nq, int P, int NW, uint32_t* __restrict__ gbits,
+                                                         int64_t* __restrict__ bcounters, unsigned* err) {
+    extern __shared__ uint32_t sm_gb[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* bits = sm_gb + warp * NW;
+    if (blockIdx.x == 0)
+        for (int x = threadIdx.x; x < Hkv * 2; x += blockDim.x) bcounters[x] = 0;
+    const long long total = (long long)Hkv * Nq;
+    for (long long it = (long long)blockIdx.x * 8 + warp; it < total; it += (long long)gridDim.x * 8) {
+        const int h = (int)(it / Nq), gi = (int)(it % Nq);
+        if (gi >= n_groups[h]) continue;  // warp-uniform
+        for (int x = lane; x < NW; x += 32) bits[x] = 0;
+        __syncwarp();
+        const int u0 = union_ptr[(size_t)h * (Nq + 1) + gi], u1 = union_ptr[(size_t)h * (Nq + 1) + gi + 1];
+        for (int e = u0 + lane; e < u1; e += 32) {
+            const int p = union_pages[e];
+            if (p < 0 || p >= P) {
+                atomicOr(err, QUP_ERR_PAGE_ID);
+                continue;
+            }
+            atomicOr(&bits[p >> 5], 1u << (p & 31));
+        }
+        __syncwarp();
+        uint32_t* dst = gbits + ((size_t)h * Nq + gi) * NW;
+        for (int x = lane; x < NW; x += 32) dst[x] = bits[x];
+        __syncwarp();
+    }
+}
+
+// One CTA per (bundle window, KV head): absolute offsets from the earlier
+// windows' totals, then one warp per bundle writes the merged union (sorted,
+// from the OR of the group bitsets), the 128-bit row masks (each group's row
+// mask placed at its slot) and the row -> query table.
+__global__ void __launch_bounds__(256) bnd_emit_kernel(
+    const uint32_t* __restrict__ gbits, int Hkv, int Nq, int NW, int g, int RS, int slots, int WB, int nwin,
+    const int32_t* __restrict__ group_ptr, const int32_t* __restrict__ members,
+    const int32_t* __restrict__ union_ptr, const int32_t* __restrict__ union_pages,
+    const uint64_t* __restrict__ row_mask, const int32_t* __restrict__ n_bundles,
+    const int32_t* __restrict__ bundle_ptr, const int32_t* __restrict__ bundle_groups,
+    const int32_t* __restrict__ ws_usize, const int32_t* __restrict__ ws_wtot, int32_t* __restrict__ bunion_ptr,
+    int32_t* __restrict__ bunion_pages, uint32_t* __restrict__ bunion_mask, int32_t* __restrict__ bundle_qid,
+    long long cap, int64_t* __restrict__ bcounters, unsigned* err) {
+    extern __shared__ uint32_t sm_be[];
+    __shared__ long long red[8];
+    __shared__ long long s_base;
+    __shared__ int goff[257];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w = blockIdx.x, h = blockIdx.y;
+    const int f = h * nwin + w;
+    const int MQ = 128 / g;
+    long long s = 0;
+    for (int x = threadIdx.x; x < f; x += blockDim.x) s += ws_wtot[x];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[warp] = s;
+    __syncthreads();
+    const int nb = n_bundles[h];
+    const int bbase = w * (WB / slots);
+    const int nbw = max(0, min(WB / slots, nb - bbase));
+    if (threadIdx.x == 0) {
+        long long b = 0;
+        for (int x = 0; x < 8; ++x) b += red[x];
+        s_base = b;
+        int o = 0;
+        for (int k = 0; k < nbw; ++k) {
+            goff[k] = o;
+            bunion_ptr[(size_t)h * (Nq + 1) + bbase + k] = (int32_t)(b + o);
+            o += ws_usize[(size_t)h * Nq + bbase + k];
+        }
+        goff[nbw] = o;
+        if (bbase + nbw == nb && (nbw > 0 || w == 0)) bunion_ptr[(size_t)h * (Nq + 1) + nb] = (int32_t)(b + o);
+        if (b + o > cap) atomicOr(err, QUP_ERR_CAPACITY);
+        if (o > 0) atomicAdd(reinterpret_cast<unsigned long long*>(&bcounters[h * 2]), (unsigned long long)o);
+    }
+    __syncthreads();
+    const long long base = s_base;
+    if (nbw == 0 || base + goff[nbw] > cap) return;
+    uint32_t* Uw = sm_be + warp * NW;
+    for (int k = warp; k < nbw; k += 8) {
+        const int bi = bbase + k;
+        const int q0 = bundle_ptr[(size_t)h * (Nq + 1) + bi];
+        const int cnt = bundle_ptr[(size_t)h * (Nq + 1) + bi + 1] - q0;
+        // row -> query table
+        int32_t* qt = bundle_qid + ((size_t)h * Nq + bi) * MQ;
+        for (int x = lane; x < MQ; x += 32) qt[x] = -1;
+        __syncwarp();
+        for (int j = 0; j < cnt; ++j) {
+            const int gj = bundle_groups[(size_t)h * Nq + q0 + j];
+            const int m0 = group_ptr[(size_t)h * (Nq + 1) + gj], m1 = group_ptr[(size_t)h * (Nq + 1) + gj + 1];
+            for (int m = lane; m < m1 - m0; m += 32) qt[j * (RS / g) + m] = members[(size_t)h * Nq + m0 + m];
+        }
+        // merged union bitset
+        for (int wd = lane; wd < NW; wd += 32) {
+            uint32_t u = 0;
+            for (int j = 0; j < cnt; ++j)
+                u |= gbits[((size_t)h * Nq + bundle_groups[(size_t)h * Nq + q0 + j]) * NW + wd];
+            Uw[wd] = u;
+        }
+        __syncwarp();
+        const int wpl = (NW + 31) >> 5;
+        const int wb = min(NW, lane * wpl), we = min(NW, wb + wpl);
+        int c = 0;
+        for (int wd = wb; wd < we; ++wd) c += __popc(Uw[wd]);
+        int incl = c;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const long long out0 = base + goff[k] + (incl - c);
+        // pages, zeroed masks
+        {
+            long long e = out0;
+            for (int wd = wb; wd < we; ++wd) {
+                uint32_t word = Uw[wd];
+                while (word) {
+                    const int b = __ffs(word) - 1;
+                    word &= word - 1;
+                    bunion_pages[e] = wd * 32 + b;
+                    bunion_mask[e * 4 + 0] = bunion_mask[e * 4 + 1] = bunion_mask[e * 4 + 2] =
+                        bunion_mask[e * 4 + 3] = 0u;
+                    ++e;
+                }
+            }
+        }
+        // each slot's row masks: walk the group's sorted union alongside this lane's pages
+        for (int j = 0; j < cnt; ++j) {
+            const int gj = bundle_groups[(size_t)h * Nq + q0 + j];
+            const int u0 = union_ptr[(size_t)h * (Nq + 1) + gj], u1 = union_ptr[(size_t)h * (Nq + 1) + gj + 1];
+            int lo = u0, hi = u1;  // first entry with page >= 32 * wb
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (union_pages[mid] < wb * 32) lo = mid + 1;
+                else hi = mid;
+            }
+            int kk = lo;
+            long long e = out0;
+            const int bit0 = j * RS;
+            for (int wd = wb; wd < we; ++wd) {
+                uint32_t word = Uw[wd];
+                while (word) {
+                    const int b = __ffs(word) - 1;
+                    word &= word - 1;
+                    const int pg = wd * 32 + b;
+                    while (kk < u1 && union_pages[kk] < pg) ++kk;
+                    if (kk < u1 && union_pages[kk] == pg) {
+                        const uint32_t mk = (uint32_t)row_mask[kk] & (RS == 32 ? 0xffffffffu : ((1u << RS) - 1u));
+                        bunion_mask[e * 4 + (bit0 >> 5)] |= mk << (bit0 & 31);
+                    }
+                    ++e;
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
 size_t group_greedy_smem(int W, int NW) {
     const int NWp = NW | 1;
     return sizeof(uint32_t) * ((size_t)W * NWp + NWp + W);
@@ -303,13 +484,46 @@ cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
     grp_rowbits_kernel<<<grid1, 256, sm1, stream>>>(a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW,
                                                    a.rowbits, a.counters, a.err);
     const dim3 grid2(a.nwin, a.Hkv);
-    grp_greedy_kernel<<<grid2, 128, sm2, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
-                                                   a.nwin, a.group_ptr, a.members, a.n_groups, a.ws_usize,
-                                                   a.ws_wtot, a.ws_wcnt);
+    grp_greedy_kernel<<<grid2, 128, sm2, stream>>>(a.rowbits, a.Hq / a.Hkv, a.Hkv, a.Nq, nullptr, a.NW,
+                                                   a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
+                                                   a.ws_usize, a.ws_wtot, a.ws_wcnt, nullptr);
     grp_emit_kernel<<<grid2, 256, sm1, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
                                                  a.nwin, a.group_ptr, a.members, a.ws_usize, a.ws_wtot,
                                                  a.ws_wcnt, a.union_ptr, a.union_pages, a.row_mask, a.cap,
                                                  a.counters, a.err);
+    return cudaGetLastError();
+}
+
+}  // namespace qup
+
+namespace qup {
+
+cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream) {
+    const size_t smw = sizeof(uint32_t) * 8 * (size_t)a.NW;
+    const size_t smg = group_greedy_smem(a.WB, a.NW);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(bnd_gbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(grp_greedy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bnd_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw)) !=
+        cudaSuccess)
+        return e;
+    const long long items = (long long)a.Hkv * a.Nq;
+    const int grid1 = (int)std::min<long long>((items + 7) / 8, (long long)a.sms * 8);
+    bnd_gbits_kernel<<<grid1, 256, smw, stream>>>(a.n_groups, a.union_ptr, a.union_pages, a.Hkv, a.Nq, a.P, a.NW,
+                                                  a.gbits, a.bcounters, a.err);
+    const dim3 grid2(a.nwin, a.Hkv);
+    grp_greedy_kernel<<<grid2, 128, smg, stream>>>(a.gbits, 1, a.Hkv, a.Nq, a.n_groups, a.NW, a.slots, a.WB,
+                                                   a.nwin, a.bundle_ptr, a.bundle_groups, a.n_bundles, a.ws_usize,
+                                                   a.ws_wtot, a.ws_wcnt, a.bcounters);
+    bnd_emit_kernel<<<grid2, 256, smw, stream>>>(a.gbits, a.Hkv, a.Nq, a.NW, a.g, a.RS, a.slots, a.WB, a.nwin,
+                                                 a.group_ptr, a.members, a.union_ptr, a.union_pages, a.row_mask,
+                                                 a.n_bundles, a.bundle_ptr, a.bundle_groups, a.ws_usize, a.ws_wtot,
+                                                 a.bunion_ptr, a.bunion_pages, a.bunion_mask, a.bundle_qid, a.cap,
+                                                 a.bcounters, a.err);
     return cudaGetLastError();
 }
 

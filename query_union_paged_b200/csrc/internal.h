@@ -17,28 +17,27 @@ struct AttnParams {
     const float* k_scale;
     const float* v_scale;
     const int32_t* page_table;
-    const int32_t* n_groups;
-    const int32_t* group_ptr;
-    const int32_t* members;
-    const int32_t* union_ptr;
-    const int32_t* union_pages;
-    const uint64_t* row_mask;
+    const int32_t* n_bundles;    // [Hkv]
+    const int32_t* union_ptr;    // bundle unions: [Hkv][Nq+1] absolute offsets
+    const int32_t* union_pages;  // [cap]
+    const uint32_t* row_mask;    // [cap][4] 128-bit row masks
+    const int32_t* bundle_qid;   // [Hkv][Nq][128/g]
     const int32_t* q_pos;
     void* O;
     float* lse;
     unsigned* err;
     long long cap_union;
-    int num_logical_pages, P_phys, T, kv_len, Hq, Hkv, Nq, g, max_members;
+    int num_logical_pages, P_phys, T, kv_len, Hq, Hkv, Nq, g;
     float scale_log2;  // softmax_scale * log2(e)
     int n_stages;
     unsigned long long wait_limit_ns;
     int dbg_skip_stage;
 };
 
-// dynamic shared memory of the attention kernel for (element size, padded rows, stages, KV heads)
-size_t attn_smem_bytes(int es, int r_pad, int n_stages, int Hkv);
+// dynamic shared memory of the attention kernel for (element size, step tokens, stages, KV heads)
+size_t attn_smem_bytes(int es, int st, int n_stages, int Hkv);
 
-cudaError_t launch_union_attn(int es, int r_pad, const CUtensorMap& tmK, const CUtensorMap& tmV,
+cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);
 
 struct GroupLaunch {
@@ -62,5 +61,32 @@ struct GroupLaunch {
 
 size_t group_greedy_smem(int W, int NW);
 cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream);
+
+struct BundleLaunch {
+    int Hkv, Nq, P, NW, g, RS, slots, WB, nwin;
+    const int32_t* n_groups;
+    const int32_t* group_ptr;
+    const int32_t* members;
+    const int32_t* union_ptr;
+    const int32_t* union_pages;
+    const uint64_t* row_mask;
+    uint32_t* gbits;
+    int32_t* ws_usize;
+    int32_t* ws_wtot;
+    int32_t* ws_wcnt;
+    int32_t* n_bundles;
+    int32_t* bundle_ptr;
+    int32_t* bundle_groups;
+    int32_t* bunion_ptr;
+    int32_t* bunion_pages;
+    uint32_t* bunion_mask;
+    int32_t* bundle_qid;
+    long long cap;
+    int64_t* bcounters;
+    unsigned* err;
+    int sms;
+};
+
+cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream);
 
 }  // namespace qup

@@ -1,40 +1,36 @@
 // union_attn.cu -- ID-aware union attention for sm_100a (PageWeaver,
 // Abstract; Figure 1; Figure 3), re-designed for tcgen05 + TMEM.
 //
-// One persistent CTA per SM walks (KV head, group) work items.  A group has
-// R = members * g query rows (g = Hq / Hkv), at most 32, which is far below
-// the M = 128 rows of a tcgen05 MMA, so the two products are computed
-// transposed, with the page tokens on the M side:
-//      S^T[t][r] = sum_d K[t][d] Q[r][d]          M = 128 tokens, N = R_pad, K = d
-//      O^T[d][r] += sum_t V^T[d][t] P^T[t][r]     M = d = 128,    N = R_pad, K = 128 tokens
-// A pipeline step covers 128 consecutive union tokens (128 / T union pages).
-// Both accumulators live in TMEM: two S^T buffers (double-buffered so the QK^T
-// of step s+1 overlaps the softmax of step s) and one O^T.
+// Work item: a bundle of up to 128 query rows (up to 128 / rows_per_group
+// page-affine groups of one KV head, see qup_groups).  Pages of the bundle
+// union are streamed once per bundle, one step = ST tokens (one page when
+// T >= 64, else 64 / T pages), through an NS-slot TMA ring.  Per step g:
+//      S_b  = Q K^T     M = 128 rows, N = ST tokens, K = d      (smem x smem -> TMEM)
+//      P    = masked online softmax of S_b, written back over S_b in TMEM
+//      O_b += P V       M = 128 rows, N = d, K = ST tokens      (TMEM x smem -> TMEM)
+// with b = g & 1.  The two softmax warpgroups ping-pong: warpgroup b owns the
+// steps of parity b, with its own S buffer, running max, row sum and O
+// accumulator, so the softmax of one step overlaps the next; the epilogue
+// merges the two partial results.  A thread owns one query row, so the row
+// max and the row sum never leave the thread.  A row's max is only raised
+// when a score exceeds it by more than kTau (log2 units); O and the row sum
+// are rescaled then, which after the first steps is rare.
 //
-// Warp roles (192 threads):
-//   warp 0     producer: loads the union page list, row masks and physical
-//              pages (warp-parallel), then TMA-loads each step's K and V
-//              tiles into an NS-slot shared-memory ring (Figure 3's KV slots,
-//              with mbarrier "ready" and "released" events).
-//   warp 1     MMA issuer (one thread) and TMEM owner.
-//   warps 2-5  softmax / epilogue (128 threads, thread = one TMEM lane):
-//              gather the members' Q rows by original ID into the swizzled
-//              Q operand tile, then per step read S^T, apply the row mask
-//              (bit r of the union page's mask), the causal mask
-//              (pos(t) <= q_pos) and t < kv_len, run the fp32 online softmax
-//              (the column max is a warp transpose-reduce plus a 4-warp
-//              exchange), rescale O^T in TMEM when a row max grows, and
-//              write P^T into the MN-major P operand tile.  The epilogue
-//              divides by the row sums and writes each row to O[qid][h'].
+// Warp roles (320 threads):
+//   warps 0-7  softmax / epilogue: warpgroup b = warps 4b..4b+3, thread =
+//              TMEM lane = bundle row.  They also gather the rows of Q by
+//              original query ID (no reordered Q tensor) at bundle start.
+//   warp 8     producer: loads the bundle's page list, row masks and
+//              physical pages (warp-parallel) and TMA-loads K and V pages.
+//   warp 9     MMA issuer (one thread) and TMEM owner (512 columns: S0, S1,
+//              O_0, O_1, 128 each).
+// Operand types: bf16 (kind::f16), fp32 (kind::tf32), FP8 E4M3 (kind::f8f6f4:
+// K and V straight from the cache, Q quantised per row with its own scale,
+// P stored as E4M3 of 64 * p).  Every MMA consumes 32 bytes of its K extent
+// per row, so the descriptor arithmetic is shared by the three types.
 //
-// Operand element types: bf16 (kind::f16), fp32 (kind::tf32) and FP8 E4M3
-// (kind::f8f6f4: K and V straight from the cache; Q is quantised per row
-// with its own scale, P is stored as E4M3 of 256 * p).  Every MMA consumes 32
-// bytes of its K extent per row, so the descriptor arithmetic is the same for
-// all three.
-//
-// Every wait is bounded (ptx.cuh: mbar_wait); on a timeout the CTA raises an
-// abort flag, drains its in-flight TMA loads and MMAs, frees TMEM and exits.
+// Every wait is bounded (ptx.cuh); on a timeout the CTA raises an abort flag,
+// drains its in-flight TMA loads and MMAs, frees TMEM and exits.
 #include <cstdint>
 #include <cuda.h>
 
@@ -44,179 +40,138 @@
 
 namespace qup {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kRows = 128;
 constexpr int kD = kHeadDim;
-constexpr int kTmemCols = 128;  // S^T buffers at columns [0,32) and [32,64), O^T at [64,96)
+constexpr int kTmemCols = 512;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 
 struct StageMeta {
-    int32_t upage[kMaxPPS];
-    uint64_t mask[kMaxPPS];
+    int32_t upage[4];
+    uint32_t mask[4][4];
 };
 
-template <int ES>
+template <int ES, int T>
 struct Geo {
-    static constexpr int kTile = kStepTok * kD * ES;  // one K or V tile of a step
+    static constexpr int ST = T < 64 ? 64 : T;          // tokens per step
+    static constexpr int PPS = ST / T;                  // pages per step
+    static constexpr int kTile = ST * kD * ES;          // one K or V tile of a step
     static constexpr int kStage = 2 * kTile;
-    static constexpr int kChunkElems = 128 / ES;      // elements per 128-byte swizzle row
-    static constexpr int kNChunk = kD * ES / 128;     // 128-byte chunks along d
-    static constexpr int kChunkBytes = kStepTok * 128;  // one chunk column of a tile
-    static constexpr int kMmaK = 32 / ES;             // K elements per MMA instruction
-    static constexpr int kNumMma = kD * ES / 32;      // MMAs per S^T (K = d) and per PV (K = 128 tokens)
+    static constexpr int kChunkElems = 128 / ES;        // elements per 128-byte swizzle row
+    static constexpr int kNChunk = kD * ES / 128;       // 128-byte chunks along d
+    static constexpr int kChunkBytes = ST * 128;        // one chunk column of a K or V tile
+    static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of the Q tile
+    static constexpr int kMmaK = 32 / ES;               // K elements per MMA instruction
+    static constexpr int kNumMmaS = kD * ES / 32;       // MMAs per S (K = d)
+    static constexpr int kNumMmaPV = ST * ES / 32;      // MMAs per O update (K = ST tokens)
+    static constexpr int kPCols = ST * ES / 4;          // TMEM columns of P
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
+    static constexpr float kTau = ES == 1 ? 2.f : 8.f;      // lazy-rescale margin (log2 units)
+    static constexpr float kPScale = ES == 1 ? 64.f : 1.f;  // E4M3 P = 64 p, p <= 2^kTau
 };
 
 struct SmemLayout {
-    uint32_t stages, q, p, bars, meta, red, bc, qsc, misc;
-    uint32_t total;
+    uint32_t stages, q, bars, meta, xch, qsc, misc, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int es, int r_pad, int n_stages, int Hkv) {
+__host__ __device__ inline SmemLayout smem_layout(int es, int st, int n_stages, int Hkv) {
     SmemLayout L;
     uint32_t off = 0;
     L.stages = off;
-    off += (uint32_t)n_stages * 2u * kStepTok * kD * es;
+    off += (uint32_t)n_stages * 2u * st * kD * es;
     L.q = off;
-    off += (uint32_t)r_pad * kD * es;
-    off = (off + 1023u) & ~1023u;
-    L.p = off;
-    off += (uint32_t)kStepTok * r_pad * es;
-    off = (off + 1023u) & ~1023u;
+    off += (uint32_t)kRows * kD * es;
     L.bars = off;
-    off += 8u * (2u * n_stages + 8u);
+    off += 8u * (2u * n_stages + 10u);
     L.meta = off;
     off += (uint32_t)sizeof(StageMeta) * n_stages;
-    L.red = off;
-    off += 2u * 4u * 32u * 4u;
-    L.bc = off;
-    off += 4u * 2u * 32u * 4u;
+    L.xch = off;
+    off += 2u * kRows * 2u * 4u;
     L.qsc = off;
-    off += 32u * 4u;
+    off += kRows * 4u;
     L.misc = off;
     off += 16u + 4u * (uint32_t)(Hkv + 1);
     L.total = off + 1024u;  // slack for aligning the dynamic base to 1024
     return L;
 }
 
-// barrier indices inside the barrier block
+// barrier block
 __device__ __forceinline__ uint32_t bar_full(uint32_t b, int s) { return b + 8u * s; }
 __device__ __forceinline__ uint32_t bar_empty(uint32_t b, int s, int ns) { return b + 8u * (ns + s); }
 __device__ __forceinline__ uint32_t bar_sfull(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + i); }
-__device__ __forceinline__ uint32_t bar_sfree(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 2 + i); }
-__device__ __forceinline__ uint32_t bar_pfull(uint32_t b, int ns) { return b + 8u * (2 * ns + 4); }
-__device__ __forceinline__ uint32_t bar_pvdone(uint32_t b, int ns) { return b + 8u * (2 * ns + 5); }
+__device__ __forceinline__ uint32_t bar_pfull(uint32_t b, int w, int ns) { return b + 8u * (2 * ns + 2 + w); }
+__device__ __forceinline__ uint32_t bar_pvdone(uint32_t b, int w, int ns) { return b + 8u * (2 * ns + 4 + w); }
 __device__ __forceinline__ uint32_t bar_qfull(uint32_t b, int ns) { return b + 8u * (2 * ns + 6); }
 __device__ __forceinline__ uint32_t bar_drain(uint32_t b, int ns) { return b + 8u * (2 * ns + 7); }
 
 struct Item {
-    int h, nm, ub, nU, nsteps, gp0;
+    int h, bi, ub, nU, nsteps;
     bool ok;
 };
 
-// Decode flat work item f; every role calls this and reaches the same verdict.
-__device__ __forceinline__ Item load_item(const AttnParams& p, const int* ng_prefix, int f) {
+// Decode flat bundle f; every role calls this and reaches the same verdict.
+__device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_prefix, int f, int pps) {
     Item it;
     int h = 0;
-    while (h + 1 < p.Hkv && ng_prefix[h + 1] <= f) ++h;
-    const int gi = f - ng_prefix[h];
-    const size_t gp = (size_t)h * (p.Nq + 1) + gi;
+    while (h + 1 < p.Hkv && nb_prefix[h + 1] <= f) ++h;
     it.h = h;
-    it.gp0 = p.group_ptr[gp];
-    it.nm = p.group_ptr[gp + 1] - it.gp0;
-    it.ub = p.union_ptr[gp];
-    it.nU = p.union_ptr[gp + 1] - it.ub;
-    const int pps = kStepTok / p.T;
-    it.ok = it.nm >= 1 && it.nm <= p.max_members && it.gp0 >= 0 && it.gp0 + it.nm <= p.Nq &&
-            it.ub >= 0 && it.nU >= 0 && (long long)it.ub + it.nU <= p.cap_union;
+    it.bi = f - nb_prefix[h];
+    const size_t bp = (size_t)h * (p.Nq + 1) + it.bi;
+    it.ub = p.union_ptr[bp];
+    it.nU = p.union_ptr[bp + 1] - it.ub;
+    it.ok = it.ub >= 0 && it.nU >= 0 && (long long)it.ub + it.nU <= p.cap_union;
     if (!it.ok) it.nU = 0;
-    it.nsteps = it.ok ? (it.nU + pps - 1) / pps : 0;
+    it.nsteps = (it.nU + pps - 1) / pps;
     return it;
 }
 
-// byte offset of 16-byte chunk c of row r inside a K-major SW128 operand tile with `rows` rows
+// byte offset of 16-byte chunk c of row r inside a K-major SW128 operand tile of `rows` rows
 __device__ __forceinline__ uint32_t kmajor_sw128(int r, int c, int rows) {
     return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// swizzle the byte offset of an MN-major P tile (row = token, rowbytes = 32/64/128):
-// 16-byte units XOR the row bits (32/64/128-byte swizzle), or for 32-bit (tf32)
-// operands, whose only MN-major layout is the 128-byte swizzle with 32-byte
-// atoms, 32-byte units XOR (row & 3).
-template <int ES>
-__device__ __forceinline__ uint32_t swz_off(uint32_t off, uint32_t mask) {
-    if constexpr (ES == 4) return off ^ (((off >> 7) & 3u) << 5);
-    else return off ^ (((off >> 7) & mask) << 4);
-}
-
-// After this, lane r of the warp holds the max (or sum) over the warp's 32
-// lanes of column r of v (RP = 32 columns), or of column r & 15 (RP = 16).
-// A recursive-halving transpose: 31 shuffles instead of 32 x 5.
-template <int RP, bool MAX>
-__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
-    auto op = [](float a, float b) { return MAX ? fmaxf(a, b) : a + b; };
-    if constexpr (RP == 32) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const bool up = lane & 16;
-            const float send = up ? v[i] : v[i + 16];
-            const float keep = up ? v[i + 16] : v[i];
-            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = op(v[i], __shfl_xor_sync(0xffffffffu, v[i], 16));
-    }
-#pragma unroll
-    for (int s = 8; s >= 1; s >>= 1) {
-#pragma unroll
-        for (int i = 0; i < s; ++i) {
-            const bool up = lane & s;
-            const float send = up ? v[i] : v[i + s];
-            const float keep = up ? v[i + s] : v[i];
-            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, s));
-        }
-    }
-}
-
-template <int RP>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[32]) {
-    if constexpr (RP == 32) {
-        tmem_ld32(taddr, v);
-    } else {
-        tmem_ld16(taddr, v);
-#pragma unroll
-        for (int r = 16; r < 32; ++r) v[r] = 0u;
-    }
-}
-
-template <int RP>
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[32]) {
-    if constexpr (RP == 32) tmem_st32(taddr, v);
-    else tmem_st16(taddr, v);
-}
-
-// every lane agrees: a failed wait anywhere in the warp fails the warp
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-template <int ES, int RP>
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* v) {
+    static_assert(N % 32 == 0, "loads come in 32-column pieces");
+#pragma unroll
+    for (int i = 0; i < N / 32; ++i) tmem_ld32(taddr + 32u * i, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * i));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
+    if constexpr (N == 8) {
+        tmem_st_x8(taddr, v);
+    } else if constexpr (N == 16) {
+        tmem_st_x16(taddr, v);
+    } else {
+        static_assert(N % 32 == 0, "stores come in 8, 16 or 32-column pieces");
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) tmem_st_x32(taddr + 32u * i, v + 32 * i);
+    }
+}
+
+template <int ES, int T>
 __global__ void __launch_bounds__(kThreads, 1)
     union_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ AttnParams p) {
-    using G = Geo<ES>;
+    using G = Geo<ES, T>;
+    constexpr int ST = G::ST, PPS = G::PPS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(ES, RP, p.n_stages, p.Hkv);
+    const SmemLayout L = smem_layout(ES, ST, p.n_stages, p.Hkv);
     const int NS = p.n_stages;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bars = sbase + L.bars;
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L.meta);
-    float* red = reinterpret_cast<float*>(smem + L.red);
-    float* bc = reinterpret_cast<float*>(smem + L.bc);
+    float* xch = reinterpret_cast<float*>(smem + L.xch);
     float* qsc = reinterpret_cast<float*>(smem + L.qsc);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
-    int* ng_prefix = reinterpret_cast<int*>(smem + L.misc + 16);
+    int* nb_prefix = reinterpret_cast<int*>(smem + L.misc + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t lim = p.wait_limit_ns;
 
@@ -228,62 +183,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_sfull(bars, i, NS), 1);
-            mbar_init(bar_sfree(bars, i, NS), 128);
+            mbar_init(bar_pfull(bars, i, NS), 128);
+            mbar_init(bar_pvdone(bars, i, NS), 1);
         }
-        mbar_init(bar_pfull(bars, NS), 128);
-        mbar_init(bar_pvdone(bars, NS), 1);
-        mbar_init(bar_qfull(bars, NS), 128);
+        mbar_init(bar_qfull(bars, NS), 256);
         mbar_init(bar_drain(bars, NS), 1);
         fence_mbar_init();
         *abort_flag = 0;
         int acc = 0;
         for (int h = 0; h < p.Hkv; ++h) {
-            ng_prefix[h] = acc;
-            int n = p.n_groups[h];
+            nb_prefix[h] = acc;
+            int n = p.n_bundles[h];
             if (n < 0 || n > p.Nq) {
                 atomicOr(p.err, QUP_ERR_GROUP);
                 n = 0;
             }
             acc += n;
         }
-        ng_prefix[p.Hkv] = acc;
+        nb_prefix[p.Hkv] = acc;
     }
-    if (threadIdx.x == 32) {
+    if (threadIdx.x == kProducerWarp * 32) {
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
     }
-    // Q and P operand tiles start zeroed: rows past a group's R must hold finite values
-    for (uint32_t o = threadIdx.x * 16u; o < L.bars - L.q; o += kThreads * 16u)
-        *reinterpret_cast<uint4*>(smem + L.q + o) = make_uint4(0, 0, 0, 0);
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
         tmem_relinquish();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_items = ng_prefix[p.Hkv];
-    const int pps = kStepTok / p.T;
+    const int n_items = nb_prefix[p.Hkv];
 
-    if (warp == 0) {
+    if (warp == kProducerWarp) {
         // ============================================================ producer (whole warp)
         int gs = 0;
-        int last_issue[kMaxStages];
-#pragma unroll
-        for (int s = 0; s < kMaxStages; ++s) last_issue[s] = -1;
         bool ok = true;
         for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x) {
-            const Item it = load_item(p, ng_prefix, f);
-            const int n_ent = it.nsteps * pps;  // union entries incl. padding of the last step
+            const Item it = load_item(p, nb_prefix, f, PPS);
+            const int n_ent = it.nsteps * PPS;  // union entries incl. padding of the last step
             for (int c0 = 0; c0 < n_ent && ok; c0 += 32) {
                 const int idx = c0 + lane;
-                int u = 0, phys = p.P_phys;  // P_phys: out of the tensor, TMA fills zeros
-                uint64_t mk = 0;
+                int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
+                uint4 mk = make_uint4(0, 0, 0, 0);
                 if (idx < it.nU) {
                     u = p.union_pages[it.ub + idx];
-                    mk = p.row_mask[it.ub + idx];
+                    mk = reinterpret_cast<const uint4*>(p.row_mask)[it.ub + idx];
                     if (u < 0 || u >= p.num_logical_pages) {
                         atomicOr(p.err, QUP_ERR_PAGE_ID);
                         u = 0;
@@ -294,9 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             phys = p.P_phys;
                         }
                     }
-                    if (phys == p.P_phys) mk = 0;
+                    if (phys == p.P_phys) mk = make_uint4(0, 0, 0, 0);
                 }
-                const int steps_here = min(32, n_ent - c0) / pps;
+                const int steps_here = min(32, n_ent - c0) / PPS;
                 for (int sl = 0; sl < steps_here; ++sl, ++gs) {
                     const int slot = gs % NS;
                     int okv = 0;
@@ -305,68 +251,73 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         QUP_ERR_TIMEOUT, lim);
                     ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
                     if (!ok) break;
-                    int up_l[kMaxPPS], ph_l[kMaxPPS];
-                    uint64_t mk_l[kMaxPPS];
+                    const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
+                                                      gs == p.dbg_skip_stage);
+                    int ph[PPS];
 #pragma unroll
-                    for (int q = 0; q < kMaxPPS; ++q) {
-                        const int src = (sl * pps + q) & 31;
-                        up_l[q] = __shfl_sync(0xffffffffu, u, src);
-                        ph_l[q] = __shfl_sync(0xffffffffu, phys, src);
-                        mk_l[q] = __shfl_sync(0xffffffffu, mk, src);
-                    }
-                    if (lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 && gs == p.dbg_skip_stage)) {
-                        StageMeta& m = meta[slot];
-                        for (int q = 0; q < pps; ++q) {
-                            m.upage[q] = up_l[q];
-                            m.mask[q] = mk_l[q];
+                    for (int q = 0; q < PPS; ++q) {
+                        const int src = (sl * PPS + q) & 31;
+                        const int uq = __shfl_sync(0xffffffffu, u, src);
+                        ph[q] = __shfl_sync(0xffffffffu, phys, src);
+                        const uint32_t m0 = __shfl_sync(0xffffffffu, mk.x, src);
+                        const uint32_t m1 = __shfl_sync(0xffffffffu, mk.y, src);
+                        const uint32_t m2 = __shfl_sync(0xffffffffu, mk.z, src);
+                        const uint32_t m3 = __shfl_sync(0xffffffffu, mk.w, src);
+                        if (issue) {
+                            StageMeta& m = meta[slot];
+                            m.upage[q] = uq;
+                            m.mask[q][0] = m0;
+                            m.mask[q][1] = m1;
+                            m.mask[q][2] = m2;
+                            m.mask[q][3] = m3;
                         }
+                    }
+                    if (issue) {
+                        // the arrive releases the metadata stores; the copies complete the phase
                         const uint32_t fb = bar_full(bars, slot);
                         mbar_arrive_expect_tx(fb, G::kStage);
                         const uint32_t kdst = sbase + L.stages + (uint32_t)slot * G::kStage;
                         const uint32_t vdst = kdst + G::kTile;
-                        for (int q = 0; q < pps; ++q) {
+#pragma unroll
+                        for (int q = 0; q < PPS; ++q) {
 #pragma unroll
                             for (int c = 0; c < G::kNChunk; ++c) {
-                                const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * p.T) * 128u;
-                                tma_load_4d(kdst + off, &tmK, fb, c * G::kChunkElems, 0, it.h, ph_l[q]);
-                                tma_load_4d(vdst + off, &tmV, fb, c * G::kChunkElems, 0, it.h, ph_l[q]);
+                                const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * T) * 128u;
+                                tma_load_4d(kdst + off, &tmK, fb, c * G::kChunkElems, 0, it.h, ph[q]);
+                                tma_load_4d(vdst + off, &tmV, fb, c * G::kChunkElems, 0, it.h, ph[q]);
                             }
                         }
-                        last_issue[slot] = gs;
                     }
                     __syncwarp();
                 }
             }
         }
-        // every issued load lands before the CTA may exit
+        // every issued load lands before the CTA may exit: the last NS stages
         if (lane == 0) {
-            for (int s = 0; s < NS; ++s)
-                if (last_issue[s] >= 0) mbar_wait_drain(bar_full(bars, s), (last_issue[s] / NS) & 1, lim);
+            for (int i = max(0, gs - NS); i < gs; ++i) {
+                if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
+                mbar_wait_drain(bar_full(bars, i % NS), (i / NS) & 1, lim);
+            }
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer (one thread)
         if (lane == 0) {
-            constexpr uint32_t prow = (uint32_t)RP * ES;  // P row bytes: 32, 64 or 128
-            // MN-major operands: 128/64/32-byte swizzle with 8-row atoms; tf32 needs the
-            // 128-byte swizzle with 32-byte atoms (layout 1), whose atoms are 4 rows
-            constexpr uint32_t playout = ES == 4 ? 1u : (prow == 128 ? 2u : (prow == 64 ? 4u : 6u));
-            constexpr uint32_t psbo = ES == 4 ? 4 * prow : 8 * prow;
+            const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, ST, kRows);
+            const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
+            // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
+            // has only the 128-byte swizzle with 32-byte atoms (layout 1, 4-row atoms)
             constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
             constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
-            const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, RP, 128);
-            const uint32_t idesc_o = instr_desc(G::kFmt, 1, 1, RP, 128);
-            const uint32_t qbase = sbase + L.q, pbase = sbase + L.p;
+            const uint32_t qbase = sbase + L.q;
+            const bool pv_first = NS == 1;  // one slot: O(g-1) must free it before S(g) can load
             int gs = 0, item_no = 0;
             bool ok = true;
             for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x, ++item_no) {
-                const Item it = load_item(p, ng_prefix, f);
+                const Item it = load_item(p, nb_prefix, f, PPS);
                 ok = mbar_wait(bar_qfull(bars, NS), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
                 if (!ok) break;
                 tc_fence_after();
-                // S(s) is issued before PV(s-1) so QK^T overlaps the softmax; with a
-                // single ring stage S(s) needs the slot PV(s-1) frees, so PV goes first
-                const bool pv_first = NS == 1;
                 for (int s = 0; s <= it.nsteps && ok; ++s) {
                     for (int half = 0; half < 2 && ok; ++half) {
                         const bool do_s = (half == (pv_first ? 1 : 0)) && s < it.nsteps;
@@ -374,39 +325,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (do_s) {
                             const int g = gs + s, slot = g % NS, b = g & 1;
                             ok = mbar_wait(bar_full(bars, slot), (g / NS) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
-                                           lim) &&
-                                 mbar_wait(bar_sfree(bars, b, NS), ((g >> 1) & 1) ^ 1, abort_flag, p.err,
-                                           QUP_ERR_TIMEOUT, lim);
+                                           lim);
+                            // S_b last held P(g-2), read by the O_b update of step g-2
+                            if (ok && g >= 2)
+                                ok = mbar_wait(bar_pvdone(bars, b, NS), ((g - 2) >> 1) & 1, abort_flag, p.err,
+                                               QUP_ERR_TIMEOUT, lim);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t kbase = sbase + L.stages + (uint32_t)slot * G::kStage;
 #pragma unroll
-                            for (int k = 0; k < G::kNumMma; ++k) {
+                            for (int k = 0; k < G::kNumMmaS; ++k) {
                                 const uint32_t koff = (uint32_t)(k >> 2) * G::kChunkBytes + (uint32_t)(k & 3) * 32u;
-                                const uint32_t qoff = (uint32_t)(k >> 2) * (RP * 128u) + (uint32_t)(k & 3) * 32u;
-                                tc_mma<G::kKind>(tmem + (uint32_t)b * 32u, smem_desc(kbase + koff, 16, 1024, 2),
-                                                 smem_desc(qbase + qoff, 16, 1024, 2), idesc_s, k > 0);
+                                const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunkBytes + (uint32_t)(k & 3) * 32u;
+                                tc_mma<G::kKind>(tmem + (uint32_t)b * 128u, smem_desc(qbase + qoff, 16, 1024, 2),
+                                                 smem_desc(kbase + koff, 16, 1024, 2), idesc_s, k > 0);
                             }
                             tc_commit(bar_sfull(bars, b, NS));
                         }
                         if (do_pv) {
-                            const int g = gs + s - 1, slot = g % NS;
-                            ok = mbar_wait(bar_pfull(bars, NS), g & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
+                            const int g = gs + s - 1, slot = g % NS, b = g & 1;
+                            const uint32_t vbase = sbase + L.stages + (uint32_t)slot * G::kStage + G::kTile;
+                            ok = mbar_wait(bar_pfull(bars, b, NS), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
+                                           lim);
                             if (!ok) break;
                             tc_fence_after();
-                            const uint32_t vbase = sbase + L.stages + (uint32_t)slot * G::kStage + G::kTile;
+                            // steps 0 and 1 of a bundle open O_0 / O_1 (overwrite)
 #pragma unroll
-                            for (int k = 0; k < G::kNumMma; ++k) {
-                                // K step = kMmaK tokens: kMmaK rows of V (128 B) and of P (prow B)
-                                tc_mma<G::kKind>(tmem + 64u,
-                                                 smem_desc(vbase + (uint32_t)(k * G::kMmaK) * 128u,
-                                                           (uint32_t)G::kChunkBytes, vsbo, vlayout),
-                                                 smem_desc(pbase + (uint32_t)(k * G::kMmaK) * prow, 16 * prow,
-                                                           psbo, playout),
-                                                 idesc_o, (s - 1) > 0 || k > 0);
+                            for (int k = 0; k < G::kNumMmaPV; ++k) {
+                                // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
+                                tc_mma_ts<G::kKind>(tmem + 256u + 128u * b, tmem + (uint32_t)b * 128u + 8u * k,
+                                                    smem_desc(vbase + (uint32_t)(k * G::kMmaK) * 128u,
+                                                              (uint32_t)G::kChunkBytes, vsbo, vlayout),
+                                                    idesc_o, (s - 1) >= 2 || k > 0);
                             }
+                            tc_commit(bar_pvdone(bars, b, NS));
                             tc_commit(bar_empty(bars, slot, NS));
-                            tc_commit(bar_pvdone(bars, NS));
                         }
                     }
                 }
@@ -418,281 +371,259 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ============================================================ softmax / epilogue (128 threads)
-        const int sw = warp - 2;                 // 0..3
-        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-        const int L_tok = quad * 32 + lane;      // step-tile token == S^T lane; O^T lane == feature d
-        const int tid = sw * 32 + lane;
+        // ============================================================ softmax / epilogue (256 threads)
+        const int wg = warp >> 2;            // warpgroup: owns the steps of parity wg
+        const int quad = warp & 3;           // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;      // bundle row == TMEM lane
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const uint32_t s_addr = tmem + lane_base + 128u * wg;        // S_wg / P_wg of this row
+        const uint32_t o_addr = tmem + lane_base + 256u + 128u * wg; // O_wg of this row
         const float kNegInf = -__int_as_float(0x7f800000);
-        constexpr uint32_t prow = (uint32_t)RP * ES;
-        constexpr uint32_t pmask = prow == 128 ? 7u : (prow == 64 ? 3u : 1u);
-        uint8_t* qtile = smem + L.q;
-        uint8_t* ptile = smem + L.p;
-        int gs = 0, xphase = 0;  // xphase alternates the two 4-warp exchange buffers
+        const int g = p.g, MQ = kRows / g;
+        int gs = 0;
         bool ok = true;
         for (int f = blockIdx.x; f < n_items; f += gridDim.x) {
-            const Item it = load_item(p, ng_prefix, f);
-            if (!it.ok && tid == 0) atomicOr(p.err, QUP_ERR_GROUP);
-            // ---- members (lane m holds member m), positions, Q gather by original ID
-            int qid_m = 0, qpos_m = 0;
-            bool mem_ok = true;
-            if (lane < it.nm) {
-                qid_m = p.members[(size_t)it.h * p.Nq + it.gp0 + lane];
-                if (qid_m < 0 || qid_m >= p.Nq) {
-                    mem_ok = false;
-                    qid_m = 0;
-                }
-                qpos_m = p.q_pos[qid_m];
+            const Item it = load_item(p, nb_prefix, f, PPS);
+            if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
+            // ---- this row's query (original ID) and head
+            int qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
+            if (qid >= p.Nq) {
+                atomicOr(p.err, QUP_ERR_GROUP);
+                qid = -1;
             }
-            if (!warp_ok(mem_ok) && tid == 0) atomicOr(p.err, QUP_ERR_GROUP);
-            const int R = it.nm * p.g;
+            const int head = it.h * g + (r % g);
+            const int qpos = qid >= 0 ? p.q_pos[qid] : -1;
+            const int vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
+            // ---- Q row by original ID -> K-major SW128 operand tile
             {
-                constexpr int CPR = 8 * ES;    // 16-byte chunks per Q row in shared memory
-                constexpr int RPP = 128 / CPR;  // rows per pass
-                const int c = tid % CPR;
-#pragma unroll 1
-                for (int r0 = 0; r0 < RP; r0 += RPP) {
-                    const int r = r0 + tid / CPR;
-                    const int m = r / p.g, j = r % p.g;
-                    const int qid = __shfl_sync(0xffffffffu, qid_m, m & 7);
-                    const bool live = r < R;
-                    const size_t row_off = ((size_t)qid * p.Hq + (size_t)it.h * p.g + j) * kD;
-                    uint4 out = make_uint4(0, 0, 0, 0);
-                    if constexpr (ES == 4) {
-                        if (live) out = *reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off + c * 4);
-                    } else if constexpr (ES == 2) {
-                        if (live) out = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off + c * 8);
-                    } else {
-                        // 16 bf16 -> 16 E4M3 with the row's scale amax / 448
-                        float x[16];
+                uint8_t* qt = smem + L.q;
+                const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+                if constexpr (ES == 2) {
+                    const uint4* src =
+                        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off) + wg * 8;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) x[e] = 0.f;
-                        if (live) {
-                            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off + c * 16);
-                            const uint4 a0 = src[0], a1 = src[1];
-                            const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, wg * 8 + c, kRows)) = v;
+                    }
+                } else if constexpr (ES == 4) {
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off) + wg * 16;
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                x[2 * e] = __uint_as_float(w[e] << 16);
-                                x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-                            }
-                        }
+                    for (int c = 0; c < 16; ++c) {
+                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, wg * 16 + c, kRows)) = v;
+                    }
+                } else {
+                    if (wg == 0) {  // whole row: bf16 -> E4M3 with the row's scale amax / 448
+                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
+                        uint4 raw[16];
                         float amax = 0.f;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+                        for (int c = 0; c < 16; ++c) {
+                            raw[c] = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
 #pragma unroll
-                        for (int o = 1; o < CPR; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                            for (int e = 0; e < 4; ++e)
+                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                                         fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+                        }
                         const float inv = amax > 0.f ? 448.f / amax : 0.f;
-                        out.x = pack_e4m3x4(x[0] * inv, x[1] * inv, x[2] * inv, x[3] * inv);
-                        out.y = pack_e4m3x4(x[4] * inv, x[5] * inv, x[6] * inv, x[7] * inv);
-                        out.z = pack_e4m3x4(x[8] * inv, x[9] * inv, x[10] * inv, x[11] * inv);
-                        out.w = pack_e4m3x4(x[12] * inv, x[13] * inv, x[14] * inv, x[15] * inv);
-                        if (c == 0) qsc[r] = amax * (1.f / 448.f);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {  // 16 output bytes from 2 input chunks
+                            float x[16];
+                            const uint32_t w8[8] = {raw[2 * c].x,     raw[2 * c].y,     raw[2 * c].z,     raw[2 * c].w,
+                                                    raw[2 * c + 1].x, raw[2 * c + 1].y, raw[2 * c + 1].z, raw[2 * c + 1].w};
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                x[2 * e] = __uint_as_float(w8[e] << 16) * inv;
+                                x[2 * e + 1] = __uint_as_float(w8[e] & 0xffff0000u) * inv;
+                            }
+                            uint4 o;
+                            o.x = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                            o.y = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                            o.z = pack_e4m3x4(x[8], x[9], x[10], x[11]);
+                            o.w = pack_e4m3x4(x[12], x[13], x[14], x[15]);
+                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = o;
+                        }
+                        qsc[r] = amax * (1.f / 448.f);
                     }
-                    *reinterpret_cast<uint4*>(qtile + kmajor_sw128(r, c, RP)) = out;
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_qfull(bars, NS));
-            // ---- per-row constants: score scale (log2 domain), causal bound, output row
-            float cs[32];
+            float cs = p.scale_log2;  // score scale (log2 domain) of this row
             if constexpr (ES == 1) {
-                bar_sync(1, 128);  // qsc written by the gather
-                const float ks = p.k_scale[it.h] * p.scale_log2;
-#pragma unroll
-                for (int r = 0; r < 32; ++r) cs[r] = (r < RP) ? qsc[r] * ks : 0.f;
-            } else {
-#pragma unroll
-                for (int r = 0; r < 32; ++r) cs[r] = p.scale_log2;
+                bar_sync(1, 256);  // qsc written by warpgroup 0
+                cs = qsc[r] * p.k_scale[it.h] * p.scale_log2;
             }
-            int rpos[32];
-#pragma unroll
-            for (int r = 0; r < 32; ++r) rpos[r] = __shfl_sync(0xffffffffu, qpos_m, (r / p.g) & 7);
-            const uint32_t live_rows = (R >= 32) ? 0xffffffffu : ((1u << R) - 1u);
+            float m_used = kNegInf, lsum = 0.f;
+            int mine_steps = 0;  // steps of this bundle this warpgroup has processed
 
-            float m_lane = kNegInf;  // lane r holds the running max of row r (log2 domain)
-            float lpart[32];         // this thread's token partial of each row's sum
-#pragma unroll
-            for (int r = 0; r < 32; ++r) lpart[r] = 0.f;
-
-            for (int s = 0; s < it.nsteps; ++s, ++gs) {
-                const int slot = gs % NS, b = gs & 1;
+            for (int s = 0; s < it.nsteps; ++s) {
+                const int gstep = gs + s;
+                if ((gstep & 1) != wg) continue;  // the other warpgroup's step
+                const int slot = gstep % NS;
                 if (ok)
-                    ok = mbar_wait(bar_full(bars, slot), (gs / NS) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                         mbar_wait(bar_sfull(bars, b, NS), (gs >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
-                ok = warp_ok(ok);
-                float x[32];
-                if (ok) {
-                    uint32_t sr[32];
-                    tc_fence_after();
-                    tmem_ld_cols<RP>(tmem + lane_base + (uint32_t)b * 32u, sr);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(bar_sfree(bars, b, NS));
-                    const int ps = L_tok / p.T, o = L_tok - ps * p.T;
-                    const int u = meta[slot].upage[ps];
-                    const uint64_t mk = meta[slot].mask[ps];
-                    const int pos = u * p.T + o;
-                    uint32_t valid = (uint32_t)mk & live_rows;
-                    if (s * pps + ps >= it.nU) valid = 0;
-                    if (pos >= p.kv_len) {
-                        valid = 0;
-                        // cache slots past kv_len may hold non-finite bytes: zero this V row
+                    ok = warp_ok(mbar_wait(bar_full(bars, slot), (gstep / NS) & 1, abort_flag, p.err,
+                                           QUP_ERR_TIMEOUT, lim) &&
+                                 mbar_wait(bar_sfull(bars, wg, NS), (gstep >> 1) & 1, abort_flag, p.err,
+                                           QUP_ERR_TIMEOUT, lim));
+                if (!ok) continue;
+                tc_fence_after();
+                uint32_t sv[ST];
+                tmem_ld_n<ST>(s_addr, sv);
+                const StageMeta& mt = meta[slot];
+                // cache slots at or past kv_len may hold non-finite bytes: zero those V rows
+                if (r < ST) {
+                    const int q = r / T;
+                    if (mt.upage[q] * T + (r - q * T) >= p.kv_len) {
                         uint8_t* vt = smem + L.stages + (uint32_t)slot * G::kStage + G::kTile;
+#pragma unroll
                         for (int c = 0; c < G::kNChunk; ++c)
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                *reinterpret_cast<uint4*>(vt + c * G::kChunkBytes + L_tok * 128 + e * 16) =
+                                *reinterpret_cast<uint4*>(vt + c * G::kChunkBytes + r * 128 + e * 16) =
                                     make_uint4(0, 0, 0, 0);
                     }
+                }
+                // row r sees token j of page q iff the page is in its own TopK row
+                // (bit r of the page's mask) and the token's position is < vis_end
+                int lim_q[PPS];
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) {
-                        const bool v = r < RP && ((valid >> r) & 1u) && pos <= rpos[r];
-                        x[r] = v ? __uint_as_float(sr[r]) * cs[r] : kNegInf;
+                for (int q = 0; q < PPS; ++q) {
+                    const bool mine = (mt.mask[q][r >> 5] >> (r & 31)) & 1u;
+                    lim_q[q] = mine ? max(0, min(T, vis_end - mt.upage[q] * T)) : 0;
+                }
+                tmem_wait_ld();
+                float mloc = kNegInf;
+#pragma unroll
+                for (int j = 0; j < ST; ++j) {
+                    const float v = (j % T) < lim_q[j / T] ? __uint_as_float(sv[j]) * cs : kNegInf;
+                    sv[j] = __float_as_uint(v);
+                    mloc = fmaxf(mloc, v);
+                }
+                // lazy running max: raise it only when a score exceeds it by more than kTau
+                const bool need = mloc > m_used + G::kTau;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = ex2(m_used - mloc);  // 0 when m_used is -inf
+                    m_used = mloc;
+                    lsum *= alpha;
+                }
+                const float msafe = m_used == kNegInf ? 0.f : m_used;
+                uint32_t pk[G::kPCols];
+                float part0 = 0.f, part1 = 0.f;
+                if constexpr (ES == 2) {
+#pragma unroll
+                    for (int j = 0; j < ST; j += 2) {
+                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                        const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
+                        part0 += p0;
+                        part1 += p1;
+                        pk[j / 2] = pack_bf16x2(p0, p1);
+                    }
+                } else if constexpr (ES == 4) {
+#pragma unroll
+                    for (int j = 0; j < ST; ++j) {
+                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                        if (j & 1) part1 += p0; else part0 += p0;
+                        pk[j] = __float_as_uint(p0);
                     }
                 } else {
 #pragma unroll
-                    for (int r = 0; r < 32; ++r) x[r] = kNegInf;
+                    for (int j = 0; j < ST; j += 4) {
+                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                        const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
+                        const float p2 = ex2(__uint_as_float(sv[j + 2]) - msafe);
+                        const float p3 = ex2(__uint_as_float(sv[j + 3]) - msafe);
+                        part0 += p0 + p2;
+                        part1 += p1 + p3;
+                        pk[j / 4] = pack_e4m3x4(p0 * G::kPScale, p1 * G::kPScale, p2 * G::kPScale, p3 * G::kPScale);
+                    }
                 }
-                // ---- row max over the step's 128 tokens
-                float v[32];
-#pragma unroll
-                for (int r = 0; r < 32; ++r) v[r] = x[r];
-                transpose_reduce<RP, true>(v, lane);
-                float* rb = red + (xphase & 1) * 128;
-                ++xphase;
-                rb[sw * 32 + lane] = v[0];
-                ok = bar_and(1, 128, ok);
-                if (!ok) break;
-                {
-                    const float mx = fmaxf(fmaxf(rb[lane], rb[32 + lane]), fmaxf(rb[64 + lane], rb[96 + lane]));
-                    const float m_new = fmaxf(m_lane, mx);
-                    const float m_safe = (m_new == kNegInf) ? 0.f : m_new;
-                    const float alpha = ex2(m_lane - m_safe);
-                    m_lane = m_new;
-                    bc[sw * 64 + lane] = m_safe;
-                    bc[sw * 64 + 32 + lane] = alpha;
-                }
-                __syncwarp();
-                float msafe[32], alpha[32];
-#pragma unroll
-                for (int r = 0; r < 32; r += 4) {
-                    const float4 a = *reinterpret_cast<const float4*>(bc + sw * 64 + r);
-                    const float4 c = *reinterpret_cast<const float4*>(bc + sw * 64 + 32 + r);
-                    msafe[r] = a.x; msafe[r + 1] = a.y; msafe[r + 2] = a.z; msafe[r + 3] = a.w;
-                    alpha[r] = c.x; alpha[r + 1] = c.y; alpha[r + 2] = c.z; alpha[r + 3] = c.w;
-                }
-                float pv[32];
-                bool rescale = false;
-#pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    pv[r] = ex2(x[r] - msafe[r]);
-                    lpart[r] = lpart[r] * alpha[r] + pv[r];
-                    if (r < RP) rescale |= alpha[r] != 1.f;
-                }
-                if (s > 0) {
-                    ok = warp_ok(mbar_wait(bar_pvdone(bars, NS), (gs - 1) & 1, abort_flag, p.err,
+                lsum += part0 + part1;
+                // this warpgroup's previous O update must be done before O is rescaled and
+                // before P overwrites S (the MMA of step gstep-2 reads P from the same columns)
+                if (gstep >= 2)
+                    ok = warp_ok(mbar_wait(bar_pvdone(bars, wg, NS), ((gstep - 2) >> 1) & 1, abort_flag, p.err,
                                            QUP_ERR_TIMEOUT, lim));
-                    if (ok) {
-                        tc_fence_after();
-                        if (rescale) {  // uniform: alpha comes from the shared exchange
-                            uint32_t ov[32];
-                            const uint32_t oaddr = tmem + lane_base + 64u;
-                            tmem_ld_cols<RP>(oaddr, ov);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int r = 0; r < 32; ++r)
-                                ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
-                            tmem_st_cols<RP>(oaddr, ov);
-                            tmem_wait_st();
-                        }
-                    }
-                }
-                if (ok) {
-                    // ---- this token's P^T row into the MN-major operand tile
-                    const uint32_t rowoff = (uint32_t)L_tok * prow;
-                    if constexpr (ES == 2) {
-#pragma unroll
-                        for (int c = 0; c < RP / 8; ++c) {
-                            uint4 w;
-                            w.x = pack_bf16x2(pv[c * 8 + 0], pv[c * 8 + 1]);
-                            w.y = pack_bf16x2(pv[c * 8 + 2], pv[c * 8 + 3]);
-                            w.z = pack_bf16x2(pv[c * 8 + 4], pv[c * 8 + 5]);
-                            w.w = pack_bf16x2(pv[c * 8 + 6], pv[c * 8 + 7]);
-                            *reinterpret_cast<uint4*>(ptile + swz_off<ES>(rowoff + c * 16, pmask)) = w;
-                        }
-                    } else if constexpr (ES == 4) {
-#pragma unroll
-                        for (int c = 0; c < RP / 4; ++c) {
-                            const uint4 w = make_uint4(__float_as_uint(pv[c * 4]), __float_as_uint(pv[c * 4 + 1]),
-                                                       __float_as_uint(pv[c * 4 + 2]), __float_as_uint(pv[c * 4 + 3]));
-                            *reinterpret_cast<uint4*>(ptile + swz_off<ES>(rowoff + c * 16, pmask)) = w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < RP / 16; ++c) {
-                            const float* q = pv + c * 16;
-                            uint4 w;
-                            w.x = pack_e4m3x4(q[0] * 256.f, q[1] * 256.f, q[2] * 256.f, q[3] * 256.f);
-                            w.y = pack_e4m3x4(q[4] * 256.f, q[5] * 256.f, q[6] * 256.f, q[7] * 256.f);
-                            w.z = pack_e4m3x4(q[8] * 256.f, q[9] * 256.f, q[10] * 256.f, q[11] * 256.f);
-                            w.w = pack_e4m3x4(q[12] * 256.f, q[13] * 256.f, q[14] * 256.f, q[15] * 256.f);
-                            *reinterpret_cast<uint4*>(ptile + swz_off<ES>(rowoff + c * 16, pmask)) = w;
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(bar_pfull(bars, NS));
-                }
-            }
-            // ---- epilogue: row sums, lse, O^T / l -> O[qid][h*g + j][d]
-            if (ok && it.nsteps > 0)
-                ok = mbar_wait(bar_pvdone(bars, NS), (gs - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
-            ok = warp_ok(ok);
-            transpose_reduce<RP, false>(lpart, lane);
-            float* rb = red + (xphase & 1) * 128;
-            ++xphase;
-            rb[sw * 32 + lane] = lpart[0];
-            ok = bar_and(1, 128, ok);
-            if (!ok) break;
-            {
-                const float l = rb[lane] + rb[32 + lane] + rb[64 + lane] + rb[96 + lane];
-                bc[sw * 64 + lane] = l > 0.f ? 1.f / l : 0.f;
-            }
-            if (p.lse != nullptr && sw == 0) {
-                // m_lane is in the log2 domain (scores * log2 e); lse is a natural log
-                const float l = rb[lane] + rb[32 + lane] + rb[64 + lane] + rb[96 + lane];
-                const int qid = __shfl_sync(0xffffffffu, qid_m, (lane / p.g) & 7);
-                if (lane < R) {
-                    const int j = lane % p.g;
-                    p.lse[(size_t)qid * p.Hq + (size_t)it.h * p.g + j] =
-                        l > 0.f ? (m_lane + __log2f(l)) * 0.69314718055994531f : kNegInf;
-                }
-            }
-            __syncwarp();
-            float vsc = 1.f;
-            if constexpr (ES == 1) vsc = p.v_scale[it.h] * (1.f / 256.f);
-            uint32_t ov[32];
-            if (it.nsteps > 0) {
+                if (!ok) continue;
                 tc_fence_after();
-                tmem_ld_cols<RP>(tmem + lane_base + 64u, ov);
-                tmem_wait_ld();
-            } else {
+                if (mine_steps > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(o_addr + 32u * c, ov);
+                        tmem_wait_ld();
 #pragma unroll
-                for (int r = 0; r < 32; ++r) ov[r] = 0u;
-            }
-#pragma unroll
-            for (int r = 0; r < RP; ++r) {
-                const int qid = __shfl_sync(0xffffffffu, qid_m, (r / p.g) & 7);
-                if (r < R) {
-                    const float val = __uint_as_float(ov[r]) * bc[sw * 64 + r] * vsc;
-                    const size_t oi = ((size_t)qid * p.Hq + (size_t)it.h * p.g + (r % p.g)) * kD + L_tok;
-                    if constexpr (ES == 4) static_cast<float*>(p.O)[oi] = val;
-                    else static_cast<uint16_t*>(p.O)[oi] = (uint16_t)(pack_bf16x2(val, 0.f) & 0xffffu);
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st_x32(o_addr + 32u * c, ov);
+                    }
+                    tmem_wait_st();
                 }
+                tmem_st_n<G::kPCols>(s_addr, pk);
+                tmem_wait_st();
+                fence_proxy_async_smem();  // zeroed V rows -> async proxy
+                tc_fence_before();
+                mbar_arrive(bar_pfull(bars, wg, NS));
+                ++mine_steps;
+            }
+            // ---- epilogue: merge the two partial results; O / l -> O[qid][head][:]
+            if (ok && mine_steps > 0) {
+                int last = gs + it.nsteps - 1;
+                if ((last & 1) != wg) --last;
+                ok = warp_ok(mbar_wait(bar_pvdone(bars, wg, NS), (last >> 1) & 1, abort_flag, p.err,
+                                       QUP_ERR_TIMEOUT, lim));
+            }
+            gs += it.nsteps;
+            xch[(wg * kRows + r) * 2 + 0] = mine_steps > 0 ? m_used : kNegInf;
+            xch[(wg * kRows + r) * 2 + 1] = mine_steps > 0 ? lsum : 0.f;
+            ok = bar_and(1, 256, ok);
+            if (!ok) break;
+            const float m0 = xch[r * 2], l0 = xch[r * 2 + 1];
+            const float m1 = xch[(kRows + r) * 2], l1 = xch[(kRows + r) * 2 + 1];
+            const float M = fmaxf(m0, m1);
+            const float f0 = (m0 == kNegInf) ? 0.f : ex2(m0 - M);
+            const float f1 = (m1 == kNegInf) ? 0.f : ex2(m1 - M);
+            const float Lsum = l0 * f0 + l1 * f1;
+            float vsc = 1.f;
+            if constexpr (ES == 1) vsc = p.v_scale[it.h] * (1.f / G::kPScale);
+            const float inv = Lsum > 0.f ? vsc / Lsum : 0.f;
+            const float g0 = f0 * inv, g1 = f1 * inv;
+            const bool use0 = m0 != kNegInf && Lsum > 0.f, use1 = m1 != kNegInf && Lsum > 0.f;
+            tc_fence_after();
+            // this warpgroup writes features [64 wg, 64 wg + 64) of the row
+            float o[64];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t a[32], e2[32];
+                tmem_ld32(tmem + lane_base + 256u + (uint32_t)(64 * wg + 32 * c), a);
+                tmem_ld32(tmem + lane_base + 384u + (uint32_t)(64 * wg + 32 * c), e2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[32 * c + e] = (use0 ? __uint_as_float(a[e]) * g0 : 0.f) + (use1 ? __uint_as_float(e2[e]) * g1 : 0.f);
+            }
+            if (qid >= 0) {
+                const size_t oi = ((size_t)qid * p.Hq + head) * kD + 64 * wg;
+                if constexpr (ES == 4) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + oi);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(o[8 * e], o[8 * e + 1]), pack_bf16x2(o[8 * e + 2], o[8 * e + 3]),
+                                            pack_bf16x2(o[8 * e + 4], o[8 * e + 5]),
+                                            pack_bf16x2(o[8 * e + 6], o[8 * e + 7]));
+                }
+                if (wg == 0 && p.lse != nullptr)
+                    p.lse[(size_t)qid * p.Hq + head] =
+                        Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : kNegInf;
             }
             tc_fence_before();
+            bar_sync(1, 256);  // O_0 and O_1 read by both halves before the next bundle overwrites them
         }
     }
 
@@ -700,29 +631,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-size_t attn_smem_bytes(int es, int r_pad, int n_stages, int Hkv) {
-    return smem_layout(es, r_pad, n_stages, Hkv).total;
+size_t attn_smem_bytes(int es, int st, int n_stages, int Hkv) {
+    return smem_layout(es, st, n_stages, Hkv).total;
 }
 
-template <int ES, int RP>
+template <int ES, int T>
 static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p, int grid,
                             size_t smem, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(union_attn_kernel<ES, RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(union_attn_kernel<ES, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    union_attn_kernel<ES, RP><<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
+    union_attn_kernel<ES, T><<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_union_attn(int es, int r_pad, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                              const AttnParams& p, int grid, size_t smem, cudaStream_t stream) {
-    if (es == 2 && r_pad == 32) return launch_t<2, 32>(tmK, tmV, p, grid, smem, stream);
-    if (es == 2 && r_pad == 16) return launch_t<2, 16>(tmK, tmV, p, grid, smem, stream);
-    if (es == 4 && r_pad == 32) return launch_t<4, 32>(tmK, tmV, p, grid, smem, stream);
-    if (es == 1 && r_pad == 32) return launch_t<1, 32>(tmK, tmV, p, grid, smem, stream);
+cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p,
+                              int grid, size_t smem, cudaStream_t stream) {
+    if (es == 2 && T == 16) return launch_t<2, 16>(tmK, tmV, p, grid, smem, stream);
+    if (es == 2 && T == 32) return launch_t<2, 32>(tmK, tmV, p, grid, smem, stream);
+    if (es == 2 && T == 64) return launch_t<2, 64>(tmK, tmV, p, grid, smem, stream);
+    if (es == 2 && T == 128) return launch_t<2, 128>(tmK, tmV, p, grid, smem, stream);
+    if (es == 1 && T == 64) return launch_t<1, 64>(tmK, tmV, p, grid, smem, stream);
+    if (es == 1 && T == 128) return launch_t<1, 128>(tmK, tmV, p, grid, smem, stream);
+    if (es == 4 && T == 32) return launch_t<4, 32>(tmK, tmV, p, grid, smem, stream);
+    if (es == 4 && T == 64) return launch_t<4, 64>(tmK, tmV, p, grid, smem, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -28,11 +28,20 @@ def groups_to_host(gr):
     union_ptr = gr.union_ptr.cpu().numpy()
     Hkv = n_groups.size
     total = int(union_ptr[Hkv - 1, n_groups[Hkv - 1]]) if Hkv else 0
-    return dict(n_groups=n_groups, group_ptr=gr.group_ptr.cpu().numpy(),
-                members=gr.members.cpu().numpy(), union_ptr=union_ptr,
-                union_pages=gr.union_pages[:total].cpu().numpy(),
-                row_mask=gr.row_mask[:total].cpu().numpy().view(np.uint64),
-                counters=gr.counters.cpu().numpy())
+    d = dict(n_groups=n_groups, group_ptr=gr.group_ptr.cpu().numpy(),
+             members=gr.members.cpu().numpy(), union_ptr=union_ptr,
+             union_pages=gr.union_pages[:total].cpu().numpy(),
+             row_mask=gr.row_mask[:total].cpu().numpy().view(np.uint64),
+             counters=gr.counters.cpu().numpy())
+    nb = gr.n_bundles.cpu().numpy()
+    bptr = gr.bunion_ptr.cpu().numpy()
+    btotal = int(bptr[Hkv - 1, nb[Hkv - 1]]) if Hkv else 0
+    d.update(n_bundles=nb, bundle_ptr=gr.bundle_ptr.cpu().numpy(),
+             bundle_groups=gr.bundle_groups.cpu().numpy(), bunion_ptr=bptr,
+             bunion_pages=gr.bunion_pages[:btotal].cpu().numpy(),
+             bunion_mask=gr.bunion_mask[:btotal].cpu().numpy().view(np.uint32),
+             bundle_qid=gr.bundle_qid.cpu().numpy(), bcounters=gr.bcounters.cpu().numpy())
+    return d
 
 
 def assert_groups_equal(got, ref):
@@ -47,6 +56,21 @@ def assert_groups_equal(got, ref):
         assert np.array_equal(got["union_ptr"][h, :n + 1], ref["union_ptr"][h, :n + 1])
     assert np.array_equal(got["union_pages"], ref["union_pages"])
     assert np.array_equal(got["row_mask"], ref["row_mask"])
+
+
+def assert_bundles_equal(got, ref):
+    Hkv = ref["n_bundles"].size
+    assert np.array_equal(got["n_bundles"], ref["n_bundles"])
+    assert np.array_equal(got["bcounters"], ref["bcounters"])
+    for h in range(Hkv):
+        n = int(ref["n_bundles"][h])
+        assert np.array_equal(got["bundle_ptr"][h, :n + 1], ref["bundle_ptr"][h, :n + 1])
+        m = int(ref["bundle_ptr"][h, n])
+        assert np.array_equal(got["bundle_groups"][h, :m], ref["bundle_groups"][h, :m])
+        assert np.array_equal(got["bunion_ptr"][h, :n + 1], ref["bunion_ptr"][h, :n + 1])
+        assert np.array_equal(got["bundle_qid"][h, :n], ref["bundle_qid"][h, :n])
+    assert np.array_equal(got["bunion_pages"], ref["bunion_pages"])
+    assert np.array_equal(got["bunion_mask"], ref["bunion_mask"])
 
 
 def out_to_f64(O):

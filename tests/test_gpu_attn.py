@@ -70,7 +70,8 @@ def test_small_full_output_three_groupings(kw):
     mg = w.max_group
     for name, gr in (("online", _gpu_groups(w, dev, mg, w.window)),
                      ("fixed", _gpu_groups(w, dev, mg, mg)),
-                     ("random", qup.Groups.from_host(_perm_groups(w, kw["seed"], mg), "cuda"))):
+                     ("random", qup.groups_from_host(_perm_groups(w, kw["seed"], mg), w.Hq, w.Hkv,
+                                                     w.num_logical_pages, mg))):
         got = out_to_f64(_attn(w, dev, gr))
         check_close(got, ref, w.kv_dtype, f"{w.name}/{name}")
 

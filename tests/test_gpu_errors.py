@@ -36,7 +36,7 @@ def test_bad_group_sets_error_bit():
     w = W.random_small(22)
     dev = to_device(w)
     gr = qup.sparse_group(dev["topk"], w.Hq, w.Hkv, w.num_logical_pages, 8, 64)
-    gr.members[0, 0] = w.Nq + 3
+    gr.bundle_qid[0, 0, 0] = w.Nq + 3
     _call(w, dev, gr)
     assert qup.get_error() & qup.ERR["GROUP"]
 

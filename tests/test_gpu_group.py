@@ -6,7 +6,7 @@ import oracle
 import query_union_paged_b200 as qup
 from query_union_paged_b200 import workloads as W
 
-from helpers import assert_groups_equal, groups_to_host
+from helpers import assert_bundles_equal, assert_groups_equal, groups_to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -35,6 +35,7 @@ def test_random_small_bitexact(seed):
     got = _run(topk, Hkv * g, Hkv, P, max_group, window)
     ref = oracle.group(topk, Hkv * g, Hkv, Nq, P, max_group, window)
     assert_groups_equal(got, ref)
+    assert_bundles_equal(got, oracle.bundle(ref, Hkv * g, Hkv, Nq, max_group))
 
 
 @pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c", "5"])
@@ -44,6 +45,7 @@ def test_workload_bitexact(cfg, window):
     got = _run(w.topk, w.Hq, w.Hkv, w.num_logical_pages, 8, window)
     ref = oracle.group(w.topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, 8, window)
     assert_groups_equal(got, ref)
+    assert_bundles_equal(got, oracle.bundle(ref, w.Hq, w.Hkv, w.Nq, 8))
 
 
 def test_figure2_example_on_gpu():
@@ -61,6 +63,27 @@ def test_max_window_and_large_page_range():
     got = _run(topk, 8, 2, P, 8, 256)
     ref = oracle.group(topk, 8, 2, 600, P, 8, 256)
     assert_groups_equal(got, ref)
+    assert_bundles_equal(got, oracle.bundle(ref, 8, 2, 600, 8))
+
+
+def test_bundles_of_a_given_partition_match_reference():
+    import query_union_paged_b200 as qup
+    rng = np.random.default_rng(9)
+    Hq, Hkv, Nq, P = 8, 2, 150, 90
+    topk = rng.integers(-1, P, size=(Hq, Nq, 7)).astype(np.int32)
+    part = []
+    for _ in range(Hkv):
+        perm = rng.permutation(Nq)
+        groups, i = [], 0
+        while i < Nq:
+            k = int(rng.integers(1, 9))
+            groups.append(sorted(int(x) for x in perm[i:i + k]))
+            i += k
+        part.append(groups)
+    ref = oracle.build_unions(topk, Hq, Hkv, Nq, P, part)
+    gr = qup.groups_from_host(ref, Hq, Hkv, P, 8)
+    assert qup.get_error() == 0
+    assert_bundles_equal(groups_to_host(gr), oracle.bundle(ref, Hq, Hkv, Nq, 8))
 
 
 def test_out_of_range_page_id_sets_error_bit():

@@ -187,3 +187,93 @@ def test_block_union_workload_groups_align_with_query_blocks():
     # every row keeps exactly its own block row, so masked row slots are the
     # union minus each head's row, and members of one block share their support
     assert np.all(out["counters"][:, 2] == 0)
+
+
+# ----------------------------------------------------------- bundles
+
+def py_bundle(out, Hq, Hkv, Nq, max_group, wb=64):
+    """The bundling rule written with Python sets: greedy over group unions."""
+    g = Hq // Hkv
+    rs = 1
+    while rs < max_group * g:
+        rs *= 2
+    slots = 128 // rs
+    wb = max(slots, (wb // slots) * slots)
+    res = []
+    for h in range(Hkv):
+        groups = _groups_of(out, h)
+        bundles = []
+        for w0 in range(0, len(groups), wb):
+            left = list(range(w0, min(len(groups), w0 + wb)))
+            while left:
+                seed = left.pop(0)
+                U, b = set(groups[seed][1]), [seed]
+                while len(b) < slots and left:
+                    c = min(left, key=lambda q: (len(set(groups[q][1]) - U), q))
+                    left.remove(c)
+                    b.append(c)
+                    U |= set(groups[c][1])
+                b.sort()
+                pages = sorted(U)
+                masks = []
+                for p in pages:
+                    m = 0
+                    for j, gi in enumerate(b):
+                        mem, gp, gm = groups[gi]
+                        if p in gp:
+                            m |= gm[gp.index(p)] << (j * rs)
+                    masks.append(m)
+                qids = [-1] * (128 // g)
+                for j, gi in enumerate(b):
+                    for k, q in enumerate(groups[gi][0]):
+                        qids[j * (rs // g) + k] = q
+                bundles.append((b, pages, masks, qids))
+        res.append(bundles)
+    return res
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_bundles_match_python_brute_force(seed):
+    rng = np.random.default_rng(50 + seed)
+    Hkv = int(rng.integers(1, 3))
+    g = int(rng.choice([1, 2, 4]))
+    max_group = int(rng.choice([1, 2, 4, 8]))
+    Hq, Nq, K, P = Hkv * g, int(rng.integers(1, 200)), int(rng.integers(1, 6)), int(rng.integers(2, 60))
+    topk = rng.integers(-1, P, size=(Hq, Nq, K)).astype(np.int32)
+    out = oracle.group(topk, Hq, Hkv, Nq, P, max_group, max_group * 4)
+    b = oracle.bundle(out, Hq, Hkv, Nq, max_group)
+    ref = py_bundle(out, Hq, Hkv, Nq, max_group)
+    for h in range(Hkv):
+        assert b["n_bundles"][h] == len(ref[h])
+        for k, (grp, pages, masks, qids) in enumerate(ref[h]):
+            bp = b["bundle_ptr"][h]
+            assert list(b["bundle_groups"][h, bp[k]:bp[k + 1]]) == grp
+            up = b["bunion_ptr"][h]
+            assert list(b["bunion_pages"][up[k]:up[k + 1]]) == pages
+            words = b["bunion_mask"][up[k]:up[k + 1]].astype(np.uint64)
+            got = [int(w[0]) | int(w[1]) << 32 | int(w[2]) << 64 | int(w[3]) << 96 for w in words]
+            assert got == masks
+            assert list(b["bundle_qid"][h, k]) == qids
+        assert b["bcounters"][h, 0] == sum(len(x[1]) for x in ref[h])
+
+
+def test_bundles_partition_groups_and_keep_row_supports():
+    w = W.random_small(8, Hq=8, Hkv=2, Nq=200, K=6)
+    out = oracle.group(w.topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, 8, 64)
+    b = oracle.bundle(out, w.Hq, w.Hkv, w.Nq, 8)
+    g = w.g
+    for h in range(w.Hkv):
+        seen = np.zeros(out["n_groups"][h], int)
+        for k in range(b["n_bundles"][h]):
+            bp, up = b["bundle_ptr"][h], b["bunion_ptr"][h]
+            seen[b["bundle_groups"][h, bp[k]:bp[k + 1]]] += 1
+            assert bp[k + 1] - bp[k] <= 128 // 32
+            for e in range(up[k], up[k + 1]):
+                p = b["bunion_pages"][e]
+                m = int(b["bunion_mask"][e][0]) | int(b["bunion_mask"][e][1]) << 32 | \
+                    int(b["bunion_mask"][e][2]) << 64 | int(b["bunion_mask"][e][3]) << 96
+                for row in range(128):
+                    q = b["bundle_qid"][h, k, row // g]
+                    want = q >= 0 and p in set(w.topk[h * g + row % g, q].tolist())
+                    assert bool((m >> row) & 1) == want
+        assert np.all(seen == 1)
