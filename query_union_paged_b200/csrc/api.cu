@@ -300,7 +300,7 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                                            : (es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)Hkv, (cuuint64_t)P_phys};
     const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)T * d * es, (cuuint64_t)Hkv * T * d * es};
-    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)T, 1, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), (cuuint32_t)std::min(T, 64), 1, 1};  // one 64-token step
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const void* srcs[2] = {K_cache, V_cache};
     for (int i = 0; i < 2; ++i) {
@@ -311,13 +311,12 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QUP_ERR_ARG;
     }
-    // a pipeline step covers one page (T >= 64) or 64 tokens of smaller pages
-    const int st = T >= 64 ? T : 64;
-    const size_t stage = 2u * st * qup::kHeadDim * es;
-    const size_t fixed = qup::attn_smem_bytes(es, st, 0, Hkv);
+    // a pipeline step is 64 tokens: as many K+V steps in flight as shared memory allows
+    const size_t stage = qup::attn_stage_bytes(es);
+    const size_t fixed = qup::attn_smem_bytes(es, 0, Hkv);
     if ((size_t)ds->smem_optin < fixed + stage) return QUP_ERR_ARG;
     const int ns = (int)std::min<size_t>(qup::kMaxStages, ((size_t)ds->smem_optin - fixed) / stage);
-    const size_t smem = qup::attn_smem_bytes(es, st, ns, Hkv);
+    const size_t smem = qup::attn_smem_bytes(es, ns, Hkv);
 
     qup::AttnParams p;
     std::memset(&p, 0, sizeof(p));

@@ -34,8 +34,9 @@ struct AttnParams {
     int dbg_skip_stage;
 };
 
-// dynamic shared memory of the attention kernel for (element size, step tokens, stages, KV heads)
-size_t attn_smem_bytes(int es, int st, int n_stages, int Hkv);
+// dynamic shared memory of the attention kernel for (element size, stages, KV heads), and one ring stage
+size_t attn_smem_bytes(int es, int n_stages, int Hkv);
+size_t attn_stage_bytes(int es);
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);

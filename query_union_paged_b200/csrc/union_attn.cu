@@ -3,31 +3,37 @@
 //
 // Work item: a bundle of up to 128 query rows (up to 128 / rows_per_group
 // page-affine groups of one KV head, see qup_groups).  Pages of the bundle
-// union are streamed once per bundle, one step = ST tokens (one page when
-// T >= 64, else 64 / T pages), through an NS-slot TMA ring.  Per step g:
-//      S_b  = Q K^T     M = 128 rows, N = ST tokens, K = d      (smem x smem -> TMEM)
-//      P    = masked online softmax of S_b, written back over S_b in TMEM
-//      O_b += P V       M = 128 rows, N = d, K = ST tokens      (TMEM x smem -> TMEM)
-// with b = g & 1.  The two softmax warpgroups ping-pong: warpgroup b owns the
-// steps of parity b, with its own S buffer, running max, row sum and O
-// accumulator, so the softmax of one step overlaps the next; the epilogue
-// merges the two partial results.  A thread owns one query row, so the row
-// max and the row sum never leave the thread.  A row's max is only raised
-// when a score exceeds it by more than kTau (log2 units); O and the row sum
-// are rescaled then, which after the first steps is rare.
+// union are streamed once per bundle in steps of 64 tokens (a 128-token page
+// is two steps; 64 / T smaller pages make one step) through an NS-slot TMA
+// ring.  Per step g, with b = g & 1:
+//      S_b  = Q K^T     M = 128 rows, N = 64 tokens, K = d   (Q from TMEM, K from smem)
+//      P_b  = masked online softmax of S_b                    (TMEM -> registers -> TMEM)
+//      O_b += P_b V     M = 128 rows, N = d, K = 64 tokens    (P from TMEM, V from smem)
+// The two softmax warpgroups ping-pong: warpgroup b owns the steps of parity
+// b, with its own S, P and O columns, running max and row sum, so the softmax
+// of one step overlaps the next; the epilogue merges the two partial results.
+// Keeping Q in TMEM halves the shared-memory operand traffic of QK^T, and a
+// separate P lets S(g+2) start as soon as the softmax has read S(g).  A
+// thread owns one query row, so the row max and the row sum never leave the
+// thread.  A row's max is only raised when a score exceeds it by more than
+// kTau (log2 units); O and the row sum are rescaled then, which after the
+// first steps is rare.  A warp whose 32 rows selected none of a step's pages
+// skips that step's exponentials.
 //
 // Warp roles (320 threads):
 //   warps 0-7  softmax / epilogue: warpgroup b = warps 4b..4b+3, thread =
 //              TMEM lane = bundle row.  They also gather the rows of Q by
-//              original query ID (no reordered Q tensor) at bundle start.
+//              original query ID (no reordered Q tensor) into TMEM.
 //   warp 8     producer: loads the bundle's page list, row masks and
-//              physical pages (warp-parallel) and TMA-loads K and V pages.
-//   warp 9     MMA issuer (one thread) and TMEM owner (512 columns: S0, S1,
-//              O_0, O_1, 128 each).
-// Operand types: bf16 (kind::f16), fp32 (kind::tf32), FP8 E4M3 (kind::f8f6f4:
-// K and V straight from the cache, Q quantised per row with its own scale,
-// P stored as E4M3 of 64 * p).  Every MMA consumes 32 bytes of its K extent
-// per row, so the descriptor arithmetic is shared by the three types.
+//              physical pages (warp-parallel) and TMA-loads K and V.
+//   warp 9     MMA issuer (one elected lane of a warp-uniform loop) and TMEM
+//              owner (512 columns).
+// TMEM columns: S_0, S_1 [0,128); P_0, P_1 from 128; Q after them (bf16 and
+// E4M3); O_0 [256,384), O_1 [384,512).
+// Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
+// FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
+// row with its own scale, P stored as E4M3 of 64 * p).  Every MMA consumes 32
+// bytes of its K extent per row, so the descriptor arithmetic is shared.
 //
 // Every wait is bounded (ptx.cuh); on a timeout the CTA raises an abort flag,
 // drains its in-flight TMA loads and MMAs, frees TMEM and exits.
@@ -43,28 +49,37 @@ namespace qup {
 constexpr int kThreads = 320;
 constexpr int kRows = 128;
 constexpr int kD = kHeadDim;
+constexpr int kST = 64;  // tokens per pipeline step
 constexpr int kTmemCols = 512;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 
 struct StageMeta {
     int32_t upage[4];
     uint32_t mask[4][4];
+    int32_t tok0;  // first token of the step inside its page (128-token pages)
+    int32_t pad[3];
 };
 
 template <int ES, int T>
 struct Geo {
-    static constexpr int ST = T < 64 ? 64 : T;          // tokens per step
-    static constexpr int PPS = ST / T;                  // pages per step
-    static constexpr int kTile = ST * kD * ES;          // one K or V tile of a step
+    static constexpr int SPP = T > kST ? T / kST : 1;   // steps per page
+    static constexpr int PPS = T < kST ? kST / T : 1;   // pages per step
+    static constexpr int BOXR = T < kST ? T : kST;      // token rows per TMA box
+    static constexpr int kTile = kST * kD * ES;         // one K or V tile of a step
     static constexpr int kStage = 2 * kTile;
     static constexpr int kChunkElems = 128 / ES;        // elements per 128-byte swizzle row
     static constexpr int kNChunk = kD * ES / 128;       // 128-byte chunks along d
-    static constexpr int kChunkBytes = ST * 128;        // one chunk column of a K or V tile
-    static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of the Q tile
+    static constexpr int kChunkBytes = kST * 128;       // one chunk column of a K or V tile
+    static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of a shared-memory Q tile
     static constexpr int kMmaK = 32 / ES;               // K elements per MMA instruction
     static constexpr int kNumMmaS = kD * ES / 32;       // MMAs per S (K = d)
-    static constexpr int kNumMmaPV = ST * ES / 32;      // MMAs per O update (K = ST tokens)
-    static constexpr int kPCols = ST * ES / 4;          // TMEM columns of P
+    static constexpr int kNumMmaPV = kST * ES / 32;     // MMAs per O update (K = 64 tokens)
+    static constexpr int kPCols = kST * ES / 4;         // TMEM columns of P
+    static constexpr bool kQTmem = ES != 4;             // Q as the TMEM A operand (bf16, E4M3)
+    static constexpr int kQCols = kD * ES / 4;          // TMEM columns of Q
+    static constexpr uint32_t kColP = 128, kColQ = 128 + 2 * kPCols, kColO = 256;
+    static_assert(!kQTmem || kColQ + kQCols <= kColO, "TMEM budget");
+    static_assert(kColP + 2 * kPCols <= kColO, "TMEM budget");
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
     static constexpr float kTau = ES == 1 ? 2.f : 8.f;      // lazy-rescale margin (log2 units)
@@ -75,15 +90,15 @@ struct SmemLayout {
     uint32_t stages, q, bars, meta, xch, qsc, misc, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int es, int st, int n_stages, int Hkv) {
+__host__ __device__ inline SmemLayout smem_layout(int es, int n_stages, int Hkv) {
     SmemLayout L;
     uint32_t off = 0;
     L.stages = off;
-    off += (uint32_t)n_stages * 2u * st * kD * es;
+    off += (uint32_t)n_stages * 2u * kST * kD * es;
     L.q = off;
-    off += (uint32_t)kRows * kD * es;
+    if (es == 4) off += (uint32_t)kRows * kD * es;  // fp32 Q stays in shared memory
     L.bars = off;
-    off += 8u * (2u * n_stages + 10u);
+    off += 8u * (2u * n_stages + 12u);
     L.meta = off;
     off += (uint32_t)sizeof(StageMeta) * n_stages;
     L.xch = off;
@@ -100,10 +115,11 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int st, int n_stages, 
 __device__ __forceinline__ uint32_t bar_full(uint32_t b, int s) { return b + 8u * s; }
 __device__ __forceinline__ uint32_t bar_empty(uint32_t b, int s, int ns) { return b + 8u * (ns + s); }
 __device__ __forceinline__ uint32_t bar_sfull(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + i); }
-__device__ __forceinline__ uint32_t bar_pfull(uint32_t b, int w, int ns) { return b + 8u * (2 * ns + 2 + w); }
-__device__ __forceinline__ uint32_t bar_pvdone(uint32_t b, int w, int ns) { return b + 8u * (2 * ns + 4 + w); }
-__device__ __forceinline__ uint32_t bar_qfull(uint32_t b, int ns) { return b + 8u * (2 * ns + 6); }
-__device__ __forceinline__ uint32_t bar_drain(uint32_t b, int ns) { return b + 8u * (2 * ns + 7); }
+__device__ __forceinline__ uint32_t bar_sfree(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 2 + i); }
+__device__ __forceinline__ uint32_t bar_pfull(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 4 + i); }
+__device__ __forceinline__ uint32_t bar_pvdone(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 6 + i); }
+__device__ __forceinline__ uint32_t bar_qfull(uint32_t b, int ns) { return b + 8u * (2 * ns + 8); }
+__device__ __forceinline__ uint32_t bar_drain(uint32_t b, int ns) { return b + 8u * (2 * ns + 9); }
 
 struct Item {
     int h, bi, ub, nU, nsteps;
@@ -111,7 +127,8 @@ struct Item {
 };
 
 // Decode flat bundle f; every role calls this and reaches the same verdict.
-__device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_prefix, int f, int pps) {
+template <int SPP, int PPS>
+__device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_prefix, int f) {
     Item it;
     int h = 0;
     while (h + 1 < p.Hkv && nb_prefix[h + 1] <= f) ++h;
@@ -122,7 +139,7 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_pre
     it.nU = p.union_ptr[bp + 1] - it.ub;
     it.ok = it.ub >= 0 && it.nU >= 0 && (long long)it.ub + it.nU <= p.cap_union;
     if (!it.ok) it.nU = 0;
-    it.nsteps = (it.nU + pps - 1) / pps;
+    it.nsteps = SPP > 1 ? it.nU * SPP : (it.nU + PPS - 1) / PPS;
     return it;
 }
 
@@ -132,13 +149,6 @@ __device__ __forceinline__ uint32_t kmajor_sw128(int r, int c, int rows) {
 }
 
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
-
-template <int N>
-__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* v) {
-    static_assert(N % 32 == 0, "loads come in 32-column pieces");
-#pragma unroll
-    for (int i = 0; i < N / 32; ++i) tmem_ld32(taddr + 32u * i, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * i));
-}
 
 template <int N>
 __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
@@ -158,11 +168,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     union_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ AttnParams p) {
     using G = Geo<ES, T>;
-    constexpr int ST = G::ST, PPS = G::PPS;
+    constexpr int SPP = G::SPP, PPS = G::PPS, BOXR = G::BOXR;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(ES, ST, p.n_stages, p.Hkv);
+    const SmemLayout L = smem_layout(ES, p.n_stages, p.Hkv);
     const int NS = p.n_stages;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bars = sbase + L.bars;
@@ -183,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_sfull(bars, i, NS), 1);
+            mbar_init(bar_sfree(bars, i, NS), 128);
             mbar_init(bar_pfull(bars, i, NS), 128);
             mbar_init(bar_pvdone(bars, i, NS), 1);
         }
@@ -221,10 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int gs = 0;
         bool ok = true;
         for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x) {
-            const Item it = load_item(p, nb_prefix, f, PPS);
-            const int n_ent = it.nsteps * PPS;  // union entries incl. padding of the last step
-            for (int c0 = 0; c0 < n_ent && ok; c0 += 32) {
-                const int idx = c0 + lane;
+            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
+            const int n_ent = SPP > 1 ? it.nU : it.nsteps * PPS;  // incl. padding of the last step
+            for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
+                const int idx = e0 + lane;
                 int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
                 uint4 mk = make_uint4(0, 0, 0, 0);
                 if (idx < it.nU) {
@@ -242,8 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (phys == p.P_phys) mk = make_uint4(0, 0, 0, 0);
                 }
-                const int steps_here = min(32, n_ent - c0) / PPS;
-                for (int sl = 0; sl < steps_here; ++sl, ++gs) {
+                const int ecnt = min(32, n_ent - e0);
+                const int nst = SPP > 1 ? ecnt * SPP : ecnt / PPS;
+                for (int k = 0; k < nst; ++k, ++gs) {
                     const int slot = gs % NS;
                     int okv = 0;
                     if (lane == 0)
@@ -253,10 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
                                                       gs == p.dbg_skip_stage);
+                    const int tok0 = SPP > 1 ? (k % SPP) * kST : 0;
                     int ph[PPS];
 #pragma unroll
                     for (int q = 0; q < PPS; ++q) {
-                        const int src = (sl * PPS + q) & 31;
+                        const int src = SPP > 1 ? (k / SPP) : (k * PPS + q);
                         const int uq = __shfl_sync(0xffffffffu, u, src);
                         ph[q] = __shfl_sync(0xffffffffu, phys, src);
                         const uint32_t m0 = __shfl_sync(0xffffffffu, mk.x, src);
@@ -270,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             m.mask[q][1] = m1;
                             m.mask[q][2] = m2;
                             m.mask[q][3] = m3;
+                            m.tok0 = tok0;
                         }
                     }
                     if (issue) {
@@ -282,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int q = 0; q < PPS; ++q) {
 #pragma unroll
                             for (int c = 0; c < G::kNChunk; ++c) {
-                                const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * T) * 128u;
-                                tma_load_4d(kdst + off, &tmK, fb, c * G::kChunkElems, 0, it.h, ph[q]);
-                                tma_load_4d(vdst + off, &tmV, fb, c * G::kChunkElems, 0, it.h, ph[q]);
+                                const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * BOXR) * 128u;
+                                tma_load_4d(kdst + off, &tmK, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
+                                tma_load_4d(vdst + off, &tmV, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
                             }
                         }
                     }
@@ -301,74 +315,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // ============================================================ MMA issuer (one thread)
-        if (lane == 0) {
-            const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, ST, kRows);
-            const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
-            // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
-            // has only the 128-byte swizzle with 32-byte atoms (layout 1, 4-row atoms)
-            constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
-            constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
-            const uint32_t qbase = sbase + L.q;
-            const bool pv_first = NS == 1;  // one slot: O(g-1) must free it before S(g) can load
-            int gs = 0, item_no = 0;
-            bool ok = true;
-            for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x, ++item_no) {
-                const Item it = load_item(p, nb_prefix, f, PPS);
-                ok = mbar_wait(bar_qfull(bars, NS), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
-                if (!ok) break;
-                tc_fence_after();
-                for (int s = 0; s <= it.nsteps && ok; ++s) {
-                    for (int half = 0; half < 2 && ok; ++half) {
-                        const bool do_s = (half == (pv_first ? 1 : 0)) && s < it.nsteps;
-                        const bool do_pv = (half == (pv_first ? 0 : 1)) && s > 0;
-                        if (do_s) {
-                            const int g = gs + s, slot = g % NS, b = g & 1;
-                            ok = mbar_wait(bar_full(bars, slot), (g / NS) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
-                                           lim);
-                            // S_b last held P(g-2), read by the O_b update of step g-2
-                            if (ok && g >= 2)
-                                ok = mbar_wait(bar_pvdone(bars, b, NS), ((g - 2) >> 1) & 1, abort_flag, p.err,
-                                               QUP_ERR_TIMEOUT, lim);
-                            if (!ok) break;
-                            tc_fence_after();
-                            const uint32_t kbase = sbase + L.stages + (uint32_t)slot * G::kStage;
+        // ============================================================ MMA issuer (whole warp, one elected lane)
+        // Issue order per bundle: S(s) then O(s - LAG).  With the two warpgroups half a
+        // period apart, the events arrive as S-free(g), P-ready(g-1), S-free(g+1),
+        // P-ready(g), ..., so LAG = 3 issues every S as soon as its buffer is read and
+        // every O update as soon as its P is written.  S(s) needs the stage of step s,
+        // whose previous use was released by O(s - NS): LAG <= NS - 1.
+        const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, kST, kRows);
+        const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
+        // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
+        // has only the 128-byte swizzle with 32-byte atoms (layout 1, 4-row atoms)
+        constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
+        constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
+        const uint32_t qbase = sbase + L.q;
+        const int LAG = NS >= 4 ? 3 : NS - 1;
+        int gs = 0, item_no = 0;
+        bool ok = true;
+        for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x, ++item_no) {
+            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
+            ok = warp_ok(mbar_wait(bar_qfull(bars, NS), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+            if (!ok) break;
+            tc_fence_after();
+            for (int s = 0; s < it.nsteps + LAG && ok; ++s) {
+                if (s < it.nsteps) {  // ---- S(g) = Q K^T into S_b
+                    const int g = gs + s, slot = g % NS, b = g & 1;
+                    ok = warp_ok(mbar_wait(bar_full(bars, slot), (g / NS) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
+                                           lim) &&
+                                 (g < 2 || mbar_wait(bar_sfree(bars, b, NS), ((g - 2) >> 1) & 1, abort_flag, p.err,
+                                                     QUP_ERR_TIMEOUT, lim)));  // softmax of g-2 has read S_b
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t kdesc = smem_desc(sbase + L.stages + (uint32_t)slot * G::kStage, 16, 1024, 2);
+                    const uint64_t qdesc = smem_desc(qbase, 16, 1024, 2);
+                    if (elect_one_sync()) {
 #pragma unroll
-                            for (int k = 0; k < G::kNumMmaS; ++k) {
-                                const uint32_t koff = (uint32_t)(k >> 2) * G::kChunkBytes + (uint32_t)(k & 3) * 32u;
-                                const uint32_t qoff = (uint32_t)(k >> 2) * G::kQChunkBytes + (uint32_t)(k & 3) * 32u;
-                                tc_mma<G::kKind>(tmem + (uint32_t)b * 128u, smem_desc(qbase + qoff, 16, 1024, 2),
-                                                 smem_desc(kbase + koff, 16, 1024, 2), idesc_s, k > 0);
+                        for (int k = 0; k < G::kNumMmaS; ++k) {
+                            const uint32_t koff = ((k >> 2) * G::kChunkBytes + (k & 3) * 32) >> 4;
+                            if constexpr (G::kQTmem) {
+                                tc_mma_ts<G::kKind>(tmem + 64u * b, tmem + G::kColQ + 8u * k, kdesc + koff, idesc_s,
+                                                    k > 0);
+                            } else {
+                                const uint32_t qoff = ((k >> 2) * G::kQChunkBytes + (k & 3) * 32) >> 4;
+                                tc_mma<G::kKind>(tmem + 64u * b, qdesc + qoff, kdesc + koff, idesc_s, k > 0);
                             }
-                            tc_commit(bar_sfull(bars, b, NS));
                         }
-                        if (do_pv) {
-                            const int g = gs + s - 1, slot = g % NS, b = g & 1;
-                            const uint32_t vbase = sbase + L.stages + (uint32_t)slot * G::kStage + G::kTile;
-                            ok = mbar_wait(bar_pfull(bars, b, NS), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
-                                           lim);
-                            if (!ok) break;
-                            tc_fence_after();
-                            // steps 0 and 1 of a bundle open O_0 / O_1 (overwrite)
-#pragma unroll
-                            for (int k = 0; k < G::kNumMmaPV; ++k) {
-                                // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
-                                tc_mma_ts<G::kKind>(tmem + 256u + 128u * b, tmem + (uint32_t)b * 128u + 8u * k,
-                                                    smem_desc(vbase + (uint32_t)(k * G::kMmaK) * 128u,
-                                                              (uint32_t)G::kChunkBytes, vsbo, vlayout),
-                                                    idesc_o, (s - 1) >= 2 || k > 0);
-                            }
-                            tc_commit(bar_pvdone(bars, b, NS));
-                            tc_commit(bar_empty(bars, slot, NS));
-                        }
+                        tc_commit(bar_sfull(bars, b, NS));
                     }
+                    __syncwarp();
                 }
-                gs += it.nsteps;
+                if (s >= LAG) {  // ---- O_b += P_b V for step g = s - LAG
+                    const int sl = s - LAG, g = gs + sl, slot = g % NS, b = g & 1;
+                    ok = warp_ok(mbar_wait(bar_pfull(bars, b, NS), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
+                                           lim));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t vdesc = smem_desc(sbase + L.stages + (uint32_t)slot * G::kStage + G::kTile,
+                                                     (uint32_t)G::kChunkBytes, vsbo, vlayout);
+                    const bool acc0 = sl >= 2;  // steps 0 and 1 of a bundle open O_0 / O_1
+                    if (elect_one_sync()) {
+#pragma unroll
+                        for (int k = 0; k < G::kNumMmaPV; ++k) {
+                            // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
+                            tc_mma_ts<G::kKind>(tmem + G::kColO + 128u * b, tmem + G::kColP + G::kPCols * b + 8u * k,
+                                                vdesc + ((k * G::kMmaK * 128) >> 4), idesc_o, acc0 || k > 0);
+                        }
+                        tc_commit(bar_pvdone(bars, b, NS));
+                        tc_commit(bar_empty(bars, slot, NS));
+                    }
+                    __syncwarp();
+                }
             }
-            // every issued MMA completes before TMEM is freed
-            tc_commit(bar_drain(bars, NS));
-            mbar_wait_drain(bar_drain(bars, NS), 0, lim);
+            gs += it.nsteps;
         }
+        // every issued MMA completes before TMEM is freed
+        if (elect_one_sync()) tc_commit(bar_drain(bars, NS));
+        __syncwarp();
+        mbar_wait_drain(bar_drain(bars, NS), 0, lim);
         __syncwarp();
     } else {
         // ============================================================ softmax / epilogue (256 threads)
@@ -376,14 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;           // TMEM lane quadrant this warp may access
         const int r = quad * 32 + lane;      // bundle row == TMEM lane
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        const uint32_t s_addr = tmem + lane_base + 128u * wg;        // S_wg / P_wg of this row
-        const uint32_t o_addr = tmem + lane_base + 256u + 128u * wg; // O_wg of this row
+        const uint32_t s_addr = tmem + lane_base + 64u * wg;                      // S_wg
+        const uint32_t p_addr = tmem + lane_base + G::kColP + G::kPCols * wg;     // P_wg
+        const uint32_t o_addr = tmem + lane_base + G::kColO + 128u * wg;          // O_wg
         const float kNegInf = -__int_as_float(0x7f800000);
         const int g = p.g, MQ = kRows / g;
         int gs = 0;
         bool ok = true;
         for (int f = blockIdx.x; f < n_items; f += gridDim.x) {
-            const Item it = load_item(p, nb_prefix, f, PPS);
+            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             // ---- this row's query (original ID) and head
             int qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
@@ -394,25 +417,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int head = it.h * g + (r % g);
             const int qpos = qid >= 0 ? p.q_pos[qid] : -1;
             const int vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
-            // ---- Q row by original ID -> K-major SW128 operand tile
+            // ---- Q row by original ID -> TMEM (bf16, E4M3) or the shared-memory tile (fp32)
             {
-                uint8_t* qt = smem + L.q;
                 const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
                 if constexpr (ES == 2) {
                     const uint4* src =
                         reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off) + wg * 8;
+                    uint32_t qv[32];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, wg * 8 + c, kRows)) = v;
+                        qv[4 * c] = v.x;
+                        qv[4 * c + 1] = v.y;
+                        qv[4 * c + 2] = v.z;
+                        qv[4 * c + 3] = v.w;
                     }
+                    tmem_st_x32(tmem + lane_base + G::kColQ + 32u * wg, qv);
                 } else if constexpr (ES == 4) {
+                    uint8_t* qt = smem + L.q;
                     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off) + wg * 16;
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
                         *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, wg * 16 + c, kRows)) = v;
                     }
+                    fence_proxy_async_smem();
                 } else {
                     if (wg == 0) {  // whole row: bf16 -> E4M3 with the row's scale amax / 448
                         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
@@ -428,28 +457,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
                         }
                         const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                        uint32_t qv[32];
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {  // 16 output bytes from 2 input chunks
-                            float x[16];
-                            const uint32_t w8[8] = {raw[2 * c].x,     raw[2 * c].y,     raw[2 * c].z,     raw[2 * c].w,
-                                                    raw[2 * c + 1].x, raw[2 * c + 1].y, raw[2 * c + 1].z, raw[2 * c + 1].w};
+                        for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
+                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+                            float x[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                x[2 * e] = __uint_as_float(w8[e] << 16) * inv;
-                                x[2 * e + 1] = __uint_as_float(w8[e] & 0xffff0000u) * inv;
+                            for (int e = 0; e < 4; ++e) {
+                                x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
+                                x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
                             }
-                            uint4 o;
-                            o.x = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-                            o.y = pack_e4m3x4(x[4], x[5], x[6], x[7]);
-                            o.z = pack_e4m3x4(x[8], x[9], x[10], x[11]);
-                            o.w = pack_e4m3x4(x[12], x[13], x[14], x[15]);
-                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = o;
+                            qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                            qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
                         }
+                        tmem_st_x32(tmem + lane_base + G::kColQ, qv);
                         qsc[r] = amax * (1.f / 448.f);
                     }
                 }
+                if constexpr (G::kQTmem) tmem_wait_st();
             }
-            fence_proxy_async_smem();
+            tc_fence_before();
             mbar_arrive(bar_qfull(bars, NS));
             float cs = p.scale_log2;  // score scale (log2 domain) of this row
             if constexpr (ES == 1) {
@@ -470,13 +497,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            QUP_ERR_TIMEOUT, lim));
                 if (!ok) continue;
                 tc_fence_after();
-                uint32_t sv[ST];
-                tmem_ld_n<ST>(s_addr, sv);
+                uint32_t sv[kST];
+                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                // while S is in flight: this warpgroup's previous O update must be done before
+                // O is rescaled and before P_wg is overwritten (usually long done)
+                const bool pv_ok = gstep < 2 || mbar_wait(bar_pvdone(bars, wg, NS), ((gstep - 2) >> 1) & 1, abort_flag,
+                                                          p.err, QUP_ERR_TIMEOUT, lim);
                 const StageMeta& mt = meta[slot];
+                const int tok0 = mt.tok0;
                 // cache slots at or past kv_len may hold non-finite bytes: zero those V rows
-                if (r < ST) {
-                    const int q = r / T;
-                    if (mt.upage[q] * T + (r - q * T) >= p.kv_len) {
+                if (r < kST) {
+                    const int q = r / BOXR;
+                    if (mt.upage[q] * T + tok0 + (r - q * BOXR) >= p.kv_len) {
                         uint8_t* vt = smem + L.stages + (uint32_t)slot * G::kStage + G::kTile;
 #pragma unroll
                         for (int c = 0; c < G::kNChunk; ++c)
@@ -489,18 +522,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // row r sees token j of page q iff the page is in its own TopK row
                 // (bit r of the page's mask) and the token's position is < vis_end
                 int lim_q[PPS];
+                bool live = false;
 #pragma unroll
                 for (int q = 0; q < PPS; ++q) {
                     const bool mine = (mt.mask[q][r >> 5] >> (r & 31)) & 1u;
-                    lim_q[q] = mine ? max(0, min(T, vis_end - mt.upage[q] * T)) : 0;
+                    lim_q[q] = mine ? max(0, min(BOXR, vis_end - (mt.upage[q] * T + tok0))) : 0;
+                    live |= lim_q[q] > 0;
                 }
                 tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar_sfree(bars, wg, NS));  // S_wg may now be overwritten by S(gstep + 2)
+                const bool warp_live = __any_sync(0xffffffffu, live);
                 float mloc = kNegInf;
+                if (warp_live) {
 #pragma unroll
-                for (int j = 0; j < ST; ++j) {
-                    const float v = (j % T) < lim_q[j / T] ? __uint_as_float(sv[j]) * cs : kNegInf;
-                    sv[j] = __float_as_uint(v);
-                    mloc = fmaxf(mloc, v);
+                    for (int j = 0; j < kST; ++j) {
+                        const float v = (j % BOXR) < lim_q[j / BOXR] ? __uint_as_float(sv[j]) * cs : kNegInf;
+                        sv[j] = __float_as_uint(v);
+                        mloc = fmaxf(mloc, v);
+                    }
                 }
                 // lazy running max: raise it only when a score exceeds it by more than kTau
                 const bool need = mloc > m_used + G::kTau;
@@ -512,41 +552,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float msafe = m_used == kNegInf ? 0.f : m_used;
                 uint32_t pk[G::kPCols];
-                float part0 = 0.f, part1 = 0.f;
-                if constexpr (ES == 2) {
+                if (warp_live) {
+                    float part0 = 0.f, part1 = 0.f;
+                    if constexpr (ES == 2) {
 #pragma unroll
-                    for (int j = 0; j < ST; j += 2) {
-                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                        const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
-                        part0 += p0;
-                        part1 += p1;
-                        pk[j / 2] = pack_bf16x2(p0, p1);
-                    }
-                } else if constexpr (ES == 4) {
+                        for (int j = 0; j < kST; j += 2) {
+                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                            const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
+                            part0 += p0;
+                            part1 += p1;
+                            pk[j / 2] = pack_bf16x2(p0, p1);
+                        }
+                    } else if constexpr (ES == 4) {
 #pragma unroll
-                    for (int j = 0; j < ST; ++j) {
-                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                        if (j & 1) part1 += p0; else part0 += p0;
-                        pk[j] = __float_as_uint(p0);
+                        for (int j = 0; j < kST; ++j) {
+                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                            if (j & 1) part1 += p0;
+                            else part0 += p0;
+                            pk[j] = __float_as_uint(p0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kST; j += 4) {
+                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
+                            const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
+                            const float p2 = ex2(__uint_as_float(sv[j + 2]) - msafe);
+                            const float p3 = ex2(__uint_as_float(sv[j + 3]) - msafe);
+                            part0 += p0 + p2;
+                            part1 += p1 + p3;
+                            pk[j / 4] = pack_e4m3x4(p0 * G::kPScale, p1 * G::kPScale, p2 * G::kPScale, p3 * G::kPScale);
+                        }
                     }
+                    lsum += part0 + part1;
                 } else {
 #pragma unroll
-                    for (int j = 0; j < ST; j += 4) {
-                        const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                        const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
-                        const float p2 = ex2(__uint_as_float(sv[j + 2]) - msafe);
-                        const float p3 = ex2(__uint_as_float(sv[j + 3]) - msafe);
-                        part0 += p0 + p2;
-                        part1 += p1 + p3;
-                        pk[j / 4] = pack_e4m3x4(p0 * G::kPScale, p1 * G::kPScale, p2 * G::kPScale, p3 * G::kPScale);
-                    }
+                    for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
                 }
-                lsum += part0 + part1;
-                // this warpgroup's previous O update must be done before O is rescaled and
-                // before P overwrites S (the MMA of step gstep-2 reads P from the same columns)
-                if (gstep >= 2)
-                    ok = warp_ok(mbar_wait(bar_pvdone(bars, wg, NS), ((gstep - 2) >> 1) & 1, abort_flag, p.err,
-                                           QUP_ERR_TIMEOUT, lim));
+                ok = warp_ok(pv_ok);
                 if (!ok) continue;
                 tc_fence_after();
                 if (mine_steps > 0 && __any_sync(0xffffffffu, need)) {
@@ -559,9 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                         tmem_st_x32(o_addr + 32u * c, ov);
                     }
-                    tmem_wait_st();
                 }
-                tmem_st_n<G::kPCols>(s_addr, pk);
+                tmem_st_n<G::kPCols>(p_addr, pk);
                 tmem_wait_st();
                 fence_proxy_async_smem();  // zeroed V rows -> async proxy
                 tc_fence_before();
@@ -597,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t a[32], e2[32];
-                tmem_ld32(tmem + lane_base + 256u + (uint32_t)(64 * wg + 32 * c), a);
-                tmem_ld32(tmem + lane_base + 384u + (uint32_t)(64 * wg + 32 * c), e2);
+                tmem_ld32(tmem + lane_base + G::kColO + (uint32_t)(64 * wg + 32 * c), a);
+                tmem_ld32(tmem + lane_base + G::kColO + 128u + (uint32_t)(64 * wg + 32 * c), e2);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
@@ -623,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : kNegInf;
             }
             tc_fence_before();
-            bar_sync(1, 256);  // O_0 and O_1 read by both halves before the next bundle overwrites them
+            bar_sync(1, 256);  // O_0, O_1 and Q read before the next bundle overwrites them
         }
     }
 
@@ -634,9 +675,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-size_t attn_smem_bytes(int es, int st, int n_stages, int Hkv) {
-    return smem_layout(es, st, n_stages, Hkv).total;
-}
+size_t attn_smem_bytes(int es, int n_stages, int Hkv) { return smem_layout(es, n_stages, Hkv).total; }
+
+size_t attn_stage_bytes(int es) { return 2u * kST * kD * es; }
 
 template <int ES, int T>
 static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p, int grid,
