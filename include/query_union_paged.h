@@ -138,6 +138,27 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
                      void* stream);
 
 /*
+ * qup_sparse_group without a caller workspace (the paper has no counterpart:
+ * it is an allocation-free calling form of the same grouping).  For callers
+ * that cannot hand over a scratch buffer: a host program holding no device
+ * allocator at the call, or a serving loop whose device memory is fixed at
+ * start-up.  The scratch lives in a fixed array of QUP_STATIC_GROUP_SCRATCH_BYTES
+ * in this library's device image (one per device); nothing is allocated.
+ * Arguments, outputs and device errors are those of qup_sparse_group.
+ *  - Returns QUP_ERR_CAPACITY when the workspace qup_group_workspace reports
+ *    for these sizes exceeds QUP_STATIC_GROUP_SCRATCH_BYTES; nothing is launched.
+ *  - The first call on a device looks up the array's device address (a host
+ *    query, with that device current); make that first call before capturing
+ *    a stream.
+ *  - Every call on one device shares the one array: two calls in flight at the
+ *    same time (other streams, other host threads) race on it and corrupt each
+ *    other's groups.  Order them on one stream.
+ */
+#define QUP_STATIC_GROUP_SCRATCH_BYTES (16u << 20)
+int qup_sparse_group_static(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages,
+                            int max_group, int window, qup_groups* out, void* stream);
+
+/*
  * Pack the groups in `g` (n_groups .. row_mask filled, for instance by a
  * caller's own partition) into bundles: fills n_bundles .. bcounters and
  * rows_per_group.  max_group bounds the members of every group (1..8,
