@@ -101,6 +101,11 @@ def profiled_traffic(workload_name: str):
     return float(m.group(1)) if m else None
 
 
+# kernels of one step: grouping (rowbits, greedy, emit), bundling (bits, greedy, emit, order),
+# union attention
+LAUNCHES_PER_STEP = 3 + 4 + 1
+
+
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples taken during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -320,7 +325,7 @@ def main():
                      ("" if w.kv_dtype == W.DT_BF16 else " x nominal dtype ratio"),
                      "unique_kv_gbs": round(uniq_bytes / (attn_ms * 1e-3) / 1e9, 1),
                      "hbm_frac_unique_kv": round(uniq_bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": e2e,
     }
     if rank == 0:

@@ -88,6 +88,10 @@ extern "C" {
  *            slot or rank is empty.
  *   bcounters[h*2 + 0..1] = bundle page visits (sum of bundle union sizes:
  *            the pages the attention kernel streams), number of bundles.
+ *   bundle_order[0 .. total bundles) = flat bundle indices (f = bundles of
+ *            earlier KV heads + b) sorted by union size, largest first, equal
+ *            sizes by index: the order in which the attention kernel deals
+ *            bundles to its CTAs.
  */
 typedef struct {
     int32_t* n_groups;     /* [Hkv] */
@@ -106,6 +110,7 @@ typedef struct {
     uint32_t* bunion_mask; /* [cap_union][4] */
     int32_t* bundle_qid;   /* [Hkv][Nq][128/g] */
     int64_t* bcounters;    /* [Hkv][2] */
+    int32_t* bundle_order; /* [Hkv*Nq] */
     int32_t rows_per_group;/* set by qup_sparse_group / qup_build_bundles */
     int32_t bundle_window; /* groups per bundling window (0: default 64) */
 } qup_groups;

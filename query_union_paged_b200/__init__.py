@@ -39,7 +39,7 @@ class QupError(RuntimeError):
 
 _GROUP_KEYS = ("n_groups", "group_ptr", "members", "union_ptr", "union_pages", "row_mask", "counters")
 _BUNDLE_KEYS = ("n_bundles", "bundle_ptr", "bundle_groups", "bunion_ptr", "bunion_pages", "bunion_mask",
-                "bundle_qid", "bcounters")
+                "bundle_qid", "bcounters", "bundle_order")
 
 
 class _Groups(ctypes.Structure):
@@ -117,6 +117,7 @@ class Groups:
     bunion_mask: "torch.Tensor" = None
     bundle_qid: "torch.Tensor" = None
     bcounters: "torch.Tensor" = None
+    bundle_order: "torch.Tensor" = None
     workspace: Optional["torch.Tensor"] = None
     rows_per_group: int = 0
     bundle_window: int = 0
@@ -155,6 +156,7 @@ def alloc_groups(Hq, Hkv, Nq, cap, ws_bytes, device) -> Groups:
                   bunion_pages=torch.empty(cap, **i32), bunion_mask=torch.empty(cap, 4, **i32),
                   bundle_qid=torch.empty(Hkv, max(Nq, 1), 128 // g, **i32),
                   bcounters=torch.empty(Hkv, 2, dtype=torch.int64, device=device),
+                  bundle_order=torch.empty(max(Hkv * Nq, 1), **i32),
                   workspace=torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device))
 
 

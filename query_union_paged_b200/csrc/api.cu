@@ -178,6 +178,7 @@ int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, i
     a.bundle_qid = g->bundle_qid;
     a.cap = g->cap_union;
     a.bcounters = g->bcounters;
+    a.bundle_order = g->bundle_order;
     a.err = ds->err;
     a.sms = ds->sms;
     return qup::launch_bundles(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
@@ -185,7 +186,7 @@ int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, i
 
 bool bundle_fields_ok(const qup_groups* g) {
     return g->n_bundles && g->bundle_ptr && g->bundle_groups && g->bunion_ptr && g->bunion_pages && g->bunion_mask &&
-           g->bundle_qid && g->bcounters;
+           g->bundle_qid && g->bcounters && g->bundle_order;
 }
 
 }  // namespace
@@ -329,6 +330,7 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.union_pages = groups->bunion_pages;
     p.row_mask = groups->bunion_mask;
     p.bundle_qid = groups->bundle_qid;
+    p.bundle_order = groups->bundle_order;
     p.q_pos = q_pos;
     p.O = O;
     p.lse = lse;

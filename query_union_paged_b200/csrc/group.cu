@@ -494,6 +494,95 @@ cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// Work order of the attention kernel: the flat bundle indices (KV heads in
+// order, then bundles) sorted by union size, largest first, equal sizes by
+// index (a stable counting sort; sizes above kOrderBuckets-1 share the top
+// bucket).  The attention kernel deals this order out to its CTAs in a snake,
+// which keeps the per-CTA sums of union pages close to the mean.
+constexpr int kOrderBuckets = 4096;
+
+__global__ void __launch_bounds__(1024) bnd_order_kernel(const int32_t* __restrict__ n_bundles,
+                                                         const int32_t* __restrict__ bunion_ptr, int Hkv, int Nq,
+                                                         int32_t* __restrict__ order) {
+    __shared__ int cursor[kOrderBuckets];
+    __shared__ int warp_sum[32];
+    extern __shared__ int head_start[];  // [Hkv + 1] flat index of each KV head's first bundle
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        int acc = 0;
+        for (int h = 0; h < Hkv; ++h) {
+            head_start[h] = acc;
+            const int n = n_bundles[h];
+            acc += (n >= 0 && n <= Nq) ? n : 0;  // the attention kernel reports a bad count
+        }
+        head_start[Hkv] = acc;
+    }
+    for (int k = tid; k < kOrderBuckets; k += blockDim.x) cursor[k] = 0;
+    __syncthreads();
+    const int n = head_start[Hkv];
+    auto key_of = [&](int h, int bi) {
+        const size_t b = (size_t)h * (Nq + 1) + bi;
+        const int size = bunion_ptr[b + 1] - bunion_ptr[b];
+        return kOrderBuckets - 1 - min(max(size, 0), kOrderBuckets - 1);  // larger union -> smaller key
+    };
+    for (int h = 0; h < Hkv; ++h)
+        for (int bi = tid; bi < head_start[h + 1] - head_start[h]; bi += blockDim.x) atomicAdd(&cursor[key_of(h, bi)], 1);
+    __syncthreads();
+    // exclusive scan of the histogram: kOrderBuckets / blockDim.x buckets per thread
+    constexpr int kPer = kOrderBuckets / 1024;
+    int v[kPer], run = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        v[k] = run;
+        run += cursor[tid * kPer + k];
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_sum[lane], wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        warp_sum[lane] = wi - w;
+    }
+    __syncthreads();
+    const int base = warp_sum[warp] + incl - run;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) cursor[tid * kPer + k] = base + v[k];
+    __syncthreads();
+    // stable scatter: one warp walks the flat indices in order, 32 at a time
+    if (warp == 0) {
+        int h = 0;
+        for (int f0 = 0; f0 < n; f0 += 32) {
+            const int f = f0 + lane;
+            const unsigned live = __ballot_sync(0xffffffffu, f < n);
+            if (f < n) {
+                while (head_start[h + 1] <= f) ++h;
+                const int key = key_of(h, f - head_start[h]);
+                const unsigned peers = __match_any_sync(live, key);
+                const int leader = __ffs(peers) - 1;
+                const int rank = __popc(peers & ((1u << lane) - 1u));
+                int start = 0;
+                if (lane == leader) {
+                    start = cursor[key];
+                    cursor[key] = start + __popc(peers);
+                }
+                start = __shfl_sync(live, start, leader);
+                order[start + rank] = f;
+            }
+            __syncwarp();
+        }
+    }
+}
+
 }  // namespace qup
 
 namespace qup {
@@ -524,6 +613,8 @@ cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream) {
                                                  a.n_bundles, a.bundle_ptr, a.bundle_groups, a.ws_usize, a.ws_wtot,
                                                  a.bunion_ptr, a.bunion_pages, a.bunion_mask, a.bundle_qid, a.cap,
                                                  a.bcounters, a.err);
+    bnd_order_kernel<<<1, 1024, sizeof(int) * (a.Hkv + 1), stream>>>(a.n_bundles, a.bunion_ptr, a.Hkv, a.Nq,
+                                                                      a.bundle_order);
     return cudaGetLastError();
 }
 

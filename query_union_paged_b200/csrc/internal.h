@@ -22,6 +22,7 @@ struct AttnParams {
     const int32_t* union_pages;  // [cap]
     const uint32_t* row_mask;    // [cap][4] 128-bit row masks
     const int32_t* bundle_qid;   // [Hkv][Nq][128/g]
+    const int32_t* bundle_order; // [n_items] flat bundle indices, largest union first
     const int32_t* q_pos;
     void* O;
     float* lse;
@@ -84,6 +85,7 @@ struct BundleLaunch {
     int32_t* bundle_qid;
     long long cap;
     int64_t* bcounters;
+    int32_t* bundle_order;
     unsigned* err;
     int sms;
 };

@@ -143,6 +143,20 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_pre
     return it;
 }
 
+// Flat bundle index of this CTA's r-th work item, -1 past the end, -2 for a bad
+// order entry (skipped; QUP_ERR_GROUP).  The bundle order (largest unions first)
+// is dealt out in a snake: round r gives CTA b the position r*G + b when r is
+// even and r*G + G-1-b when r is odd, so each CTA's total work stays near the
+// mean.  Positions only grow with r, so the first position past the end ends
+// the walk.  Every role calls this and reaches the same verdict.
+__device__ __forceinline__ int item_at(const AttnParams& p, int r, int n_items) {
+    const long long G = gridDim.x;
+    const long long pos = (long long)r * G + ((r & 1) ? G - 1 - blockIdx.x : (long long)blockIdx.x);
+    if (pos >= n_items) return -1;
+    const int f = p.bundle_order[pos];
+    return (f >= 0 && f < n_items) ? f : -2;
+}
+
 // byte offset of 16-byte chunk c of row r inside a K-major SW128 operand tile of `rows` rows
 __device__ __forceinline__ uint32_t kmajor_sw128(int r, int c, int rows) {
     return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
@@ -231,7 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================================================ producer (whole warp)
         int gs = 0;
         bool ok = true;
-        for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x) {
+        for (int rnd = 0; ok; ++rnd) {
+            const int f = item_at(p, rnd, n_items);
+            if (f == -1) break;
+            if (f < 0) continue;
             const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
             const int n_ent = SPP > 1 ? it.nU : it.nsteps * PPS;  // incl. padding of the last step
             for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
@@ -331,7 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int LAG = NS >= 4 ? 3 : NS - 1;
         int gs = 0, item_no = 0;
         bool ok = true;
-        for (int f = blockIdx.x; f < n_items && ok; f += gridDim.x, ++item_no) {
+        for (int rnd = 0; ok; ++rnd) {
+            const int f = item_at(p, rnd, n_items);
+            if (f == -1) break;
+            if (f < 0) continue;
             const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
             ok = warp_ok(mbar_wait(bar_qfull(bars, NS), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
             if (!ok) break;
@@ -386,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             gs += it.nsteps;
+            ++item_no;
         }
         // every issued MMA completes before TMEM is freed
         if (elect_one_sync()) tc_commit(bar_drain(bars, NS));
@@ -405,7 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = p.g, MQ = kRows / g;
         int gs = 0;
         bool ok = true;
-        for (int f = blockIdx.x; f < n_items; f += gridDim.x) {
+        for (int rnd = 0;; ++rnd) {
+            const int f = item_at(p, rnd, n_items);
+            if (f == -1) break;
+            if (f < 0) {
+                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
+                continue;
+            }
             const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             // ---- this row's query (original ID) and head

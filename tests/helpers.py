@@ -41,7 +41,21 @@ def groups_to_host(gr):
              bunion_pages=gr.bunion_pages[:btotal].cpu().numpy(),
              bunion_mask=gr.bunion_mask[:btotal].cpu().numpy().view(np.uint32),
              bundle_qid=gr.bundle_qid.cpu().numpy(), bcounters=gr.bcounters.cpu().numpy())
+    if gr.bundle_order is not None:
+        d["bundle_order"] = gr.bundle_order[:int(nb.sum())].cpu().numpy()
     return d
+
+
+def expected_bundle_order(d):
+    """Flat bundle indices sorted by union size, largest first, equal sizes by index (sizes above
+    4095 count as 4095), from the bundle CSR of `d`."""
+    sizes = []
+    for h in range(d["n_bundles"].size):
+        p = d["bunion_ptr"][h, :int(d["n_bundles"][h]) + 1].astype(np.int64)
+        sizes.append(np.diff(p))
+    sizes = np.concatenate(sizes) if sizes else np.zeros(0, np.int64)
+    key = np.minimum(sizes, 4095)
+    return np.argsort(-key, kind="stable").astype(np.int32)
 
 
 def assert_groups_equal(got, ref):
@@ -71,6 +85,8 @@ def assert_bundles_equal(got, ref):
         assert np.array_equal(got["bundle_qid"][h, :n], ref["bundle_qid"][h, :n])
     assert np.array_equal(got["bunion_pages"], ref["bunion_pages"])
     assert np.array_equal(got["bunion_mask"], ref["bunion_mask"])
+    if "bundle_order" in got:
+        assert np.array_equal(got["bundle_order"], expected_bundle_order(ref))
 
 
 def out_to_f64(O):
