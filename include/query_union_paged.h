@@ -184,7 +184,7 @@ int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
  *   Q, q_dtype        device [Nq][Hq][d]; (QUP_F32 with kv QUP_F32) or
  *                     (QUP_BF16 with kv QUP_BF16 or QUP_E4M3)
  *   K_cache, V_cache  device [P_phys][Hkv][T][d], kv_dtype; 16-byte aligned
- *   k_scale, v_scale  device fp32 [Hkv], required iff kv_dtype == QUP_E4M3
+ *   k_scale, v_scale  device fp32 [Hkv], > 0, required iff kv_dtype == QUP_E4M3
  *   page_table        device int32 [num_logical_pages]
  *   T                 page tokens: 16, 32, 64 or 128
  *   topk, Ksel        accepted for the problem statement's signature; the
@@ -193,7 +193,7 @@ int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
  *   groups            output of qup_sparse_group (or qup_build_bundles on
  *                     any partition); the kernel walks its bundles
  *   q_pos, kv_len     device int32 [Nq]; tokens >= kv_len are never attended
- *   d                 must be 128; softmax_scale is applied to q.k
+ *   d                 must be 128; softmax_scale (finite, > 0) is applied to q.k
  *   O                 device [Nq][Hq][d], dtype of Q; rows of queries that
  *                     are in no group are not written
  *   lse               device fp32 [Nq][Hq] natural-log sum of exponentials of

@@ -276,7 +276,7 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
     // supported (dtype, page size) pairs: bf16 16/32/64/128, E4M3 64/128, fp32 32/64
     if (num_logical_pages <= 0 || P_phys <= 0 || kv_len < 0) return QUP_ERR_ARG;
-    if (!(std::isfinite(softmax_scale))) return QUP_ERR_ARG;
+    if (!(std::isfinite(softmax_scale) && softmax_scale > 0.f)) return QUP_ERR_ARG;
     int es;
     if (q_dtype == QUP_F32 && kv_dtype == QUP_F32) es = 4;
     else if (q_dtype == QUP_BF16 && kv_dtype == QUP_BF16) es = 2;
@@ -312,12 +312,13 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QUP_ERR_ARG;
     }
-    // a pipeline step is 64 tokens: as many K+V steps in flight as shared memory allows
-    const size_t stage = qup::attn_stage_bytes(es);
-    const size_t fixed = qup::attn_smem_bytes(es, 0, Hkv);
-    if ((size_t)ds->smem_optin < fixed + stage) return QUP_ERR_ARG;
-    const int ns = (int)std::min<size_t>(qup::kMaxStages, ((size_t)ds->smem_optin - fixed) / stage);
-    const size_t smem = qup::attn_smem_bytes(es, ns, Hkv);
+    // a pipeline step is 64 tokens: as many K and V tiles in flight as shared memory allows,
+    // split between the K ring and the V ring (a V slot is held longer: through the softmax)
+    int nt = 2 * qup::kMaxStages;
+    while (nt >= 4 && qup::attn_smem_bytes(es, nt / 2, nt - nt / 2, Hkv) > (size_t)ds->smem_optin) --nt;
+    if (nt < 4) return QUP_ERR_ARG;
+    const int nsk = nt / 2, nsv = nt - nt / 2;
+    const size_t smem = qup::attn_smem_bytes(es, nsk, nsv, Hkv);
 
     qup::AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -345,7 +346,8 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.Nq = Nq;
     p.g = g;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.n_stages = ns;
+    p.nsk = nsk;
+    p.nsv = nsv;
     p.wait_limit_ns = (unsigned long long)(g_wait_limit_ms > 0 ? g_wait_limit_ms : 2000) * 1000000ull;
     p.dbg_skip_stage = g_skip_stage;
     const cudaError_t e =

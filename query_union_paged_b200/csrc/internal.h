@@ -30,14 +30,15 @@ struct AttnParams {
     long long cap_union;
     int num_logical_pages, P_phys, T, kv_len, Hq, Hkv, Nq, g;
     float scale_log2;  // softmax_scale * log2(e)
-    int n_stages;
+    int nsk, nsv;  // slots of the K ring and of the V ring
     unsigned long long wait_limit_ns;
     int dbg_skip_stage;
 };
 
-// dynamic shared memory of the attention kernel for (element size, stages, KV heads), and one ring stage
-size_t attn_smem_bytes(int es, int n_stages, int Hkv);
-size_t attn_stage_bytes(int es);
+// dynamic shared memory of the attention kernel for (element size, K slots, V slots, KV heads),
+// and one K or V tile (one ring slot)
+size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv);
+size_t attn_tile_bytes(int es);
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);

@@ -4,8 +4,10 @@
 // Work item: a bundle of up to 128 query rows (up to 128 / rows_per_group
 // page-affine groups of one KV head, see qup_groups).  Pages of the bundle
 // union are streamed once per bundle in steps of 64 tokens (a 128-token page
-// is two steps; 64 / T smaller pages make one step) through an NS-slot TMA
-// ring.  Per step g, with b = g & 1:
+// is two steps; 64 / T smaller pages make one step) through two TMA rings,
+// one of K tiles and one of V tiles.  A K slot is released as soon as its S
+// is computed, a V slot when its O update is done, so the loads of K run
+// further ahead than one joint ring would allow.  Per step g, with b = g & 1:
 //      S_b  = Q K^T     M = 128 rows, N = 64 tokens, K = d   (Q from TMEM, K from smem)
 //      P_b  = masked online softmax of S_b                    (TMEM -> registers -> TMEM)
 //      O_b += P_b V     M = 128 rows, N = d, K = 64 tokens    (P from TMEM, V from smem)
@@ -20,19 +22,29 @@
 // first steps is rare.  A warp whose 32 rows selected none of a step's pages
 // skips that step's exponentials.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads):
 //   warps 0-7  softmax / epilogue: warpgroup b = warps 4b..4b+3, thread =
 //              TMEM lane = bundle row.  They also gather the rows of Q by
 //              original query ID (no reordered Q tensor) into TMEM.
-//   warp 8     producer: loads the bundle's page list, row masks and
-//              physical pages (warp-parallel) and TMA-loads K and V.
-//   warp 9     MMA issuer (one elected lane of a warp-uniform loop) and TMEM
-//              owner (512 columns).
+//   warp 8     K producer: walks the bundle's page list, resolves physical
+//              pages (warp-parallel) and TMA-loads the K tiles.
+//   warp 10    V producer: the same walk for the V tiles; it also writes each
+//              step's page numbers and row masks, which live as long as the
+//              V slot (until the step's O update).
+//   warp 9     S issuer (one elected lane of a warp-uniform loop) and TMEM
+//              owner (512 columns): S(g) as soon as K tile g and S buffer
+//              g & 1 are ready.
+//   warp 11    PV issuer: O_b += P_b V as soon as P(g) and V tile g are
+//              ready.  Issuing the two streams from two warps on different SM
+//              sub-partitions keeps either from waiting behind the other, and
+//              keeps each issuer's loop short: a single issuing warp that
+//              shares its sub-partition with two busy softmax warps gets too
+//              few issue slots to keep the tensor pipe fed.
 // TMEM columns: S_0, S_1 [0,128); P_0, P_1 from 128; Q after them (bf16 and
 // E4M3); O_0 [256,384), O_1 [384,512).
 // Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
 // FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
-// row with its own scale, P stored as E4M3 of 64 * p).  Every MMA consumes 32
+// row with its own scale, P stored as E4M3 of 2^6 p).  Every MMA consumes 32
 // bytes of its K extent per row, so the descriptor arithmetic is shared.
 //
 // Every wait is bounded (ptx.cuh); on a timeout the CTA raises an abort flag,
@@ -46,12 +58,12 @@
 
 namespace qup {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kRows = 128;
 constexpr int kD = kHeadDim;
 constexpr int kST = 64;  // tokens per pipeline step
 constexpr int kTmemCols = 512;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10, kPvWarp = 11;
 
 struct StageMeta {
     int32_t upage[4];
@@ -66,7 +78,6 @@ struct Geo {
     static constexpr int PPS = T < kST ? kST / T : 1;   // pages per step
     static constexpr int BOXR = T < kST ? T : kST;      // token rows per TMA box
     static constexpr int kTile = kST * kD * ES;         // one K or V tile of a step
-    static constexpr int kStage = 2 * kTile;
     static constexpr int kChunkElems = 128 / ES;        // elements per 128-byte swizzle row
     static constexpr int kNChunk = kD * ES / 128;       // 128-byte chunks along d
     static constexpr int kChunkBytes = kST * 128;       // one chunk column of a K or V tile
@@ -83,24 +94,28 @@ struct Geo {
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
     static constexpr float kTau = ES == 1 ? 2.f : 8.f;      // lazy-rescale margin (log2 units)
-    static constexpr float kPScale = ES == 1 ? 64.f : 1.f;  // E4M3 P = 64 p, p <= 2^kTau
+    // E4M3 P is stored as 2^kPLog2 p (p <= 2^kTau, so at most 256 < 448); the row sum carries
+    // the same factor, which cancels in O / l
+    static constexpr float kPLog2 = ES == 1 ? 6.f : 0.f;
 };
 
 struct SmemLayout {
-    uint32_t stages, q, bars, meta, xch, qsc, misc, total;
+    uint32_t kst, vst, q, bars, meta, xch, qsc, misc, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int es, int n_stages, int Hkv) {
+__host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv) {
     SmemLayout L;
     uint32_t off = 0;
-    L.stages = off;
-    off += (uint32_t)n_stages * 2u * kST * kD * es;
+    L.kst = off;
+    off += (uint32_t)nsk * kST * kD * es;
+    L.vst = off;
+    off += (uint32_t)nsv * kST * kD * es;
     L.q = off;
     if (es == 4) off += (uint32_t)kRows * kD * es;  // fp32 Q stays in shared memory
     L.bars = off;
-    off += 8u * (2u * n_stages + 12u);
+    off += 8u * (2u * (nsk + nsv) + 12u);
     L.meta = off;
-    off += (uint32_t)sizeof(StageMeta) * n_stages;
+    off += (uint32_t)sizeof(StageMeta) * nsv;
     L.xch = off;
     off += 2u * kRows * 2u * 4u;
     L.qsc = off;
@@ -111,15 +126,23 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int n_stages, int Hkv)
     return L;
 }
 
-// barrier block
-__device__ __forceinline__ uint32_t bar_full(uint32_t b, int s) { return b + 8u * s; }
-__device__ __forceinline__ uint32_t bar_empty(uint32_t b, int s, int ns) { return b + 8u * (ns + s); }
-__device__ __forceinline__ uint32_t bar_sfull(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + i); }
-__device__ __forceinline__ uint32_t bar_sfree(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 2 + i); }
-__device__ __forceinline__ uint32_t bar_pfull(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 4 + i); }
-__device__ __forceinline__ uint32_t bar_pvdone(uint32_t b, int i, int ns) { return b + 8u * (2 * ns + 6 + i); }
-__device__ __forceinline__ uint32_t bar_qfull(uint32_t b, int ns) { return b + 8u * (2 * ns + 8); }
-__device__ __forceinline__ uint32_t bar_drain(uint32_t b, int ns) { return b + 8u * (2 * ns + 9); }
+// barrier block: K ring full/empty, V ring full/empty, then the fixed barriers
+struct Bars {
+    uint32_t base;
+    int nsk, nsv;
+    __device__ __forceinline__ uint32_t kfull(int s) const { return base + 8u * s; }
+    __device__ __forceinline__ uint32_t kempty(int s) const { return base + 8u * (nsk + s); }
+    __device__ __forceinline__ uint32_t vfull(int s) const { return base + 8u * (2 * nsk + s); }
+    __device__ __forceinline__ uint32_t vempty(int s) const { return base + 8u * (2 * nsk + nsv + s); }
+    __device__ __forceinline__ uint32_t fixed(int i) const { return base + 8u * (2 * (nsk + nsv) + i); }
+    __device__ __forceinline__ uint32_t sfull(int i) const { return fixed(i); }
+    __device__ __forceinline__ uint32_t sfree(int i) const { return fixed(2 + i); }
+    __device__ __forceinline__ uint32_t pfull(int i) const { return fixed(4 + i); }
+    __device__ __forceinline__ uint32_t pvdone(int i) const { return fixed(6 + i); }
+    __device__ __forceinline__ uint32_t qfull() const { return fixed(8); }
+    __device__ __forceinline__ uint32_t drain() const { return fixed(9); }
+    __device__ __forceinline__ uint32_t drain2() const { return fixed(10); }
+};
 
 struct Item {
     int h, bi, ub, nU, nsteps;
@@ -186,10 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(ES, p.n_stages, p.Hkv);
-    const int NS = p.n_stages;
+    const SmemLayout L = smem_layout(ES, p.nsk, p.nsv, p.Hkv);
+    const int NSK = p.nsk, NSV = p.nsv;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bars = sbase + L.bars;
+    const Bars B{sbase + L.bars, NSK, NSV};
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L.meta);
     float* xch = reinterpret_cast<float*>(smem + L.xch);
     float* qsc = reinterpret_cast<float*>(smem + L.qsc);
@@ -201,18 +224,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(bar_full(bars, s), 1);
-            mbar_init(bar_empty(bars, s, NS), 1);
+        for (int s = 0; s < NSK; ++s) {
+            mbar_init(B.kfull(s), 1);
+            mbar_init(B.kempty(s), 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(B.vfull(s), 1);
+            mbar_init(B.vempty(s), 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_sfull(bars, i, NS), 1);
-            mbar_init(bar_sfree(bars, i, NS), 128);
-            mbar_init(bar_pfull(bars, i, NS), 128);
-            mbar_init(bar_pvdone(bars, i, NS), 1);
+            mbar_init(B.sfull(i), 1);
+            mbar_init(B.sfree(i), 4);  // one arrive per softmax warp
+            mbar_init(B.pfull(i), 4);
+            mbar_init(B.pvdone(i), 1);
         }
-        mbar_init(bar_qfull(bars, NS), 256);
-        mbar_init(bar_drain(bars, NS), 1);
+        mbar_init(B.qfull(), 8);
+        mbar_init(B.drain(), 1);
+        mbar_init(B.drain2(), 1);
         fence_mbar_init();
         *abort_flag = 0;
         int acc = 0;
@@ -227,10 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         nb_prefix[p.Hkv] = acc;
     }
-    if (threadIdx.x == kProducerWarp * 32) {
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-    }
+    if (threadIdx.x == kProducerWarp * 32) prefetch_tensormap(&tmK);
+    if (threadIdx.x == kVProducerWarp * 32) prefetch_tensormap(&tmV);
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
         tmem_relinquish();
@@ -241,8 +267,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_items = nb_prefix[p.Hkv];
 
-    if (warp == kProducerWarp) {
-        // ============================================================ producer (whole warp)
+    if (warp == kProducerWarp || warp == kVProducerWarp) {
+        // ============================================================ producers (whole warp each)
+        // Both walk the same bundles and pages; the K warp fills the K ring, the V warp the
+        // V ring and the step metadata (indexed by V slot: it is read by the softmax of the
+        // step, which precedes the step's O update and so the slot's release).
+        const bool isV = warp == kVProducerWarp;
+        const int NR = isV ? NSV : NSK;
+        const CUtensorMap* tm = isV ? &tmV : &tmK;
+        const uint32_t ring = sbase + (isV ? L.vst : L.kst);
         int gs = 0;
         bool ok = true;
         for (int rnd = 0; ok; ++rnd) {
@@ -257,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 mk = make_uint4(0, 0, 0, 0);
                 if (idx < it.nU) {
                     u = p.union_pages[it.ub + idx];
-                    mk = reinterpret_cast<const uint4*>(p.row_mask)[it.ub + idx];
+                    if (isV) mk = reinterpret_cast<const uint4*>(p.row_mask)[it.ub + idx];
                     if (u < 0 || u >= p.num_logical_pages) {
                         atomicOr(p.err, QUP_ERR_PAGE_ID);
                         u = 0;
@@ -273,11 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ecnt = min(32, n_ent - e0);
                 const int nst = SPP > 1 ? ecnt * SPP : ecnt / PPS;
                 for (int k = 0; k < nst; ++k, ++gs) {
-                    const int slot = gs % NS;
+                    const int slot = gs % NR;
                     int okv = 0;
                     if (lane == 0)
-                        okv = mbar_wait(bar_empty(bars, slot, NS), ((gs / NS) & 1) ^ 1, abort_flag, p.err,
-                                        QUP_ERR_TIMEOUT, lim);
+                        okv = mbar_wait(isV ? B.vempty(slot) : B.kempty(slot), ((gs / NR) & 1) ^ 1, abort_flag,
+                                        p.err, QUP_ERR_TIMEOUT, lim);
                     ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
                     if (!ok) break;
                     const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
@@ -287,35 +320,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < PPS; ++q) {
                         const int src = SPP > 1 ? (k / SPP) : (k * PPS + q);
-                        const int uq = __shfl_sync(0xffffffffu, u, src);
                         ph[q] = __shfl_sync(0xffffffffu, phys, src);
-                        const uint32_t m0 = __shfl_sync(0xffffffffu, mk.x, src);
-                        const uint32_t m1 = __shfl_sync(0xffffffffu, mk.y, src);
-                        const uint32_t m2 = __shfl_sync(0xffffffffu, mk.z, src);
-                        const uint32_t m3 = __shfl_sync(0xffffffffu, mk.w, src);
-                        if (issue) {
-                            StageMeta& m = meta[slot];
-                            m.upage[q] = uq;
-                            m.mask[q][0] = m0;
-                            m.mask[q][1] = m1;
-                            m.mask[q][2] = m2;
-                            m.mask[q][3] = m3;
-                            m.tok0 = tok0;
+                        if (isV) {
+                            const int uq = __shfl_sync(0xffffffffu, u, src);
+                            const uint32_t m0 = __shfl_sync(0xffffffffu, mk.x, src);
+                            const uint32_t m1 = __shfl_sync(0xffffffffu, mk.y, src);
+                            const uint32_t m2 = __shfl_sync(0xffffffffu, mk.z, src);
+                            const uint32_t m3 = __shfl_sync(0xffffffffu, mk.w, src);
+                            if (issue) {
+                                StageMeta& m = meta[slot];
+                                m.upage[q] = uq;
+                                m.mask[q][0] = m0;
+                                m.mask[q][1] = m1;
+                                m.mask[q][2] = m2;
+                                m.mask[q][3] = m3;
+                                m.tok0 = tok0;
+                            }
                         }
                     }
                     if (issue) {
                         // the arrive releases the metadata stores; the copies complete the phase
-                        const uint32_t fb = bar_full(bars, slot);
-                        mbar_arrive_expect_tx(fb, G::kStage);
-                        const uint32_t kdst = sbase + L.stages + (uint32_t)slot * G::kStage;
-                        const uint32_t vdst = kdst + G::kTile;
+                        const uint32_t fb = isV ? B.vfull(slot) : B.kfull(slot);
+                        mbar_arrive_expect_tx(fb, G::kTile);
+                        const uint32_t dst = ring + (uint32_t)slot * G::kTile;
 #pragma unroll
                         for (int q = 0; q < PPS; ++q) {
 #pragma unroll
                             for (int c = 0; c < G::kNChunk; ++c) {
                                 const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * BOXR) * 128u;
-                                tma_load_4d(kdst + off, &tmK, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
-                                tma_load_4d(vdst + off, &tmV, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
+                                tma_load_4d(dst + off, tm, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
                             }
                         }
                     }
@@ -323,21 +356,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        // every issued load lands before the CTA may exit: the last NS stages
+        // every issued load lands before the CTA may exit: the last NR stages of this ring
         if (lane == 0) {
-            for (int i = max(0, gs - NS); i < gs; ++i) {
+            for (int i = max(0, gs - NR); i < gs; ++i) {
                 if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
-                mbar_wait_drain(bar_full(bars, i % NS), (i / NS) & 1, lim);
+                mbar_wait_drain(isV ? B.vfull(i % NR) : B.kfull(i % NR), (i / NR) & 1, lim);
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // ============================================================ MMA issuer (whole warp, one elected lane)
-        // Issue order per bundle: S(s) then O(s - LAG).  With the two warpgroups half a
-        // period apart, the events arrive as S-free(g), P-ready(g-1), S-free(g+1),
-        // P-ready(g), ..., so LAG = 3 issues every S as soon as its buffer is read and
-        // every O update as soon as its P is written.  S(s) needs the stage of step s,
-        // whose previous use was released by O(s - NS): LAG <= NS - 1.
+    } else if (warp == kMmaWarp || warp == kPvWarp) {
+        // ============================================================ MMA issuers (whole warp, one elected lane)
+        // Two in-order streams, one warp each (on different SM sub-partitions, so each keeps
+        // its share of issue slots next to the busy softmax warps):
+        //   S warp:  S(g) = Q K^T  needs K tile g and S buffer g & 1, released by the softmax
+        //            of step g - 2; commits S-full(b) and the K slot.
+        //   PV warp: O_b += P_b V  needs P(g) and V tile g; commits PV-done(b) and the V slot.
+        // The PV warp needs no Q barrier: P(g) of a bundle's first step is written after the
+        // softmax warps have finished the previous bundle's epilogue (its reads of O).
+        const bool isS = warp == kMmaWarp;
         const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, kST, kRows);
         const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
         // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
@@ -345,27 +381,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
         constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
         const uint32_t qbase = sbase + L.q;
-        const int LAG = NS >= 4 ? 3 : NS - 1;
         int gs = 0, item_no = 0;
+        int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slot and phase of step gs
         bool ok = true;
         for (int rnd = 0; ok; ++rnd) {
             const int f = item_at(p, rnd, n_items);
             if (f == -1) break;
             if (f < 0) continue;
             const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
-            ok = warp_ok(mbar_wait(bar_qfull(bars, NS), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-            if (!ok) break;
-            tc_fence_after();
-            for (int s = 0; s < it.nsteps + LAG && ok; ++s) {
-                if (s < it.nsteps) {  // ---- S(g) = Q K^T into S_b
-                    const int g = gs + s, slot = g % NS, b = g & 1;
-                    ok = warp_ok(mbar_wait(bar_full(bars, slot), (g / NS) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
-                                           lim) &&
-                                 (g < 2 || mbar_wait(bar_sfree(bars, b, NS), ((g - 2) >> 1) & 1, abort_flag, p.err,
-                                                     QUP_ERR_TIMEOUT, lim)));  // softmax of g-2 has read S_b
+            if (isS) {
+                ok = warp_ok(mbar_wait(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                if (!ok) break;
+                tc_fence_after();
+                for (int s = 0; s < it.nsteps; ++s) {
+                    const int g = gs + s, b = g & 1;
+                    ok = warp_ok(mbar_wait(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                 (g < 2 || mbar_wait(B.sfree(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
+                                                     QUP_ERR_TIMEOUT, lim)));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t kdesc = smem_desc(sbase + L.stages + (uint32_t)slot * G::kStage, 16, 1024, 2);
+                    const uint64_t kdesc = smem_desc(sbase + L.kst + (uint32_t)ks * G::kTile, 16, 1024, 2);
                     const uint64_t qdesc = smem_desc(qbase, 16, 1024, 2);
                     if (elect_one_sync()) {
 #pragma unroll
@@ -379,19 +414,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tc_mma<G::kKind>(tmem + 64u * b, qdesc + qoff, kdesc + koff, idesc_s, k > 0);
                             }
                         }
-                        tc_commit(bar_sfull(bars, b, NS));
+                        tc_commit(B.sfull(b));
+                        tc_commit(B.kempty(ks));
                     }
                     __syncwarp();
+                    if (++ks == NSK) {
+                        ks = 0;
+                        kph ^= 1;
+                    }
                 }
-                if (s >= LAG) {  // ---- O_b += P_b V for step g = s - LAG
-                    const int sl = s - LAG, g = gs + sl, slot = g % NS, b = g & 1;
-                    ok = warp_ok(mbar_wait(bar_pfull(bars, b, NS), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
-                                           lim));
+            } else {
+                for (int s = 0; s < it.nsteps; ++s) {
+                    const int g = gs + s, b = g & 1;
+                    ok = warp_ok(mbar_wait(B.pfull(b), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                 mbar_wait(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t vdesc = smem_desc(sbase + L.stages + (uint32_t)slot * G::kStage + G::kTile,
+                    const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
                                                      (uint32_t)G::kChunkBytes, vsbo, vlayout);
-                    const bool acc0 = sl >= 2;  // steps 0 and 1 of a bundle open O_0 / O_1
+                    const bool acc0 = s >= 2;  // steps 0 and 1 of a bundle open O_0 / O_1
                     if (elect_one_sync()) {
 #pragma unroll
                         for (int k = 0; k < G::kNumMmaPV; ++k) {
@@ -399,19 +440,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_mma_ts<G::kKind>(tmem + G::kColO + 128u * b, tmem + G::kColP + G::kPCols * b + 8u * k,
                                                 vdesc + ((k * G::kMmaK * 128) >> 4), idesc_o, acc0 || k > 0);
                         }
-                        tc_commit(bar_pvdone(bars, b, NS));
-                        tc_commit(bar_empty(bars, slot, NS));
+                        tc_commit(B.pvdone(b));
+                        tc_commit(B.vempty(vs));
                     }
                     __syncwarp();
+                    if (++vs == NSV) {
+                        vs = 0;
+                        vph ^= 1;
+                    }
                 }
             }
             gs += it.nsteps;
             ++item_no;
         }
-        // every issued MMA completes before TMEM is freed
-        if (elect_one_sync()) tc_commit(bar_drain(bars, NS));
+        // every MMA this warp issued completes before TMEM is freed
+        const uint32_t dbar = isS ? B.drain() : B.drain2();
+        if (elect_one_sync()) tc_commit(dbar);
         __syncwarp();
-        mbar_wait_drain(bar_drain(bars, NS), 0, lim);
+        mbar_wait_drain(dbar, 0, lim);
         __syncwarp();
     } else {
         // ============================================================ softmax / epilogue (256 threads)
@@ -504,7 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (G::kQTmem) tmem_wait_st();
             }
             tc_fence_before();
-            mbar_arrive(bar_qfull(bars, NS));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(B.qfull());
             float cs = p.scale_log2;  // score scale (log2 domain) of this row
             if constexpr (ES == 1) {
                 bar_sync(1, 256);  // qsc written by warpgroup 0
@@ -516,28 +563,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < it.nsteps; ++s) {
                 const int gstep = gs + s;
                 if ((gstep & 1) != wg) continue;  // the other warpgroup's step
-                const int slot = gstep % NS;
+                const int slot = gstep % NSV;  // V slot: V tile and step metadata
                 if (ok)
-                    ok = warp_ok(mbar_wait(bar_full(bars, slot), (gstep / NS) & 1, abort_flag, p.err,
+                    ok = warp_ok(mbar_wait(B.vfull(slot), (gstep / NSV) & 1, abort_flag, p.err,
                                            QUP_ERR_TIMEOUT, lim) &&
-                                 mbar_wait(bar_sfull(bars, wg, NS), (gstep >> 1) & 1, abort_flag, p.err,
+                                 mbar_wait(B.sfull(wg), (gstep >> 1) & 1, abort_flag, p.err,
                                            QUP_ERR_TIMEOUT, lim));
                 if (!ok) continue;
                 tc_fence_after();
                 uint32_t sv[kST];
                 tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(sv));
                 tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                // while S is in flight: this warpgroup's previous O update must be done before
-                // O is rescaled and before P_wg is overwritten (usually long done)
-                const bool pv_ok = gstep < 2 || mbar_wait(bar_pvdone(bars, wg, NS), ((gstep - 2) >> 1) & 1, abort_flag,
-                                                          p.err, QUP_ERR_TIMEOUT, lim);
                 const StageMeta& mt = meta[slot];
                 const int tok0 = mt.tok0;
-                // cache slots at or past kv_len may hold non-finite bytes: zero those V rows
-                if (r < kST) {
+                // a page of the step that reaches kv_len: its cache slots at or past kv_len may
+                // hold non-finite bytes, so those V rows are zeroed and the step's scores masked
+                bool tail = false;
+#pragma unroll
+                for (int q = 0; q < PPS; ++q) tail |= mt.upage[q] * T + tok0 + BOXR > p.kv_len;
+                if (tail && r < kST) {
                     const int q = r / BOXR;
                     if (mt.upage[q] * T + tok0 + (r - q * BOXR) >= p.kv_len) {
-                        uint8_t* vt = smem + L.stages + (uint32_t)slot * G::kStage + G::kTile;
+                        uint8_t* vt = smem + L.vst + (uint32_t)slot * G::kTile;
 #pragma unroll
                         for (int c = 0; c < G::kNChunk; ++c)
 #pragma unroll
@@ -549,25 +596,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // row r sees token j of page q iff the page is in its own TopK row
                 // (bit r of the page's mask) and the token's position is < vis_end
                 int lim_q[PPS];
-                bool live = false;
+                bool live = false, partial = false;
 #pragma unroll
                 for (int q = 0; q < PPS; ++q) {
                     const bool mine = (mt.mask[q][r >> 5] >> (r & 31)) & 1u;
                     lim_q[q] = mine ? max(0, min(BOXR, vis_end - (mt.upage[q] * T + tok0))) : 0;
                     live |= lim_q[q] > 0;
+                    partial |= lim_q[q] > 0 && lim_q[q] < BOXR;
                 }
                 tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(bar_sfree(bars, wg, NS));  // S_wg may now be overwritten by S(gstep + 2)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(B.sfree(wg));  // S_wg may now be overwritten by S(gstep + 2)
                 const bool warp_live = __any_sync(0xffffffffu, live);
+                // Fast path (the usual step: one whole page, every row sees all of it or none of
+                // it): the max is taken over the raw scores (cs > 0) and each exponent is one FMA.
+                // Otherwise every score is scaled and masked first.
+                const bool slow = PPS > 1 || tail || __any_sync(0xffffffffu, partial);
                 float mloc = kNegInf;
                 if (warp_live) {
+                    float mx[8];
 #pragma unroll
-                    for (int j = 0; j < kST; ++j) {
-                        const float v = (j % BOXR) < lim_q[j / BOXR] ? __uint_as_float(sv[j]) * cs : kNegInf;
-                        sv[j] = __float_as_uint(v);
-                        mloc = fmaxf(mloc, v);
+                    for (int k = 0; k < 8; ++k) mx[k] = kNegInf;
+                    if (!slow) {
+#pragma unroll
+                        for (int j = 0; j < kST; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kST; ++j) {
+                            const float v = (j % BOXR) < lim_q[j / BOXR] ? __uint_as_float(sv[j]) * cs : kNegInf;
+                            sv[j] = __float_as_uint(v);
+                            mx[j & 7] = fmaxf(mx[j & 7], v);
+                        }
                     }
+                    const float m4 = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                    mloc = slow ? m4 : (live ? m4 * cs : kNegInf);
                 }
                 // lazy running max: raise it only when a score exceeds it by more than kTau
                 const bool need = mloc > m_used + G::kTau;
@@ -577,44 +641,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_used = mloc;
                     lsum *= alpha;
                 }
-                const float msafe = m_used == kNegInf ? 0.f : m_used;
                 uint32_t pk[G::kPCols];
                 if (warp_live) {
-                    float part0 = 0.f, part1 = 0.f;
+                    // p = 2^(x - m + kPLog2); a fast-path row that sees nothing gets x - inf = -inf
+                    const float xs = slow ? 1.f : cs;
+                    const float moff = (!slow && !live) ? __int_as_float(0x7f800000)
+                                                        : (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
+                    float part[4] = {0.f, 0.f, 0.f, 0.f};
                     if constexpr (ES == 2) {
 #pragma unroll
                         for (int j = 0; j < kST; j += 2) {
-                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                            const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
-                            part0 += p0;
-                            part1 += p1;
+                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
+                            const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -moff));
+                            part[(j >> 1) & 3] += p0 + p1;
                             pk[j / 2] = pack_bf16x2(p0, p1);
                         }
                     } else if constexpr (ES == 4) {
 #pragma unroll
                         for (int j = 0; j < kST; ++j) {
-                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                            if (j & 1) part1 += p0;
-                            else part0 += p0;
+                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
+                            part[j & 3] += p0;
                             pk[j] = __float_as_uint(p0);
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < kST; j += 4) {
-                            const float p0 = ex2(__uint_as_float(sv[j]) - msafe);
-                            const float p1 = ex2(__uint_as_float(sv[j + 1]) - msafe);
-                            const float p2 = ex2(__uint_as_float(sv[j + 2]) - msafe);
-                            const float p3 = ex2(__uint_as_float(sv[j + 3]) - msafe);
-                            part0 += p0 + p2;
-                            part1 += p1 + p3;
-                            pk[j / 4] = pack_e4m3x4(p0 * G::kPScale, p1 * G::kPScale, p2 * G::kPScale, p3 * G::kPScale);
+                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
+                            const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -moff));
+                            const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -moff));
+                            const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -moff));
+                            part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
+                            pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
                         }
                     }
-                    lsum += part0 + part1;
+                    lsum += (part[0] + part[1]) + (part[2] + part[3]);
                 } else {
 #pragma unroll
                     for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
                 }
+                // this warpgroup's previous O update must be done before O is rescaled and
+                // P_wg overwritten; it was issued when the previous step's P was stored, a
+                // whole softmax ago, so this rarely waits
+                const bool pv_ok = gstep < 2 || mbar_wait(B.pvdone(wg), ((gstep - 2) >> 1) & 1, abort_flag,
+                                                          p.err, QUP_ERR_TIMEOUT, lim);
                 ok = warp_ok(pv_ok);
                 if (!ok) continue;
                 tc_fence_after();
@@ -631,16 +700,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_st_n<G::kPCols>(p_addr, pk);
                 tmem_wait_st();
-                fence_proxy_async_smem();  // zeroed V rows -> async proxy
+                if (tail) fence_proxy_async_smem();  // zeroed V rows -> async proxy
                 tc_fence_before();
-                mbar_arrive(bar_pfull(bars, wg, NS));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(B.pfull(wg));
                 ++mine_steps;
             }
             // ---- epilogue: merge the two partial results; O / l -> O[qid][head][:]
             if (ok && mine_steps > 0) {
                 int last = gs + it.nsteps - 1;
                 if ((last & 1) != wg) --last;
-                ok = warp_ok(mbar_wait(bar_pvdone(bars, wg, NS), (last >> 1) & 1, abort_flag, p.err,
+                ok = warp_ok(mbar_wait(B.pvdone(wg), (last >> 1) & 1, abort_flag, p.err,
                                        QUP_ERR_TIMEOUT, lim));
             }
             gs += it.nsteps;
@@ -655,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float f1 = (m1 == kNegInf) ? 0.f : ex2(m1 - M);
             const float Lsum = l0 * f0 + l1 * f1;
             float vsc = 1.f;
-            if constexpr (ES == 1) vsc = p.v_scale[it.h] * (1.f / G::kPScale);
+            if constexpr (ES == 1) vsc = p.v_scale[it.h];
             const float inv = Lsum > 0.f ? vsc / Lsum : 0.f;
             const float g0 = f0 * inv, g1 = f1 * inv;
             const bool use0 = m0 != kNegInf && Lsum > 0.f, use1 = m1 != kNegInf && Lsum > 0.f;
@@ -688,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (wg == 0 && p.lse != nullptr)
                     p.lse[(size_t)qid * p.Hq + head] =
-                        Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : kNegInf;
+                        Lsum > 0.f ? (M + __log2f(Lsum) - G::kPLog2) * 0.69314718055994531f : kNegInf;
             }
             tc_fence_before();
             bar_sync(1, 256);  // O_0, O_1 and Q read before the next bundle overwrites them
@@ -702,9 +772,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-size_t attn_smem_bytes(int es, int n_stages, int Hkv) { return smem_layout(es, n_stages, Hkv).total; }
+size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv) { return smem_layout(es, nsk, nsv, Hkv).total; }
 
-size_t attn_stage_bytes(int es) { return 2u * kST * kD * es; }
+size_t attn_tile_bytes(int es) { return (size_t)kST * kD * es; }
 
 template <int ES, int T>
 static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p, int grid,
