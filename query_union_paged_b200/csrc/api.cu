@@ -65,7 +65,7 @@ int device_state(DevState** out) {
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct GroupWs {
-    size_t rowbits, usize, wtot, wcnt, total;
+    size_t rowbits, usize, wtot, wcnt, fwcnt, fstatus, total;
 };
 
 GroupWs group_ws_layout(int Hq, int Hkv, int Nq, int NW, int nwin) {
@@ -79,6 +79,12 @@ GroupWs group_ws_layout(int Hq, int Hkv, int Nq, int NW, int nwin) {
     off = align256(off + sizeof(int32_t) * (size_t)Hkv * nwin);
     w.wcnt = off;
     off = align256(off + sizeof(int32_t) * 3 * (size_t)Hkv * nwin);
+    // fused path: per-window counters of both kernels, look-back status words of both
+    // kernels and the bundle kernel's completion count (windows: at most Nq per head)
+    w.fwcnt = off;
+    off = align256(off + sizeof(int32_t) * 5 * (size_t)Hkv * std::max(Nq, 1));
+    w.fstatus = off;
+    off = align256(off + sizeof(uint64_t) * 2 * (size_t)Hkv * std::max(Nq, 1) + 16);
     w.total = off;
     return w;
 }
@@ -93,6 +99,14 @@ void bundle_geometry(int g, int max_group, int bundle_window, int* RS, int* slot
     int wb = bundle_window > 0 ? bundle_window : 64;
     wb = (wb / *slots) * *slots;
     *WB = wb < *slots ? *slots : wb;
+}
+
+// The fused kernels keep a whole window in shared memory: they run when it fits.
+bool fused_group_ok(int g, int NW, int W, const DevState* ds) {
+    return W <= 256 && qup::fused_group_smem(W, g, NW) <= (size_t)ds->smem_optin;
+}
+bool fused_bundle_ok(int NW, int WB, int Hkv, const DevState* ds) {
+    return WB <= 256 && qup::fused_bundle_smem(WB, NW, Hkv) <= (size_t)ds->smem_optin;
 }
 
 int check_group_args(int Hq, int Hkv, int Nq, int K, int P, int max_group, int window) {
@@ -132,8 +146,13 @@ int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages
 
 namespace {
 
+// gbits_ready: the group bitsets are already in the workspace (written by the fused group
+// kernel, which also zeroed the bundle status words: they follow its own, at
+// fused_status_offset words into the status region).
+// max_groups: an upper bound of the groups of one KV head (Nq for any partition).
 int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group, void* ws,
-                DevState* ds, cudaStream_t st) {
+                DevState* ds, cudaStream_t st, bool gbits_ready = false, size_t fused_status_offset = 0,
+                int max_groups = -1) {
     const int gq = Hq / Hkv;
     int RS, slots, WB;
     bundle_geometry(gq, max_group, g->bundle_window, &RS, &slots, &WB);
@@ -158,7 +177,7 @@ int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, i
     a.RS = RS;
     a.slots = slots;
     a.WB = WB;
-    a.nwin = (Nq + WB - 1) / WB;
+    a.nwin = ((max_groups >= 0 ? std::min(max_groups, Nq) : Nq) + WB - 1) / WB;
     a.n_groups = g->n_groups;
     a.group_ptr = g->group_ptr;
     a.members = g->members;
@@ -181,6 +200,20 @@ int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, i
     a.bundle_order = g->bundle_order;
     a.err = ds->err;
     a.sms = ds->sms;
+    if (fused_bundle_ok(NW, WB, Hkv, ds)) {
+        // status words of the bundle windows (after those of the group windows, if any) and
+        // the completion count start at zero
+        uint64_t* status = reinterpret_cast<uint64_t*>(base + L.fstatus) + fused_status_offset;
+        unsigned* done = reinterpret_cast<unsigned*>(status + (size_t)Hkv * a.nwin);
+        int32_t* wcnt = reinterpret_cast<int32_t*>(base + L.fwcnt) + 4 * (size_t)Hkv * std::max(Nq, 1);
+        if (!gbits_ready) {
+            if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * a.nwin + sizeof(unsigned), st) !=
+                cudaSuccess)
+                return QUP_ERR_CUDA;
+        }
+        if (!gbits_ready && qup::launch_gbits(a, st) != cudaSuccess) return QUP_ERR_CUDA;
+        return qup::launch_bundles_fused(a, wcnt, status, done, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+    }
     return qup::launch_bundles(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
 }
 
@@ -261,6 +294,23 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
     a.err = ds->err;
     a.sms = ds->sms;
     if (Ksel == 0) a.topk = nullptr;
+    int RS, slots, WB;
+    bundle_geometry(Hq / Hkv, max_group, out->bundle_window, &RS, &slots, &WB);
+    if (fused_group_ok(Hq / Hkv, NW, window, ds) && fused_bundle_ok(NW, WB, Hkv, ds)) {
+        // one memset zeroes the status words of both kernels and the completion count.  Every
+        // window but the last yields window / max_group groups (groups are always filled).
+        const int max_groups = std::min(Nq, nwin * ((window + max_group - 1) / max_group));
+        const int nwinB = (max_groups + WB - 1) / WB;
+        uint64_t* status = reinterpret_cast<uint64_t*>(base + L.fstatus);
+        if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * (nwin + nwinB) + sizeof(unsigned), st) !=
+            cudaSuccess)
+            return QUP_ERR_CUDA;
+        if (qup::launch_group_fused(a, a.rowbits, reinterpret_cast<int32_t*>(base + L.fwcnt), status, st) !=
+            cudaSuccess)
+            return QUP_ERR_CUDA;
+        return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st, true, (size_t)Hkv * nwin,
+                           max_groups);
+    }
     if (qup::launch_group(a, st) != cudaSuccess) return QUP_ERR_CUDA;
     return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st);
 }
@@ -396,3 +446,32 @@ int qup_num_sms(void) {
 }
 
 }  // extern "C"
+
+namespace qup {
+
+cudaError_t ensure_smem_attr(const void* fn, size_t smem) {
+    struct Entry {
+        int dev;
+        const void* fn;
+        size_t smem;
+    };
+    static std::mutex mu;
+    static Entry table[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n; ++i)
+        if (table[i].dev == dev && table[i].fn == fn) {
+            if (table[i].smem >= smem) return cudaSuccess;
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess) table[i].smem = smem;
+            return e;
+        }
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && n < 256) table[n++] = Entry{dev, fn, smem};
+    return e;
+}
+
+}  // namespace qup

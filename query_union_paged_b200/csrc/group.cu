@@ -124,11 +124,13 @@ __global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restr
             if (!((taken >> k) & 1u)) my = min(my, (unsigned)(lane + 32 * k));
         const unsigned seed = __reduce_min_sync(0xffffffffu, my);
         if (seed == 0xffffffffu) break;
-        if ((int)(seed & 31u) == lane) taken |= 1u << (seed >> 5);
+        unsigned ing = 0;  // bit k: candidate lane + 32 k is in this group
+        if ((int)(seed & 31u) == lane) {
+            taken |= 1u << (seed >> 5);
+            ing |= 1u << (seed >> 5);
+        }
         for (int wd = lane; wd < NW; wd += 32) U[wd] = S[seed * NWp + wd];
         __syncwarp();
-        int grp[8];
-        grp[0] = (int)seed;
         int cnt = 1, sum_s = ssize[seed];
         while (cnt < max_group) {
             unsigned key = 0xffffffffu;
@@ -143,27 +145,29 @@ __global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restr
             const unsigned best = __reduce_min_sync(0xffffffffu, key);
             if (best == 0xffffffffu) break;
             const int c = (int)(best & 511u);
-            if ((c & 31) == lane) taken |= 1u << (c >> 5);
+            if ((c & 31) == lane) {
+                taken |= 1u << (c >> 5);
+                ing |= 1u << (c >> 5);
+            }
             __syncwarp();
             for (int wd = lane; wd < NW; wd += 32) U[wd] |= S[c * NWp + wd];
             __syncwarp();
-            grp[cnt++] = c;
+            ++cnt;
             sum_s += ssize[c];
         }
         int us = 0;
         for (int wd = lane; wd < NW; wd += 32) us += __popc(U[wd]);
         us = __reduce_add_sync(0xffffffffu, us);
-        for (int a = 1; a < cnt; ++a) {  // ascending members
-            const int v = grp[a];
-            int b = a - 1;
-            while (b >= 0 && grp[b] > v) {
-                grp[b + 1] = grp[b];
-                --b;
+        {  // members in ascending local ID (candidate lane + 32 k: k-major, then lane)
+            const unsigned lt = (1u << lane) - 1u;
+            int base = 0;
+            for (int k = 0; k < CPL; ++k) {
+                const unsigned bk = __ballot_sync(0xffffffffu, (ing >> k) & 1u);
+                if ((ing >> k) & 1u) members[(size_t)h * Nq + w0 + mpos + base + __popc(bk & lt)] = w0 + lane + 32 * k;
+                base += __popc(bk);
             }
-            grp[b + 1] = v;
         }
         if (lane == 0) {
-            for (int m = 0; m < cnt; ++m) members[(size_t)h * Nq + w0 + mpos + m] = w0 + grp[m];
             group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = w0 + mpos;
             ws_usize[(size_t)h * Nq + gbase + ngw] = us;
         }
@@ -466,27 +470,244 @@ size_t group_greedy_smem(int W, int NW) {
     return sizeof(uint32_t) * ((size_t)W * NWp + NWp + W);
 }
 
+// One warp per TopK row without shared memory: lane l builds words l, l + 32, ...
+// of the row's page bitset while the row's entries are broadcast one by one
+// (K <= 64 entries, at most 32 * kRbWords words).
+constexpr int kRbWords = 8;
+__global__ void __launch_bounds__(256) grp_rowbits_shfl_kernel(const int32_t* __restrict__ topk, int Hq, int Hkv,
+                                                                int Nq, int K, int P, int NW,
+                                                                uint32_t* __restrict__ rowbits,
+                                                                int64_t* __restrict__ counters, unsigned* err) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (blockIdx.x == 0)
+        for (int x = threadIdx.x; x < Hkv * 4; x += blockDim.x) counters[x] = 0;
+    const int g = Hq / Hkv;
+    const long long nrows = (long long)Hq * Nq;
+    for (long long row = (long long)blockIdx.x * 8 + warp; row < nrows; row += (long long)gridDim.x * 8) {
+        const int hq = (int)(row / Nq), i = (int)(row % Nq);
+        const int32_t* tr = topk + row * K;
+        uint32_t wb[kRbWords];
+#pragma unroll
+        for (int x = 0; x < kRbWords; ++x) wb[x] = 0u;
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            int e = k0 + lane < K ? tr[k0 + lane] : -1;
+            if (e != -1 && (e < 0 || e >= P)) {
+                atomicOr(err, QUP_ERR_PAGE_ID);
+                e = -1;
+            }
+            const int n = min(32, K - k0);
+            for (int t = 0; t < n; ++t) {
+                const int pe = __shfl_sync(0xffffffffu, e, t);
+                if (pe >= 0 && ((pe >> 5) & 31) == lane) {
+                    const int slot = pe >> 10;
+#pragma unroll
+                    for (int x = 0; x < kRbWords; ++x)
+                        if (x == slot) wb[x] |= 1u << (pe & 31);
+                }
+            }
+        }
+        const int h = hq / g, j = hq % g;
+        uint32_t* dst = rowbits + (((size_t)h * Nq + i) * g + j) * NW;
+#pragma unroll
+        for (int x = 0; x < kRbWords; ++x)
+            if (lane + 32 * x < NW) dst[lane + 32 * x] = wb[x];
+    }
+}
+
+// ------------------------------------------------------------------ register-resident greedy
+// The same greedy as grp_greedy_kernel for windows of at most 64 items whose sets
+// fit in NWR words: one warp per (window, KV head), lane l holds the sets of items
+// l and l + 32 in registers, so a pick is 2 x NWR and-not/popcounts per lane, one
+// warp min-reduction of the packed key (new_pages << 9 | local_id) and a shuffle
+// of the winner's set from its owner lane.  Members are kept as a 64-bit mask of
+// local IDs; each lane also flags which of its two items joined the current
+// group, and two ballots give every member its rank (ascending local ID).
+template <int NWR>
+__global__ void __launch_bounds__(128) grp_greedy_reg_kernel(const uint32_t* __restrict__ rowbits, int sets_per_item,
+                                                              int Hkv, int Nq, const int32_t* __restrict__ n_items_dev,
+                                                              int NW, int max_group, int W, int nwin,
+                                                              int32_t* __restrict__ group_ptr,
+                                                              int32_t* __restrict__ members,
+                                                              int32_t* __restrict__ n_groups,
+                                                              int32_t* __restrict__ ws_usize,
+                                                              int32_t* __restrict__ ws_wtot,
+                                                              int32_t* __restrict__ ws_wcnt,
+                                                              int64_t* __restrict__ out_count) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x * 4 + warp;
+    if (item >= nwin * Hkv) return;
+    const int h = item / nwin, w = item % nwin, g = sets_per_item;
+    const int n_items = n_items_dev ? n_items_dev[h] : Nq;
+    const int w0 = w * W, nw = max(0, min(W, n_items - w0));
+    if (nw == 0) {  // window past the head's last item: contributes nothing
+        if (lane == 0) {
+            const int f = h * nwin + w;
+            ws_wtot[f] = 0;
+            ws_wcnt[f * 3 + 0] = ws_wcnt[f * 3 + 1] = ws_wcnt[f * 3 + 2] = 0;
+            if (w == 0) {
+                n_groups[h] = 0;
+                group_ptr[(size_t)h * (Nq + 1)] = 0;
+                if (out_count) out_count[h * 2 + 1] = 0;
+            }
+        }
+        return;
+    }
+    constexpr unsigned kNone = 0xffffffffu;
+    uint32_t s0[NWR], s1[NWR], U[NWR];
+#pragma unroll
+    for (int x = 0; x < NWR; ++x) s0[x] = s1[x] = 0u;
+    const bool v0 = lane < nw, v1 = lane + 32 < nw;
+    if (v0) {
+        const uint32_t* src = rowbits + ((size_t)h * Nq + w0 + lane) * g * NW;
+        for (int j = 0; j < g; ++j)
+#pragma unroll
+            for (int x = 0; x < NWR; ++x)
+                if (x < NW) s0[x] |= src[(size_t)j * NW + x];
+    }
+    if (v1) {
+        const uint32_t* src = rowbits + ((size_t)h * Nq + w0 + lane + 32) * g * NW;
+        for (int j = 0; j < g; ++j)
+#pragma unroll
+            for (int x = 0; x < NWR; ++x)
+                if (x < NW) s1[x] |= src[(size_t)j * NW + x];
+    }
+    int sz0 = 0, sz1 = 0;
+#pragma unroll
+    for (int x = 0; x < NWR; ++x) {
+        sz0 += __popc(s0[x]);
+        sz1 += __popc(s1[x]);
+    }
+    const int edges = __reduce_add_sync(0xffffffffu, sz0 + sz1);  // invalid items hold empty sets
+    unsigned taken = (v0 ? 0u : 1u) | (v1 ? 0u : 2u);
+    const int gbase = w * (W / max_group);
+    int ngw = 0, mpos = 0, visits = 0, masked_q = 0;
+    while (true) {
+        const unsigned my = !(taken & 1u) ? (unsigned)lane : (!(taken & 2u) ? (unsigned)lane + 32u : kNone);
+        const unsigned seed = __reduce_min_sync(0xffffffffu, my);
+        if (seed == kNone) break;
+        int owner = (int)(seed & 31u), k = (int)(seed >> 5);
+        unsigned ing = 0;  // bit k: item lane + 32 k is in this group
+        if (lane == owner) {
+            taken |= 1u << k;
+            ing |= 1u << k;
+        }
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) U[x] = __shfl_sync(0xffffffffu, k ? s1[x] : s0[x], owner);
+        int sum_s = __shfl_sync(0xffffffffu, k ? sz1 : sz0, owner);
+        int cnt = 1;
+        while (cnt < max_group) {
+            unsigned key = kNone;
+            if (!(taken & 1u)) {
+                int nc = 0;
+#pragma unroll
+                for (int x = 0; x < NWR; ++x) nc += __popc(s0[x] & ~U[x]);
+                key = ((unsigned)nc << 9) | (unsigned)lane;
+            }
+            if (!(taken & 2u)) {
+                int nc = 0;
+#pragma unroll
+                for (int x = 0; x < NWR; ++x) nc += __popc(s1[x] & ~U[x]);
+                key = min(key, ((unsigned)nc << 9) | (unsigned)(lane + 32));
+            }
+            const unsigned best = __reduce_min_sync(0xffffffffu, key);
+            if (best == kNone) break;
+            const int c = (int)(best & 511u);
+            owner = c & 31;
+            k = c >> 5;
+            if (lane == owner) {
+                taken |= 1u << k;
+                ing |= 1u << k;
+            }
+#pragma unroll
+            for (int x = 0; x < NWR; ++x) U[x] |= __shfl_sync(0xffffffffu, k ? s1[x] : s0[x], owner);
+            sum_s += __shfl_sync(0xffffffffu, k ? sz1 : sz0, owner);
+            ++cnt;
+        }
+        int us = 0;
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) us += __popc(U[x]);
+        {  // members in ascending local ID: items 0..31 (k = 0) before 32..63 (k = 1)
+            const unsigned b0 = __ballot_sync(0xffffffffu, ing & 1u), b1 = __ballot_sync(0xffffffffu, ing & 2u);
+            const unsigned lt = (1u << lane) - 1u;
+            int32_t* dst = members + (size_t)h * Nq + w0 + mpos;
+            if (ing & 1u) dst[__popc(b0 & lt)] = w0 + lane;
+            if (ing & 2u) dst[__popc(b0) + __popc(b1 & lt)] = w0 + lane + 32;
+        }
+        if (lane == 0) {
+            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = w0 + mpos;
+            ws_usize[(size_t)h * Nq + gbase + ngw] = us;
+        }
+        mpos += cnt;
+        ++ngw;
+        visits += us;
+        masked_q += cnt * us - sum_s;
+    }
+    if (lane == 0) {
+        const int f = h * nwin + w;
+        ws_wtot[f] = visits;
+        ws_wcnt[f * 3 + 0] = visits;
+        ws_wcnt[f * 3 + 1] = masked_q;
+        ws_wcnt[f * 3 + 2] = edges;
+        if (w0 + nw == n_items) {  // the window holding the head's last item
+            n_groups[h] = gbase + ngw;
+            group_ptr[(size_t)h * (Nq + 1) + gbase + ngw] = w0 + mpos;
+            if (out_count) out_count[h * 2 + 1] = gbase + ngw;
+        }
+    }
+}
+
+// Greedy dispatch: the register kernel when the window holds at most 64 items and a
+// set fits in 32 words, else the shared-memory kernel.
+static cudaError_t launch_greedy(const uint32_t* sets, int sets_per_item, int Hkv, int Nq, const int32_t* n_items_dev,
+                                 int NW, int max_group, int W, int nwin, int32_t* group_ptr, int32_t* members,
+                                 int32_t* n_groups, int32_t* ws_usize, int32_t* ws_wtot, int32_t* ws_wcnt,
+                                 int64_t* out_count, cudaStream_t stream) {
+    if (W <= 64 && NW <= 32) {
+        const int items = nwin * Hkv, grid = (items + 3) / 4;
+#define QUP_GREEDY_REG(N)                                                                                        \
+    grp_greedy_reg_kernel<N><<<grid, 128, 0, stream>>>(sets, sets_per_item, Hkv, Nq, n_items_dev, NW, max_group, \
+                                                       W, nwin, group_ptr, members, n_groups, ws_usize, ws_wtot, \
+                                                       ws_wcnt, out_count)
+        if (NW <= 4) QUP_GREEDY_REG(4);
+        else if (NW <= 8) QUP_GREEDY_REG(8);
+        else if (NW <= 12) QUP_GREEDY_REG(12);
+        else if (NW <= 16) QUP_GREEDY_REG(16);
+        else if (NW <= 24) QUP_GREEDY_REG(24);
+        else QUP_GREEDY_REG(32);
+#undef QUP_GREEDY_REG
+        return cudaGetLastError();
+    }
+    const size_t sm = group_greedy_smem(W, NW);
+    cudaError_t e = cudaFuncSetAttribute(grp_greedy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    grp_greedy_kernel<<<dim3(nwin, Hkv), 128, sm, stream>>>(sets, sets_per_item, Hkv, Nq, n_items_dev, NW, max_group,
+                                                             W, nwin, group_ptr, members, n_groups, ws_usize, ws_wtot,
+                                                             ws_wcnt, out_count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
     const size_t sm1 = sizeof(uint32_t) * 8 * (size_t)a.NW;
-    const size_t sm2 = group_greedy_smem(a.W, a.NW);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(grp_rowbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sm1)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(grp_greedy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)sm2)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(grp_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sm1)) != cudaSuccess)
         return e;
     const long long rows = (long long)a.Hq * a.Nq;
     const int grid1 = (int)std::min<long long>((rows + 7) / 8, (long long)a.sms * 8);
-    grp_rowbits_kernel<<<grid1, 256, sm1, stream>>>(a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW,
-                                                   a.rowbits, a.counters, a.err);
+    if (a.K <= 64 && a.NW <= 32 * kRbWords)
+        grp_rowbits_shfl_kernel<<<grid1, 256, 0, stream>>>(a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW, a.rowbits,
+                                                            a.counters, a.err);
+    else
+        grp_rowbits_kernel<<<grid1, 256, sm1, stream>>>(a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW,
+                                                       a.rowbits, a.counters, a.err);
     const dim3 grid2(a.nwin, a.Hkv);
-    grp_greedy_kernel<<<grid2, 128, sm2, stream>>>(a.rowbits, a.Hq / a.Hkv, a.Hkv, a.Nq, nullptr, a.NW,
-                                                   a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
-                                                   a.ws_usize, a.ws_wtot, a.ws_wcnt, nullptr);
+    if ((e = launch_greedy(a.rowbits, a.Hq / a.Hkv, a.Hkv, a.Nq, nullptr, a.NW, a.max_group, a.W, a.nwin,
+                           a.group_ptr, a.members, a.n_groups, a.ws_usize, a.ws_wtot, a.ws_wcnt, nullptr,
+                           stream)) != cudaSuccess)
+        return e;
     grp_emit_kernel<<<grid2, 256, sm1, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
                                                  a.nwin, a.group_ptr, a.members, a.ws_usize, a.ws_wtot,
                                                  a.ws_wcnt, a.union_ptr, a.union_pages, a.row_mask, a.cap,
@@ -587,14 +808,21 @@ __global__ void __launch_bounds__(1024) bnd_order_kernel(const int32_t* __restri
 
 namespace qup {
 
+cudaError_t launch_gbits(const BundleLaunch& a, cudaStream_t stream) {
+    const size_t smw = sizeof(uint32_t) * 8 * (size_t)a.NW;
+    cudaError_t e = cudaFuncSetAttribute(bnd_gbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw);
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)a.Hkv * a.Nq;
+    const int grid1 = (int)std::min<long long>((items + 7) / 8, (long long)a.sms * 8);
+    bnd_gbits_kernel<<<grid1, 256, smw, stream>>>(a.n_groups, a.union_ptr, a.union_pages, a.Hkv, a.Nq, a.P, a.NW,
+                                                  a.gbits, a.bcounters, a.err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream) {
     const size_t smw = sizeof(uint32_t) * 8 * (size_t)a.NW;
-    const size_t smg = group_greedy_smem(a.WB, a.NW);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(bnd_gbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw)) !=
-        cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(grp_greedy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smg)) !=
         cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(bnd_emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw)) !=
@@ -605,9 +833,10 @@ cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream) {
     bnd_gbits_kernel<<<grid1, 256, smw, stream>>>(a.n_groups, a.union_ptr, a.union_pages, a.Hkv, a.Nq, a.P, a.NW,
                                                   a.gbits, a.bcounters, a.err);
     const dim3 grid2(a.nwin, a.Hkv);
-    grp_greedy_kernel<<<grid2, 128, smg, stream>>>(a.gbits, 1, a.Hkv, a.Nq, a.n_groups, a.NW, a.slots, a.WB,
-                                                   a.nwin, a.bundle_ptr, a.bundle_groups, a.n_bundles, a.ws_usize,
-                                                   a.ws_wtot, a.ws_wcnt, a.bcounters);
+    if ((e = launch_greedy(a.gbits, 1, a.Hkv, a.Nq, a.n_groups, a.NW, a.slots, a.WB, a.nwin, a.bundle_ptr,
+                           a.bundle_groups, a.n_bundles, a.ws_usize, a.ws_wtot, a.ws_wcnt, a.bcounters, stream)) !=
+        cudaSuccess)
+        return e;
     bnd_emit_kernel<<<grid2, 256, smw, stream>>>(a.gbits, a.Hkv, a.Nq, a.NW, a.g, a.RS, a.slots, a.WB, a.nwin,
                                                  a.group_ptr, a.members, a.union_ptr, a.union_pages, a.row_mask,
                                                  a.n_bundles, a.bundle_ptr, a.bundle_groups, a.ws_usize, a.ws_wtot,

@@ -5,12 +5,37 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace qup {
 
 constexpr int kStepTok = 128;   // union tokens per pipeline step (MMA M of S^T, K of PV)
 constexpr int kHeadDim = 128;
 constexpr int kMaxPPS = 8;      // pages per step at T = 16
 constexpr int kMaxStages = 16;
+
+// Raises a kernel's dynamic shared-memory limit to `smem` once per device (the
+// attribute is a maximum: later launches with less need no call).
+cudaError_t ensure_smem_attr(const void* fn, size_t smem);
+
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel of the stream finishes; it calls grid_dep_wait() before it
+// reads anything that kernel (or earlier work) produced.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct AttnParams {
     const void* Q;
@@ -92,5 +117,17 @@ struct BundleLaunch {
 };
 
 cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream);
+
+// Fused grouping path (group_fused.cu): dynamic shared memory of each kernel,
+// and the launches.  wcnt / status are workspace arrays sized for Hkv * Nq
+// windows; status (and the bundle kernel's `done` word) must be zero at launch.
+size_t fused_group_smem(int W, int g, int NW);
+size_t fused_bundle_smem(int WB, int NW, int Hkv);
+cudaError_t launch_group_fused(const GroupLaunch& a, uint32_t* gbits, int32_t* wcnt, uint64_t* status,
+                               cudaStream_t stream);
+cudaError_t launch_bundles_fused(const BundleLaunch& a, int32_t* wcnt, uint64_t* status, unsigned* done,
+                                 cudaStream_t stream);
+// group union lists -> group bitsets (a.gbits), for bundles of a caller-given partition
+cudaError_t launch_gbits(const BundleLaunch& a, cudaStream_t stream);
 
 }  // namespace qup

@@ -223,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t lim = p.wait_limit_ns;
 
     // ---------------------------------------------------------------- setup
+    // barriers, TMEM and the tensor maps first; the kernel ahead in the stream may
+    // still be running (programmatic launch): its outputs are read after grid_dep_wait
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSK; ++s) {
             mbar_init(B.kfull(s), 1);
@@ -243,6 +245,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(B.drain2(), 1);
         fence_mbar_init();
         *abort_flag = 0;
+    }
+    if (threadIdx.x == kProducerWarp * 32) prefetch_tensormap(&tmK);
+    if (threadIdx.x == kVProducerWarp * 32) prefetch_tensormap(&tmV);
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    grid_dep_wait();
+    if (threadIdx.x == 0) {
         int acc = 0;
         for (int h = 0; h < p.Hkv; ++h) {
             nb_prefix[h] = acc;
@@ -254,12 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc += n;
         }
         nb_prefix[p.Hkv] = acc;
-    }
-    if (threadIdx.x == kProducerWarp * 32) prefetch_tensormap(&tmK);
-    if (threadIdx.x == kVProducerWarp * 32) prefetch_tensormap(&tmV);
-    if (warp == kMmaWarp) {
-        tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -779,11 +784,9 @@ size_t attn_tile_bytes(int es) { return (size_t)kST * kD * es; }
 template <int ES, int T>
 static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p, int grid,
                             size_t smem, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(union_attn_kernel<ES, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_smem_attr((const void*)union_attn_kernel<ES, T>, smem);
     if (e != cudaSuccess) return e;
-    union_attn_kernel<ES, T><<<grid, kThreads, smem, stream>>>(tmK, tmV, p);
-    return cudaGetLastError();
+    return launch_pdl(union_attn_kernel<ES, T>, dim3(grid), dim3(kThreads), smem, stream, tmK, tmV, p);
 }
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p,
