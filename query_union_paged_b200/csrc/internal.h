@@ -11,7 +11,7 @@ namespace qup {
 
 constexpr int kStepTok = 128;   // union tokens per pipeline step (MMA M of S^T, K of PV)
 constexpr int kHeadDim = 128;
-constexpr int kMaxPPS = 8;      // pages per step at T = 16
+constexpr int kMaxPPS = 8;      // pages per 128-token step at T = 16
 constexpr int kMaxStages = 16;
 
 // Raises a kernel's dynamic shared-memory limit to `smem` once per device (the

@@ -3,45 +3,41 @@
 //
 // Work item: a bundle of up to 128 query rows (up to 128 / rows_per_group
 // page-affine groups of one KV head, see qup_groups).  Pages of the bundle
-// union are streamed once per bundle in steps of 64 tokens (a 128-token page
-// is two steps; 64 / T smaller pages make one step) through two TMA rings,
-// one of K tiles and one of V tiles.  A K slot is released as soon as its S
-// is computed, a V slot when its O update is done, so the loads of K run
-// further ahead than one joint ring would allow.  Per step g, with b = g & 1:
-//      S_b  = Q K^T     M = 128 rows, N = 64 tokens, K = d   (Q from TMEM, K from smem)
-//      P_b  = masked online softmax of S_b                    (TMEM -> registers -> TMEM)
-//      O_b += P_b V     M = 128 rows, N = d, K = 64 tokens    (P from TMEM, V from smem)
-// The two softmax warpgroups ping-pong: warpgroup b owns the steps of parity
-// b, with its own S, P and O columns, running max and row sum, so the softmax
-// of one step overlaps the next; the epilogue merges the two partial results.
-// Keeping Q in TMEM halves the shared-memory operand traffic of QK^T, and a
-// separate P lets S(g+2) start as soon as the softmax has read S(g).  A
-// thread owns one query row, so the row max and the row sum never leave the
-// thread.  A row's max is only raised when a score exceeds it by more than
-// kTau (log2 units); O and the row sum are rescaled then, which after the
-// first steps is rare.  A warp whose 32 rows selected none of a step's pages
-// skips that step's exponentials.
+// union are streamed once per bundle in steps of 128 tokens (one 128-token
+// page, or 128 / T smaller pages) through two TMA rings, one of K tiles and
+// one of V tiles.  Per step g, with b = g & 1:
+//      S_b  = Q K^T     M = 128 rows, N = 128 tokens, K = d  (Q from TMEM, K from smem)
+//      P_b  = masked online softmax of S_b, written over S_b  (TMEM -> registers -> TMEM)
+//      O   += P_b V     M = 128 rows, N = d, K = 128 tokens   (P from TMEM, V from smem)
+// One warpgroup runs the softmax: thread = TMEM lane = bundle row, so the row
+// max and the row sum never leave the thread, and each SM sub-partition holds
+// one softmax warp (two busy softmax warps on one sub-partition starve each
+// other's latency-bound phases).  While it works on step g the tensor pipe
+// runs O += P(g-1) V and then S(g+1) = Q K^T: P is written over the S buffer
+// it came from, so S(g+2) waits for the O update of step g.
+// A row's max is only raised when a score exceeds it by more than kTau (log2
+// units); O and the row sum are rescaled then, which after the first steps is
+// rare.  A warp whose 32 rows selected none of a step's pages skips that
+// step's exponentials.
 //
-// Warp roles (384 threads):
-//   warps 0-7  softmax / epilogue: warpgroup b = warps 4b..4b+3, thread =
-//              TMEM lane = bundle row.  They also gather the rows of Q by
-//              original query ID (no reordered Q tensor) into TMEM.
-//   warp 8     K producer: walks the bundle's page list, resolves physical
+// Warp roles (256 threads):
+//   warps 0-3  softmax / epilogue: thread = TMEM lane = bundle row.  They
+//              also gather the rows of Q by original query ID (no reordered
+//              Q tensor) into TMEM.
+//   warp 4     K producer: walks the bundle's page list, resolves physical
 //              pages (warp-parallel) and TMA-loads the K tiles.
-//   warp 10    V producer: the same walk for the V tiles; it also writes each
+//   warp 6     V producer: the same walk for the V tiles; it also writes each
 //              step's page numbers and row masks, which live as long as the
 //              V slot (until the step's O update).
-//   warp 9     S issuer (one elected lane of a warp-uniform loop) and TMEM
-//              owner (512 columns): S(g) as soon as K tile g and S buffer
-//              g & 1 are ready.
-//   warp 11    PV issuer: O_b += P_b V as soon as P(g) and V tile g are
-//              ready.  Issuing the two streams from two warps on different SM
-//              sub-partitions keeps either from waiting behind the other, and
-//              keeps each issuer's loop short: a single issuing warp that
-//              shares its sub-partition with two busy softmax warps gets too
-//              few issue slots to keep the tensor pipe fed.
-// TMEM columns: S_0, S_1 [0,128); P_0, P_1 from 128; Q after them (bf16 and
-// E4M3); O_0 [256,384), O_1 [384,512).
+//   warp 5     S issuer (one elected lane of a warp-uniform loop) and TMEM
+//              owner (512 columns): S(g) once K tile g has landed and the O
+//              update of step g - 2 has finished with S_b.
+//   warp 7     PV issuer: O += P_b V once P(g) and V tile g are ready.
+// The two issuers sit on different SM sub-partitions, each beside one softmax
+// warp and no other busy warp.
+// TMEM columns: O [0,128); S_0 [128,256); S_1 [256,384); Q from 384 (bf16:
+// 64 columns, E4M3: 32; fp32 Q stays in shared memory).  P_b occupies the
+// first kPCols columns of S_b.
 // Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
 // FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
 // row with its own scale, P stored as E4M3 of 2^6 p).  Every MMA consumes 32
@@ -58,25 +54,27 @@
 
 namespace qup {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 256;
 constexpr int kRows = 128;
 constexpr int kD = kHeadDim;
-constexpr int kST = 64;  // tokens per pipeline step
+constexpr int kST = 128;  // tokens per pipeline step
 constexpr int kTmemCols = 512;
-constexpr int kProducerWarp = 8, kMmaWarp = 9, kVProducerWarp = 10, kPvWarp = 11;
+constexpr int kKProducerWarp = 4, kSWarp = 5, kVProducerWarp = 6, kPvWarp = 7;
+constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384;
 
 struct StageMeta {
-    int32_t upage[4];
-    uint32_t mask[4][4];
-    int32_t tok0;  // first token of the step inside its page (128-token pages)
+    int32_t upage[kMaxPPS];
+    uint32_t mask[kMaxPPS][4];
+    int32_t tok0;  // first token of the step inside its page (pages longer than a step)
     int32_t pad[3];
 };
 
 template <int ES, int T>
 struct Geo {
-    static constexpr int SPP = T > kST ? T / kST : 1;   // steps per page
+    static constexpr int SPP = T > kST ? T / kST : 1;   // steps per page (not used: T <= 128)
     static constexpr int PPS = T < kST ? kST / T : 1;   // pages per step
-    static constexpr int BOXR = T < kST ? T : kST;      // token rows per TMA box
+    static constexpr int BOXR = T < 64 ? T : 64;        // token rows per TMA box
+    static constexpr int BPP = T / BOXR;                // boxes per page (along tokens)
     static constexpr int kTile = kST * kD * ES;         // one K or V tile of a step
     static constexpr int kChunkElems = 128 / ES;        // elements per 128-byte swizzle row
     static constexpr int kNChunk = kD * ES / 128;       // 128-byte chunks along d
@@ -84,23 +82,23 @@ struct Geo {
     static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of a shared-memory Q tile
     static constexpr int kMmaK = 32 / ES;               // K elements per MMA instruction
     static constexpr int kNumMmaS = kD * ES / 32;       // MMAs per S (K = d)
-    static constexpr int kNumMmaPV = kST * ES / 32;     // MMAs per O update (K = 64 tokens)
+    static constexpr int kNumMmaPV = kST * ES / 32;     // MMAs per O update (K = 128 tokens)
     static constexpr int kPCols = kST * ES / 4;         // TMEM columns of P
     static constexpr bool kQTmem = ES != 4;             // Q as the TMEM A operand (bf16, E4M3)
     static constexpr int kQCols = kD * ES / 4;          // TMEM columns of Q
-    static constexpr uint32_t kColP = 128, kColQ = 128 + 2 * kPCols, kColO = 256;
-    static_assert(!kQTmem || kColQ + kQCols <= kColO, "TMEM budget");
-    static_assert(kColP + 2 * kPCols <= kColO, "TMEM budget");
+    static_assert(!kQTmem || kColQ + kQCols <= kTmemCols, "TMEM budget");
+    static_assert(kPCols <= 128, "P fits in its S buffer");
+    static_assert(PPS <= kMaxPPS, "pages per step");
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
-    static constexpr float kTau = ES == 1 ? 2.f : 8.f;      // lazy-rescale margin (log2 units)
+    static constexpr float kTau = ES == 1 ? 2.f : 8.f;  // lazy-rescale margin (log2 units)
     // E4M3 P is stored as 2^kPLog2 p (p <= 2^kTau, so at most 256 < 448); the row sum carries
     // the same factor, which cancels in O / l
     static constexpr float kPLog2 = ES == 1 ? 6.f : 0.f;
 };
 
 struct SmemLayout {
-    uint32_t kst, vst, q, bars, meta, xch, qsc, misc, total;
+    uint32_t kst, vst, q, bars, meta, qsc, misc, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv) {
@@ -116,8 +114,6 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     off += 8u * (2u * (nsk + nsv) + 12u);
     L.meta = off;
     off += (uint32_t)sizeof(StageMeta) * nsv;
-    L.xch = off;
-    off += 2u * kRows * 2u * 4u;
     L.qsc = off;
     off += kRows * 4u;
     L.misc = off;
@@ -136,12 +132,11 @@ struct Bars {
     __device__ __forceinline__ uint32_t vempty(int s) const { return base + 8u * (2 * nsk + nsv + s); }
     __device__ __forceinline__ uint32_t fixed(int i) const { return base + 8u * (2 * (nsk + nsv) + i); }
     __device__ __forceinline__ uint32_t sfull(int i) const { return fixed(i); }
-    __device__ __forceinline__ uint32_t sfree(int i) const { return fixed(2 + i); }
-    __device__ __forceinline__ uint32_t pfull(int i) const { return fixed(4 + i); }
-    __device__ __forceinline__ uint32_t pvdone(int i) const { return fixed(6 + i); }
-    __device__ __forceinline__ uint32_t qfull() const { return fixed(8); }
-    __device__ __forceinline__ uint32_t drain() const { return fixed(9); }
-    __device__ __forceinline__ uint32_t drain2() const { return fixed(10); }
+    __device__ __forceinline__ uint32_t pfull(int i) const { return fixed(2 + i); }
+    __device__ __forceinline__ uint32_t pvdone(int i) const { return fixed(4 + i); }
+    __device__ __forceinline__ uint32_t qfull() const { return fixed(6); }
+    __device__ __forceinline__ uint32_t drain() const { return fixed(7); }
+    __device__ __forceinline__ uint32_t drain2() const { return fixed(8); }
 };
 
 struct Item {
@@ -150,7 +145,7 @@ struct Item {
 };
 
 // Decode flat bundle f; every role calls this and reaches the same verdict.
-template <int SPP, int PPS>
+template <int PPS>
 __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_prefix, int f) {
     Item it;
     int h = 0;
@@ -162,7 +157,7 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_pre
     it.nU = p.union_ptr[bp + 1] - it.ub;
     it.ok = it.ub >= 0 && it.nU >= 0 && (long long)it.ub + it.nU <= p.cap_union;
     if (!it.ok) it.nU = 0;
-    it.nsteps = SPP > 1 ? it.nU * SPP : (it.nU + PPS - 1) / PPS;
+    it.nsteps = (it.nU + PPS - 1) / PPS;
     return it;
 }
 
@@ -205,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     union_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ AttnParams p) {
     using G = Geo<ES, T>;
-    constexpr int SPP = G::SPP, PPS = G::PPS, BOXR = G::BOXR;
+    constexpr int PPS = G::PPS, BOXR = G::BOXR, BPP = G::BPP;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -214,7 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = smem_u32(smem);
     const Bars B{sbase + L.bars, NSK, NSV};
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L.meta);
-    float* xch = reinterpret_cast<float*>(smem + L.xch);
     float* qsc = reinterpret_cast<float*>(smem + L.qsc);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
@@ -236,19 +230,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(B.sfull(i), 1);
-            mbar_init(B.sfree(i), 4);  // one arrive per softmax warp
-            mbar_init(B.pfull(i), 4);
+            mbar_init(B.pfull(i), 4);  // one arrive per softmax warp
             mbar_init(B.pvdone(i), 1);
         }
-        mbar_init(B.qfull(), 8);
+        mbar_init(B.qfull(), 4);
         mbar_init(B.drain(), 1);
         mbar_init(B.drain2(), 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
-    if (threadIdx.x == kProducerWarp * 32) prefetch_tensormap(&tmK);
+    if (threadIdx.x == kKProducerWarp * 32) prefetch_tensormap(&tmK);
     if (threadIdx.x == kVProducerWarp * 32) prefetch_tensormap(&tmV);
-    if (warp == kMmaWarp) {
+    if (warp == kSWarp) {
         tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -272,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_items = nb_prefix[p.Hkv];
 
-    if (warp == kProducerWarp || warp == kVProducerWarp) {
+    if (warp == kKProducerWarp || warp == kVProducerWarp) {
         // ============================================================ producers (whole warp each)
         // Both walk the same bundles and pages; the K warp fills the K ring, the V warp the
         // V ring and the step metadata (indexed by V slot: it is read by the softmax of the
@@ -287,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = item_at(p, rnd, n_items);
             if (f == -1) break;
             if (f < 0) continue;
-            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
-            const int n_ent = SPP > 1 ? it.nU : it.nsteps * PPS;  // incl. padding of the last step
+            const Item it = load_item<PPS>(p, nb_prefix, f);
+            const int n_ent = it.nsteps * PPS;  // incl. padding of the last step
             for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
                 const int idx = e0 + lane;
                 int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
@@ -308,8 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (phys == p.P_phys) mk = make_uint4(0, 0, 0, 0);
                 }
-                const int ecnt = min(32, n_ent - e0);
-                const int nst = SPP > 1 ? ecnt * SPP : ecnt / PPS;
+                const int nst = min(32, n_ent - e0) / PPS;  // 32 is a multiple of PPS
                 for (int k = 0; k < nst; ++k, ++gs) {
                     const int slot = gs % NR;
                     int okv = 0;
@@ -320,11 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
                                                       gs == p.dbg_skip_stage);
-                    const int tok0 = SPP > 1 ? (k % SPP) * kST : 0;
                     int ph[PPS];
 #pragma unroll
                     for (int q = 0; q < PPS; ++q) {
-                        const int src = SPP > 1 ? (k / SPP) : (k * PPS + q);
+                        const int src = k * PPS + q;
                         ph[q] = __shfl_sync(0xffffffffu, phys, src);
                         if (isV) {
                             const int uq = __shfl_sync(0xffffffffu, u, src);
@@ -339,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 m.mask[q][1] = m1;
                                 m.mask[q][2] = m2;
                                 m.mask[q][3] = m3;
-                                m.tok0 = tok0;
+                                m.tok0 = 0;
                             }
                         }
                     }
@@ -351,9 +342,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int q = 0; q < PPS; ++q) {
 #pragma unroll
-                            for (int c = 0; c < G::kNChunk; ++c) {
-                                const uint32_t off = (uint32_t)c * G::kChunkBytes + (uint32_t)(q * BOXR) * 128u;
-                                tma_load_4d(dst + off, tm, fb, c * G::kChunkElems, tok0, it.h, ph[q]);
+                            for (int bb = 0; bb < BPP; ++bb) {
+#pragma unroll
+                                for (int c = 0; c < G::kNChunk; ++c) {
+                                    const uint32_t off =
+                                        (uint32_t)c * G::kChunkBytes + (uint32_t)(q * T + bb * BOXR) * 128u;
+                                    tma_load_4d(dst + off, tm, fb, c * G::kChunkElems, bb * BOXR, it.h, ph[q]);
+                                }
                             }
                         }
                     }
@@ -369,16 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp || warp == kPvWarp) {
+    } else if (warp == kSWarp || warp == kPvWarp) {
         // ============================================================ MMA issuers (whole warp, one elected lane)
-        // Two in-order streams, one warp each (on different SM sub-partitions, so each keeps
-        // its share of issue slots next to the busy softmax warps):
-        //   S warp:  S(g) = Q K^T  needs K tile g and S buffer g & 1, released by the softmax
-        //            of step g - 2; commits S-full(b) and the K slot.
-        //   PV warp: O_b += P_b V  needs P(g) and V tile g; commits PV-done(b) and the V slot.
+        //   S warp:  S(g) = Q K^T into S_b: needs K tile g, and the O update of step g - 2
+        //            (which read P from S_b) finished; commits S-full(b) and the K slot.
+        //   PV warp: O += P_b V: needs P(g) and V tile g; commits PV-done(b) and the V slot.
         // The PV warp needs no Q barrier: P(g) of a bundle's first step is written after the
         // softmax warps have finished the previous bundle's epilogue (its reads of O).
-        const bool isS = warp == kMmaWarp;
+        const bool isS = warp == kSWarp;
         const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, kST, kRows);
         const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
         // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
@@ -393,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f = item_at(p, rnd, n_items);
             if (f == -1) break;
             if (f < 0) continue;
-            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
+            const Item it = load_item<PPS>(p, nb_prefix, f);
             if (isS) {
                 ok = warp_ok(mbar_wait(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                 if (!ok) break;
@@ -401,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int s = 0; s < it.nsteps; ++s) {
                     const int g = gs + s, b = g & 1;
                     ok = warp_ok(mbar_wait(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 (g < 2 || mbar_wait(B.sfree(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
+                                 (g < 2 || mbar_wait(B.pvdone(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
                                                      QUP_ERR_TIMEOUT, lim)));
                     if (!ok) break;
                     tc_fence_after();
@@ -412,11 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < G::kNumMmaS; ++k) {
                             const uint32_t koff = ((k >> 2) * G::kChunkBytes + (k & 3) * 32) >> 4;
                             if constexpr (G::kQTmem) {
-                                tc_mma_ts<G::kKind>(tmem + 64u * b, tmem + G::kColQ + 8u * k, kdesc + koff, idesc_s,
-                                                    k > 0);
+                                tc_mma_ts<G::kKind>(tmem + kColS + 128u * b, tmem + kColQ + 8u * k, kdesc + koff,
+                                                    idesc_s, k > 0);
                             } else {
                                 const uint32_t qoff = ((k >> 2) * G::kQChunkBytes + (k & 3) * 32) >> 4;
-                                tc_mma<G::kKind>(tmem + 64u * b, qdesc + qoff, kdesc + koff, idesc_s, k > 0);
+                                tc_mma<G::kKind>(tmem + kColS + 128u * b, qdesc + qoff, kdesc + koff, idesc_s, k > 0);
                             }
                         }
                         tc_commit(B.sfull(b));
@@ -437,13 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
                                                      (uint32_t)G::kChunkBytes, vsbo, vlayout);
-                    const bool acc0 = s >= 2;  // steps 0 and 1 of a bundle open O_0 / O_1
                     if (elect_one_sync()) {
 #pragma unroll
                         for (int k = 0; k < G::kNumMmaPV; ++k) {
                             // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
-                            tc_mma_ts<G::kKind>(tmem + G::kColO + 128u * b, tmem + G::kColP + G::kPCols * b + 8u * k,
-                                                vdesc + ((k * G::kMmaK * 128) >> 4), idesc_o, acc0 || k > 0);
+                            tc_mma_ts<G::kKind>(tmem + kColO, tmem + kColS + 128u * b + 8u * k,
+                                                vdesc + ((k * G::kMmaK * 128) >> 4), idesc_o, s > 0 || k > 0);
                         }
                         tc_commit(B.pvdone(b));
                         tc_commit(B.vempty(vs));
@@ -465,17 +457,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(dbar, 0, lim);
         __syncwarp();
     } else {
-        // ============================================================ softmax / epilogue (256 threads)
-        const int wg = warp >> 2;            // warpgroup: owns the steps of parity wg
-        const int quad = warp & 3;           // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;      // bundle row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        const uint32_t s_addr = tmem + lane_base + 64u * wg;                      // S_wg
-        const uint32_t p_addr = tmem + lane_base + G::kColP + G::kPCols * wg;     // P_wg
-        const uint32_t o_addr = tmem + lane_base + G::kColO + 128u * wg;          // O_wg
+        // ============================================================ softmax / epilogue (warps 0-3)
+        const int r = warp * 32 + lane;  // bundle row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const float kNegInf = -__int_as_float(0x7f800000);
+        const float kPosInf = __int_as_float(0x7f800000);
         const int g = p.g, MQ = kRows / g;
-        int gs = 0;
+        int gs = 0, vs = 0, vph = 0;
         bool ok = true;
         for (int rnd = 0;; ++rnd) {
             const int f = item_at(p, rnd, n_items);
@@ -484,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
                 continue;
             }
-            const Item it = load_item<SPP, PPS>(p, nb_prefix, f);
+            const Item it = load_item<PPS>(p, nb_prefix, f);
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             // ---- this row's query (original ID) and head
             int qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
@@ -495,100 +483,97 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int head = it.h * g + (r % g);
             const int qpos = qid >= 0 ? p.q_pos[qid] : -1;
             const int vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
+            float cs = p.scale_log2;                      // score scale (log2 domain) of this row
             // ---- Q row by original ID -> TMEM (bf16, E4M3) or the shared-memory tile (fp32)
             {
                 const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
                 if constexpr (ES == 2) {
-                    const uint4* src =
-                        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off) + wg * 8;
-                    uint32_t qv[32];
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                        qv[4 * c] = v.x;
-                        qv[4 * c + 1] = v.y;
-                        qv[4 * c + 2] = v.z;
-                        qv[4 * c + 3] = v.w;
-                    }
-                    tmem_st_x32(tmem + lane_base + G::kColQ + 32u * wg, qv);
-                } else if constexpr (ES == 4) {
-                    uint8_t* qt = smem + L.q;
-                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off) + wg * 16;
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, wg * 16 + c, kRows)) = v;
-                    }
-                    fence_proxy_async_smem();
-                } else {
-                    if (wg == 0) {  // whole row: bf16 -> E4M3 with the row's scale amax / 448
-                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
-                        uint4 raw[16];
-                        float amax = 0.f;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            raw[c] = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
-                                                         fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
-                        }
-                        const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                    for (int half = 0; half < 2; ++half) {
                         uint32_t qv[32];
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
-                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-                            float x[8];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
-                                x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
-                            }
-                            qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-                            qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 v = qid >= 0 ? src[half * 8 + c] : make_uint4(0, 0, 0, 0);
+                            qv[4 * c] = v.x;
+                            qv[4 * c + 1] = v.y;
+                            qv[4 * c + 2] = v.z;
+                            qv[4 * c + 3] = v.w;
                         }
-                        tmem_st_x32(tmem + lane_base + G::kColQ, qv);
-                        qsc[r] = amax * (1.f / 448.f);
+                        tmem_st_x32(tmem + lane_base + kColQ + 32u * half, qv);
                     }
+                } else if constexpr (ES == 4) {
+                    uint8_t* qt = smem + L.q;
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
+                    }
+                    fence_proxy_async_smem();
+                } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
+                    uint4 raw[16];
+                    float amax = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        raw[c] = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                        const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                                     fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+                    }
+                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                    uint32_t qv[32];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
+                        const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
+                            x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
+                        }
+                        qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                        qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                    }
+                    tmem_st_x32(tmem + lane_base + kColQ, qv);
+                    cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
                 }
                 if constexpr (G::kQTmem) tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(B.qfull());
-            float cs = p.scale_log2;  // score scale (log2 domain) of this row
-            if constexpr (ES == 1) {
-                bar_sync(1, 256);  // qsc written by warpgroup 0
-                cs = qsc[r] * p.k_scale[it.h] * p.scale_log2;
-            }
             float m_used = kNegInf, lsum = 0.f;
-            int mine_steps = 0;  // steps of this bundle this warpgroup has processed
 
             for (int s = 0; s < it.nsteps; ++s) {
-                const int gstep = gs + s;
-                if ((gstep & 1) != wg) continue;  // the other warpgroup's step
-                const int slot = gstep % NSV;  // V slot: V tile and step metadata
+                const int gstep = gs + s, b = gstep & 1, slot = vs;
+                const int vphase = vph;
+                if (++vs == NSV) {
+                    vs = 0;
+                    vph ^= 1;
+                }
                 if (ok)
-                    ok = warp_ok(mbar_wait(B.vfull(slot), (gstep / NSV) & 1, abort_flag, p.err,
-                                           QUP_ERR_TIMEOUT, lim) &&
-                                 mbar_wait(B.sfull(wg), (gstep >> 1) & 1, abort_flag, p.err,
-                                           QUP_ERR_TIMEOUT, lim));
+                    ok = warp_ok(mbar_wait(B.vfull(slot), vphase, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                 mbar_wait(B.sfull(b), (gstep >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                 if (!ok) continue;
                 tc_fence_after();
+                const uint32_t s_addr = tmem + lane_base + kColS + 128u * b;
                 uint32_t sv[kST];
-                tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+#pragma unroll
+                for (int i = 0; i < kST / 32; ++i)
+                    tmem_ld32(s_addr + 32u * i, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * i));
                 const StageMeta& mt = meta[slot];
-                const int tok0 = mt.tok0;
                 // a page of the step that reaches kv_len: its cache slots at or past kv_len may
                 // hold non-finite bytes, so those V rows are zeroed and the step's scores masked
                 bool tail = false;
 #pragma unroll
-                for (int q = 0; q < PPS; ++q) tail |= mt.upage[q] * T + tok0 + BOXR > p.kv_len;
-                if (tail && r < kST) {
-                    const int q = r / BOXR;
-                    if (mt.upage[q] * T + tok0 + (r - q * BOXR) >= p.kv_len) {
+                for (int q = 0; q < PPS; ++q) tail |= mt.upage[q] * T + T > p.kv_len;
+                if (tail) {  // thread r zeroes token row r of the step if it lies past kv_len
+                    const int q = r / T;
+                    if (mt.upage[q] * T + (r - q * T) >= p.kv_len) {
                         uint8_t* vt = smem + L.vst + (uint32_t)slot * G::kTile;
 #pragma unroll
                         for (int c = 0; c < G::kNChunk; ++c)
@@ -598,45 +583,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     make_uint4(0, 0, 0, 0);
                     }
                 }
-                // row r sees token j of page q iff the page is in its own TopK row
-                // (bit r of the page's mask) and the token's position is < vis_end
+                // row r sees token t of page q iff the page is in its own TopK row (bit r of
+                // the page's mask) and the token's position is < vis_end
                 int lim_q[PPS];
                 bool live = false, partial = false;
 #pragma unroll
                 for (int q = 0; q < PPS; ++q) {
                     const bool mine = (mt.mask[q][r >> 5] >> (r & 31)) & 1u;
-                    lim_q[q] = mine ? max(0, min(BOXR, vis_end - (mt.upage[q] * T + tok0))) : 0;
+                    lim_q[q] = mine ? max(0, min(T, vis_end - mt.upage[q] * T)) : 0;
                     live |= lim_q[q] > 0;
-                    partial |= lim_q[q] > 0 && lim_q[q] < BOXR;
+                    partial |= lim_q[q] > 0 && lim_q[q] < T;
                 }
                 tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(B.sfree(wg));  // S_wg may now be overwritten by S(gstep + 2)
                 const bool warp_live = __any_sync(0xffffffffu, live);
-                // Fast path (the usual step: one whole page, every row sees all of it or none of
-                // it): the max is taken over the raw scores (cs > 0) and each exponent is one FMA.
+                // pages no row of this warp selected: no max, no exponentials (P = 0)
+                bool pg_live[PPS];
+#pragma unroll
+                for (int q = 0; q < PPS; ++q) pg_live[q] = __any_sync(0xffffffffu, lim_q[q] > 0);
+                // Fast path (every page of the step fully seen or fully unseen by each row, no
+                // kv_len tail): the max is taken over the raw scores of seen pages (cs > 0) and
+                // each exponent is one FMA, an unseen page getting an infinite offset.
                 // Otherwise every score is scaled and masked first.
-                const bool slow = PPS > 1 || tail || __any_sync(0xffffffffu, partial);
+                const bool slow = tail || __any_sync(0xffffffffu, partial);
                 float mloc = kNegInf;
                 if (warp_live) {
-                    float mx[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) mx[k] = kNegInf;
                     if (!slow) {
 #pragma unroll
-                        for (int j = 0; j < kST; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
+                        for (int q = 0; q < PPS; ++q) {
+                            if (!pg_live[q]) continue;
+                            float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+                            for (int j = q * T; j < (q + 1) * T; ++j)
+                                mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sv[j]));
+                            const float mq = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                            if (lim_q[q] > 0) mloc = fmaxf(mloc, mq * cs);
+                        }
                     } else {
+                        float mx[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) mx[k] = kNegInf;
 #pragma unroll
                         for (int j = 0; j < kST; ++j) {
-                            const float v = (j % BOXR) < lim_q[j / BOXR] ? __uint_as_float(sv[j]) * cs : kNegInf;
+                            const int q = j / T, t = j - q * T;
+                            const float v = t < lim_q[q] ? __uint_as_float(sv[j]) * cs : kNegInf;
                             sv[j] = __float_as_uint(v);
                             mx[j & 7] = fmaxf(mx[j & 7], v);
                         }
+                        mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                     }
-                    const float m4 = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                    mloc = slow ? m4 : (live ? m4 * cs : kNegInf);
                 }
                 // lazy running max: raise it only when a score exceeds it by more than kTau
                 const bool need = mloc > m_used + G::kTau;
@@ -646,127 +641,137 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_used = mloc;
                     lsum *= alpha;
                 }
-                uint32_t pk[G::kPCols];
+                // packed P (fp32 P is written back into sv: it has the width of S)
+                uint32_t pk[ES == 4 ? 1 : G::kPCols];
                 if (warp_live) {
-                    // p = 2^(x - m + kPLog2); a fast-path row that sees nothing gets x - inf = -inf
+                    // p = 2^(x - m + kPLog2); on the fast path an unseen page gets x - inf = -inf
                     const float xs = slow ? 1.f : cs;
-                    const float moff = (!slow && !live) ? __int_as_float(0x7f800000)
-                                                        : (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
+                    const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
+                    float off[PPS];
+#pragma unroll
+                    for (int q = 0; q < PPS; ++q) off[q] = (!slow && lim_q[q] == 0) ? kPosInf : mb;
                     float part[4] = {0.f, 0.f, 0.f, 0.f};
-                    if constexpr (ES == 2) {
 #pragma unroll
-                        for (int j = 0; j < kST; j += 2) {
-                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
-                            const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -moff));
-                            part[(j >> 1) & 3] += p0 + p1;
-                            pk[j / 2] = pack_bf16x2(p0, p1);
-                        }
-                    } else if constexpr (ES == 4) {
+                    for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
+                        if (slow || pg_live[q]) {
+                            if constexpr (ES == 2) {
 #pragma unroll
-                        for (int j = 0; j < kST; ++j) {
-                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
-                            part[j & 3] += p0;
-                            pk[j] = __float_as_uint(p0);
-                        }
-                    } else {
+                                for (int j = q * T; j < (q + 1) * T; j += 2) {
+                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                    const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
+                                    part[(j >> 1) & 3] += p0 + p1;
+                                    pk[j / 2] = pack_bf16x2(p0, p1);
+                                }
+                            } else if constexpr (ES == 4) {
 #pragma unroll
-                        for (int j = 0; j < kST; j += 4) {
-                            const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -moff));
-                            const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -moff));
-                            const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -moff));
-                            const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -moff));
-                            part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                            pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
+                                for (int j = q * T; j < (q + 1) * T; ++j) {
+                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                    part[j & 3] += p0;
+                                    sv[j] = __float_as_uint(p0);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = q * T; j < (q + 1) * T; j += 4) {
+                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                    const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
+                                    const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -off[q]));
+                                    const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -off[q]));
+                                    part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
+                                    pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
+                                }
+                            }
+                        } else {
+                            if constexpr (ES == 4) {
+#pragma unroll
+                                for (int j = q * T; j < (q + 1) * T; ++j) sv[j] = 0u;
+                            } else {
+#pragma unroll
+                                for (int j = q * G::kPCols / PPS; j < (q + 1) * G::kPCols / PPS; ++j) pk[j] = 0u;
+                            }
                         }
                     }
                     lsum += (part[0] + part[1]) + (part[2] + part[3]);
+                } else if constexpr (ES == 4) {
+#pragma unroll
+                    for (int j = 0; j < kST; ++j) sv[j] = 0u;
                 } else {
 #pragma unroll
                     for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
                 }
-                // this warpgroup's previous O update must be done before O is rescaled and
-                // P_wg overwritten; it was issued when the previous step's P was stored, a
-                // whole softmax ago, so this rarely waits
-                const bool pv_ok = gstep < 2 || mbar_wait(B.pvdone(wg), ((gstep - 2) >> 1) & 1, abort_flag,
-                                                          p.err, QUP_ERR_TIMEOUT, lim);
-                ok = warp_ok(pv_ok);
-                if (!ok) continue;
-                tc_fence_after();
-                if (mine_steps > 0 && __any_sync(0xffffffffu, need)) {
+                // O is rescaled only after every earlier O update has finished (rare)
+                if (s > 0 && __any_sync(0xffffffffu, need)) {
+                    const int pg = gstep - 1;
+                    ok = warp_ok(mbar_wait(B.pvdone(pg & 1), (pg >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                    if (!ok) continue;
+                    tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t ov[32];
-                        tmem_ld32(o_addr + 32u * c, ov);
+                        tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        tmem_st_x32(o_addr + 32u * c, ov);
+                        tmem_st_x32(tmem + lane_base + kColO + 32u * c, ov);
                     }
                 }
-                tmem_st_n<G::kPCols>(p_addr, pk);
+                // P over the S buffer it came from (every column of S is in registers)
+                if constexpr (ES == 4) {
+                    tmem_st_n<kST>(s_addr, sv);
+                } else {
+                    tmem_st_n<G::kPCols>(s_addr, pk);
+                }
                 tmem_wait_st();
                 if (tail) fence_proxy_async_smem();  // zeroed V rows -> async proxy
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(B.pfull(wg));
-                ++mine_steps;
+                if (lane == 0) mbar_arrive(B.pfull(b));
             }
-            // ---- epilogue: merge the two partial results; O / l -> O[qid][head][:]
-            if (ok && mine_steps > 0) {
-                int last = gs + it.nsteps - 1;
-                if ((last & 1) != wg) --last;
-                ok = warp_ok(mbar_wait(B.pvdone(wg), (last >> 1) & 1, abort_flag, p.err,
-                                       QUP_ERR_TIMEOUT, lim));
-            }
+            // ---- epilogue: O / l -> O[qid][head][:]
             gs += it.nsteps;
-            xch[(wg * kRows + r) * 2 + 0] = mine_steps > 0 ? m_used : kNegInf;
-            xch[(wg * kRows + r) * 2 + 1] = mine_steps > 0 ? lsum : 0.f;
-            ok = bar_and(1, 256, ok);
+            if (ok && it.nsteps > 0) {
+                const int last = gs - 1;
+                ok = warp_ok(mbar_wait(B.pvdone(last & 1), (last >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+            }
             if (!ok) break;
-            const float m0 = xch[r * 2], l0 = xch[r * 2 + 1];
-            const float m1 = xch[(kRows + r) * 2], l1 = xch[(kRows + r) * 2 + 1];
-            const float M = fmaxf(m0, m1);
-            const float f0 = (m0 == kNegInf) ? 0.f : ex2(m0 - M);
-            const float f1 = (m1 == kNegInf) ? 0.f : ex2(m1 - M);
-            const float Lsum = l0 * f0 + l1 * f1;
+            tc_fence_after();
             float vsc = 1.f;
             if constexpr (ES == 1) vsc = p.v_scale[it.h];
-            const float inv = Lsum > 0.f ? vsc / Lsum : 0.f;
-            const float g0 = f0 * inv, g1 = f1 * inv;
-            const bool use0 = m0 != kNegInf && Lsum > 0.f, use1 = m1 != kNegInf && Lsum > 0.f;
-            tc_fence_after();
-            // this warpgroup writes features [64 wg, 64 wg + 64) of the row
-            float o[64];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t a[32], e2[32];
-                tmem_ld32(tmem + lane_base + G::kColO + (uint32_t)(64 * wg + 32 * c), a);
-                tmem_ld32(tmem + lane_base + G::kColO + 128u + (uint32_t)(64 * wg + 32 * c), e2);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    o[32 * c + e] = (use0 ? __uint_as_float(a[e]) * g0 : 0.f) + (use1 ? __uint_as_float(e2[e]) * g1 : 0.f);
-            }
-            if (qid >= 0) {
-                const size_t oi = ((size_t)qid * p.Hq + head) * kD + 64 * wg;
-                if constexpr (ES == 4) {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+            const float inv = lsum > 0.f ? vsc / lsum : 0.f;
+            const size_t oi = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ov[32];
+                if (it.nsteps > 0) {
+                    tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
+                    tmem_wait_ld();
                 } else {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + oi);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = make_uint4(pack_bf16x2(o[8 * e], o[8 * e + 1]), pack_bf16x2(o[8 * e + 2], o[8 * e + 3]),
-                                            pack_bf16x2(o[8 * e + 4], o[8 * e + 5]),
-                                            pack_bf16x2(o[8 * e + 6], o[8 * e + 7]));
+                    for (int e = 0; e < 32; ++e) ov[e] = 0u;
                 }
-                if (wg == 0 && p.lse != nullptr)
-                    p.lse[(size_t)qid * p.Hq + head] =
-                        Lsum > 0.f ? (M + __log2f(Lsum) - G::kPLog2) * 0.69314718055994531f : kNegInf;
+                if (qid >= 0) {
+                    if constexpr (ES == 4) {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                                 __uint_as_float(ov[4 * e + 2]) * inv,
+                                                 __uint_as_float(ov[4 * e + 3]) * inv);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + oi + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(
+                                pack_bf16x2(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
+                    }
+                }
             }
+            if (qid >= 0 && p.lse != nullptr)
+                p.lse[(size_t)qid * p.Hq + head] =
+                    lsum > 0.f ? (m_used + __log2f(lsum) - G::kPLog2) * 0.69314718055994531f : kNegInf;
             tc_fence_before();
-            bar_sync(1, 256);  // O_0, O_1 and Q read before the next bundle overwrites them
         }
     }
 
@@ -774,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kSWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv) { return smem_layout(es, nsk, nsv, Hkv).total; }
