@@ -101,9 +101,9 @@ def profiled_traffic(workload_name: str):
     return float(m.group(1)) if m else None
 
 
-# kernels of one step: grouping (rowbits, greedy, emit), bundling (bits, greedy, emit, order),
-# union attention
-LAUNCHES_PER_STEP = 3 + 4 + 1
+# kernels of one step: the fused grouping kernel, the fused bundling kernel (which also orders
+# the bundles), union attention (a memset of the look-back status words precedes them)
+LAUNCHES_PER_STEP = 3
 
 
 class ClockSampler:
