@@ -596,10 +596,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_wait_ld();
                 const bool warp_live = __any_sync(0xffffffffu, live);
-                // pages no row of this warp selected: no max, no exponentials (P = 0)
-                bool pg_live[PPS];
-#pragma unroll
-                for (int q = 0; q < PPS; ++q) pg_live[q] = __any_sync(0xffffffffu, lim_q[q] > 0);
                 // Fast path (every page of the step fully seen or fully unseen by each row, no
                 // kv_len tail): the max is taken over the raw scores of seen pages (cs > 0) and
                 // each exponent is one FMA, an unseen page getting an infinite offset.
@@ -610,7 +606,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!slow) {
 #pragma unroll
                         for (int q = 0; q < PPS; ++q) {
-                            if (!pg_live[q]) continue;
                             float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
                             for (int j = q * T; j < (q + 1) * T; ++j)
@@ -653,40 +648,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
-                        if (slow || pg_live[q]) {
-                            if constexpr (ES == 2) {
+                        // (skipping the pages none of a warp's rows selected unbalances the four
+                        // warps, and each step waits for the slowest: measured slower)
+                        if constexpr (ES == 2) {
 #pragma unroll
-                                for (int j = q * T; j < (q + 1) * T; j += 2) {
-                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                    const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
-                                    part[(j >> 1) & 3] += p0 + p1;
-                                    pk[j / 2] = pack_bf16x2(p0, p1);
-                                }
-                            } else if constexpr (ES == 4) {
+                            for (int j = q * T; j < (q + 1) * T; j += 2) {
+                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
+                                part[(j >> 1) & 3] += p0 + p1;
+                                pk[j / 2] = pack_bf16x2(p0, p1);
+                            }
+                        } else if constexpr (ES == 4) {
 #pragma unroll
-                                for (int j = q * T; j < (q + 1) * T; ++j) {
-                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                    part[j & 3] += p0;
-                                    sv[j] = __float_as_uint(p0);
-                                }
-                            } else {
-#pragma unroll
-                                for (int j = q * T; j < (q + 1) * T; j += 4) {
-                                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                    const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
-                                    const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -off[q]));
-                                    const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -off[q]));
-                                    part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                                    pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
-                                }
+                            for (int j = q * T; j < (q + 1) * T; ++j) {
+                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                part[j & 3] += p0;
+                                sv[j] = __float_as_uint(p0);
                             }
                         } else {
-                            if constexpr (ES == 4) {
 #pragma unroll
-                                for (int j = q * T; j < (q + 1) * T; ++j) sv[j] = 0u;
-                            } else {
-#pragma unroll
-                                for (int j = q * G::kPCols / PPS; j < (q + 1) * G::kPCols / PPS; ++j) pk[j] = 0u;
+                            for (int j = q * T; j < (q + 1) * T; j += 4) {
+                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
+                                const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
+                                const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -off[q]));
+                                const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -off[q]));
+                                part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
+                                pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
                             }
                         }
                     }
