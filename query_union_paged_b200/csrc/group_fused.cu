@@ -61,11 +61,15 @@ struct WinSmem {
     int* gsum;        // [W] sum of member set sizes of each group
     int* misc;        // [8]: 0 groups, 1 compact words NWC, 7 compact pitch
     int* goff;        // [W + 1] exclusive prefix of gus
+    uint32_t* post;   // [kPostWords] block greedy: per-warp best keys and sets, group tallies
 };
+
+constexpr int kPostWords = 2 * 8 * (8 + 1) + 2 * 8;  // up to 8 warps, 8-word compact sets
 
 __host__ __device__ inline size_t win_smem_bytes(int W, int NW, int extra_words) {
     const int NWCp = NW | 1;
-    size_t words = (size_t)W * NW + NW + (NW + 1) + (size_t)W * NWCp + NWCp + W + W + (W + 1) + W + W + 8 + (W + 1);
+    size_t words = (size_t)W * NW + NW + (NW + 1) + (size_t)W * NWCp + NWCp + W + W + (W + 1) + W + W + 8 + (W + 1) +
+                   kPostWords;
     return 4 * (words + (size_t)extra_words) + 64;
 }
 
@@ -96,6 +100,8 @@ __device__ inline WinSmem carve(uint32_t* base, int W, int NW) {
     s.misc = reinterpret_cast<int*>(p);
     p += 8;
     s.goff = reinterpret_cast<int*>(p);
+    p += W + 1;
+    s.post = p;
     return s;
 }
 
@@ -302,10 +308,122 @@ __device__ __noinline__ void greedy_smem(const WinSmem& s, int n, int max_group)
     }
 }
 
-// Warp 0 runs the greedy on the compact sets; the CTA waits for it.  The greedy
+// Greedy with the whole CTA for windows of 65..256 items whose compact sets fit
+// in NWR words: thread t holds item t's set in registers.  A pick: each thread
+// scores its item, each warp's best lane posts its key and set to shared memory
+// (double-buffered by pick parity), one barrier, and every thread reduces the
+// posted keys and ORs the winner's set into its copy of the running union.
+// Same keys (new_pages << 9 | local_id) and so the same picks as greedy_reg.
+template <int NWR>
+__device__ __noinline__ void greedy_block(const WinSmem& s, int n, int max_group) {
+    uint32_t* post = s.post;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarp = blockDim.x >> 5;
+    const int pitch = s.misc[7], NWC = s.misc[1];
+    // post[parity][warp] = {key, set words...}
+    const int stride = NWR + 1;
+    uint32_t sv[NWR], U[NWR];
+#pragma unroll
+    for (int x = 0; x < NWR; ++x) sv[x] = (tid < n && x < NWC) ? s.cs[(size_t)tid * pitch + x] : 0u;
+    const int sz = tid < n ? s.ssize[tid] : 0;
+    bool taken = tid >= n;
+    int ng = 0, pos = 0, par = 0;
+    // block-wide argmin of `key` (kNone when nothing); the winner's set ends in `win`
+    auto block_pick = [&](unsigned key, uint32_t (&win)[NWR]) -> unsigned {
+        const unsigned wmin = __reduce_min_sync(0xffffffffu, key);
+        const unsigned hit = __ballot_sync(0xffffffffu, key == wmin);
+        uint32_t* slot = post + (size_t)(par * nwarp + warp) * stride;
+        if (lane == __ffs(hit) - 1) {
+            slot[0] = wmin;
+#pragma unroll
+            for (int x = 0; x < NWR; ++x) slot[1 + x] = sv[x];
+        }
+        __syncthreads();
+        unsigned best = kNone;
+        int bw = 0;
+        for (int w = 0; w < nwarp; ++w) {
+            const unsigned k = post[(size_t)(par * nwarp + w) * stride];
+            if (k < best) {
+                best = k;
+                bw = w;
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) win[x] = post[(size_t)(par * nwarp + bw) * stride + 1 + x];
+        par ^= 1;
+        return best;
+    };
+    while (true) {
+        uint32_t win[NWR];
+        const unsigned seed = block_pick(taken ? kNone : (unsigned)tid, win);
+        if (seed == kNone) break;
+        bool ing = (int)seed == tid;
+        if (ing) taken = true;
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) U[x] = win[x];
+        int cnt = 1;
+        while (cnt < max_group) {
+            int nc = 0;
+#pragma unroll
+            for (int x = 0; x < NWR; ++x) nc += __popc(sv[x] & ~U[x]);
+            const unsigned best = block_pick(taken ? kNone : (((unsigned)nc << 9) | (unsigned)tid), win);
+            if (best == kNone) break;
+            if ((int)(best & 511u) == tid) {
+                taken = true;
+                ing = true;
+            }
+#pragma unroll
+            for (int x = 0; x < NWR; ++x) U[x] |= win[x];
+            ++cnt;
+        }
+        int us = 0;
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) us += __popc(U[x]);
+        // members in ascending local ID: prefix over the warps' ballots (one more barrier)
+        const unsigned bal = __ballot_sync(0xffffffffu, ing);
+        int* wcount = reinterpret_cast<int*>(post + (size_t)2 * nwarp * stride);  // [nwarp]
+        int* wsum = wcount + nwarp;                                                // [nwarp]
+        const int ssum = __reduce_add_sync(0xffffffffu, ing ? sz : 0);
+        if (lane == 0) {
+            wcount[warp] = __popc(bal);
+            wsum[warp] = ssum;
+        }
+        __syncthreads();
+        int before = 0, sum_s = 0;
+        for (int w = 0; w < nwarp; ++w) {
+            if (w < warp) before += wcount[w];
+            sum_s += wsum[w];
+        }
+        if (ing) s.order[pos + before + __popc(bal & ((1u << lane) - 1u))] = tid;
+        if (tid == 0) {
+            s.gstart[ng] = pos;
+            s.gus[ng] = us;
+            s.gsum[ng] = sum_s;
+        }
+        pos += cnt;
+        ++ng;
+        __syncthreads();  // wcount / wsum are rewritten by the next group
+    }
+    if (tid == 0) {
+        s.gstart[ng] = pos;
+        s.misc[0] = ng;
+    }
+}
+
+// The greedy on the compact sets: warp 0 for windows of up to 64 items (or wide
+// sets), the whole CTA for larger windows of narrow sets; the CTA waits.  The greedy
 // functions stay out of line: inlined into the kernel body they compiled to a
 // loop several times slower.
 __device__ __noinline__ void run_greedy(const WinSmem& s, int n, int max_group) {
+    const int nwc = s.misc[1];
+    if (n > 64 && n <= (int)blockDim.x && blockDim.x <= 256 && nwc <= 8) {  // the whole CTA
+        if (nwc <= 1) greedy_block<1>(s, n, max_group);
+        else if (nwc <= 2) greedy_block<2>(s, n, max_group);
+        else if (nwc <= 4) greedy_block<4>(s, n, max_group);
+        else greedy_block<8>(s, n, max_group);
+        __syncthreads();
+        return;
+    }
     if (threadIdx.x < 32) {
         const int NWC = s.misc[1];
         if (n <= 64 && NWC <= 32) {

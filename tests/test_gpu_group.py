@@ -39,13 +39,30 @@ def test_random_small_bitexact(seed):
 
 
 @pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c", "5"])
-@pytest.mark.parametrize("window", [64, 8])
+@pytest.mark.parametrize("window", [64, 8, 256])
 def test_workload_bitexact(cfg, window):
     w = W.make(cfg)
     got = _run(w.topk, w.Hq, w.Hkv, w.num_logical_pages, 8, window)
     ref = oracle.group(w.topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, 8, window)
     assert_groups_equal(got, ref)
     assert_bundles_equal(got, oracle.bundle(ref, w.Hq, w.Hkv, w.Nq, 8))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_large_windows_small_universe_bitexact(seed):
+    """Windows of 65..256 queries whose pages fit 8 words: the whole-CTA greedy."""
+    rng = np.random.default_rng(300 + seed)
+    Hkv, g = int(rng.integers(1, 3)), int(rng.choice([1, 2, 4]))
+    max_group = min(int(rng.choice([1, 2, 4, 8])), 32 // g)
+    window = max_group * int(rng.integers(65 // max_group + 1, 256 // max_group + 1))
+    Nq = int(rng.integers(window // 2, 700))
+    K = int(rng.integers(1, 12))
+    P = int(rng.integers(8, 250))
+    topk = rng.integers(-1, P, size=(Hkv * g, Nq, K)).astype(np.int32)
+    got = _run(topk, Hkv * g, Hkv, P, max_group, window)
+    ref = oracle.group(topk, Hkv * g, Hkv, Nq, P, max_group, window)
+    assert_groups_equal(got, ref)
+    assert_bundles_equal(got, oracle.bundle(ref, Hkv * g, Hkv, Nq, max_group))
 
 
 def test_figure2_example_on_gpu():
