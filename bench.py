@@ -198,6 +198,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--window", type=int, default=None)
     ap.add_argument("--max-group", type=int, default=None)
+    ap.add_argument("--bundle-window", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -221,6 +222,7 @@ def main():
     w = W.make(args.config)
     max_group = args.max_group or w.max_group
     window = args.window or w.window
+    bundle_window = args.bundle_window if args.bundle_window is not None else w.bundle_window
     dev = {}
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     dev["Q"] = t(w.Q).view(torch.bfloat16) if w.q_dtype == W.DT_BF16 else t(w.Q)
@@ -231,6 +233,7 @@ def main():
     topk, page_table, q_pos = t(w.topk), t(w.page_table), t(w.q_pos)
     ws_bytes, cap = qup.group_workspace(w.Hq, w.Hkv, w.Nq, w.K, w.num_logical_pages, max_group, window)
     groups = qup.alloc_groups(w.Hq, w.Hkv, w.Nq, cap, ws_bytes, dev["Q"].device)
+    groups.bundle_window = bundle_window
     O = torch.empty_like(dev["Q"])
     stream = torch.cuda.current_stream()
 
@@ -305,7 +308,7 @@ def main():
         "data": "synthetic (seeded; shapes of the pages' prefill chunks)",
         "config": {"workload": w.name, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "d": w.d,
                    "page_tokens": w.T, "topk": w.K, "kv_len": w.kv_len, "max_group": max_group,
-                   "window": window, "l2": "flushed before every timed step (2x L2 write)",
+                   "window": window, "bundle_window": bundle_window, "l2": "flushed before every timed step (2x L2 write)",
                    "parallelism": f"replicas x{world} (independent chunks)"},
         "us_per_call": {"group": round(statistics.median(t_group) * 1e3, 2),
                         "attn": round(statistics.median(t_attn) * 1e3, 2),

@@ -225,6 +225,15 @@ int qup_set_debug(int wait_limit_ms, int skip_stage);
 /* Number of SMs the persistent attention kernel is sized for on the current device. */
 int qup_num_sms(void);
 
+/*
+ * Test hook (no counterpart on the pages): y[i] = 2^x[i] by the polynomial
+ * exponential the attention kernel uses for part of its softmax (x clamped to
+ * -127, where the result is exactly +0; x must be <= 16).  x and y are device
+ * float arrays of n elements; asynchronous on `stream`.  Returns QUP_ERR_ARG
+ * for n < 0 or null pointers with n > 0, QUP_ERR_CUDA for a launch failure.
+ */
+int qup_exp2_poly(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -69,8 +69,9 @@ def load():
     lib.qup_error_string.restype = ctypes.c_char_p
     lib.qup_set_debug.argtypes = [I, I]
     lib.qup_num_sms.argtypes = []
+    lib.qup_exp2_poly.argtypes = [P, P, I, P]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
-               "qup_get_error", "qup_set_debug", "qup_num_sms"):
+               "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -193,10 +194,12 @@ def build_bundles(gr: Groups, Hq: int, Hkv: int, Nq: int, num_logical_pages: int
 
 
 def sparse_group(topk, Hq: int, Hkv: int, num_logical_pages: int, max_group: int = 8,
-                 window: int = 64, out: Optional[Groups] = None, stream=None) -> Groups:
+                 window: int = 64, out: Optional[Groups] = None, stream=None,
+                 bundle_window: Optional[int] = None) -> Groups:
     """Page-affinity grouping of the queries of every KV head, then bundling (qup_sparse_group).
 
     topk: int32 CUDA tensor [Hq][Nq][Ksel], -1 = padding. Returns Groups on the device.
+    bundle_window: groups per bundling window (None keeps out's setting; 0 = library default).
     """
     lib = load()
     Hq_, Nq, Ksel = topk.shape
@@ -204,6 +207,8 @@ def sparse_group(topk, Hq: int, Hkv: int, num_logical_pages: int, max_group: int
     ws_bytes, cap = group_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window)
     if out is None:
         out = alloc_groups(Hq, Hkv, Nq, cap, ws_bytes, topk.device)
+    if bundle_window is not None:
+        out.bundle_window = int(bundle_window)
     cs = out.c_struct()
     _check(lib.qup_sparse_group(_p(topk), Hq, Hkv, Nq, Ksel, num_logical_pages, max_group, window,
                                 ctypes.byref(cs), _p(out.workspace), out.workspace.numel(),
@@ -253,6 +258,17 @@ def sparse_prefill_attn(Q, K_cache, V_cache, page_table, groups: Groups, q_pos, 
                                        _p(q_pos), kv_len, Hq, Hkv, Nq, d, float(softmax_scale),
                                        _p(out), _p(lse), _stream_ptr(stream)),
            "qup_sparse_prefill_attn")
+    return out
+
+
+def exp2_poly(x, out=None, stream=None):
+    """2^x by the attention softmax's polynomial exponential (test hook, qup_exp2_poly).
+    x: float32 CUDA tensor; returns a tensor of the same shape."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    _check(load().qup_exp2_poly(_p(x), _p(out), x.numel(), _stream_ptr(stream)), "qup_exp2_poly")
     return out
 
 

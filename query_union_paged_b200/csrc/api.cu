@@ -445,6 +445,11 @@ int qup_num_sms(void) {
     return device_state(&ds) == QUP_OK ? ds->sms : 0;
 }
 
+int qup_exp2_poly(const float* x, float* y, int n, void* stream) {
+    if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return QUP_ERR_ARG;
+    return qup::launch_exp2_poly(x, y, n, (cudaStream_t)stream) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+}
+
 }  // extern "C"
 
 namespace qup {

@@ -68,6 +68,9 @@ size_t attn_tile_bytes(int es);
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);
 
+// the softmax's polynomial 2^x over n floats (test hook)
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 struct GroupLaunch {
     const int32_t* topk;
     int Hq, Hkv, Nq, K, P, NW, max_group, W, nwin;

@@ -50,6 +50,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended in hardware (issuing
+// nothing) until the phase completes or about hint_ns have passed.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Non-blocking: true iff the phase with the given parity has completed.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -79,6 +92,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                 atomicOr(err, code);
                 return false;
             }
+        }
+    }
+}
+
+// mbar_wait for warps that share an SM sub-partition with a softmax warp: the
+// suspended try_wait leaves that sub-partition's issue slots to the softmax.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned* err, unsigned code, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = cycles();
+    for (;;) {
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (cycles() - t0 > limit_ns * kCyclesPerNs) {
+            *abort_flag = 1;
+            atomicOr(err, code);
+            return false;
         }
     }
 }
@@ -321,6 +351,77 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+
+// Two fp32 lanes in one 64-bit register pair: the packed fp32 pipe of sm_100
+// (add/sub/fma .f32x2) does both in one instruction.
+struct f2 {
+    float x, y;
+};
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^y for a pair of fp32 on the FMA pipe (offloads the MUFU unit).
+// Cody-Waite style reduction: n = round(y) by adding 1.5 * 2^23 (the sum's low
+// mantissa bits hold n), f = y - n in [-1/2, 1/2]; 2^f by a cubic
+// p(f) = 1 + f (c1 + f (c2 + f c3)) whose coefficients minimise the maximum
+// relative error on [-1/2, 1/2] (linear-programming fit, fit_exp2_poly.py:
+// max relative error 1.0e-4, below bf16's half ulp of 2^-9, so the rounded P
+// is the same as with the exact exponential except near ties); then n is added to p's exponent
+// field.  y is clamped to -127 first: there f = 0, p = 1 exactly and the
+// result is +0, so masked scores (-inf) give exactly 0.  Inputs above 127
+// overflow the exponent: callers keep y <= 16.
+constexpr float kExp2C1 = 0.6932829f, kExp2C2 = 0.24221095f, kExp2C3 = 0.055008937f;
+__device__ __forceinline__ f2 exp2_poly2(f2 y) {
+    const f2 kMagic{12582912.f, 12582912.f};
+    y.x = fmaxf(y.x, -127.f);
+    y.y = fmaxf(y.y, -127.f);
+    const f2 t = add2(y, kMagic);
+    const f2 n = sub2(t, kMagic);
+    const f2 f = sub2(y, n);
+    f2 p = fma2(f, f2{kExp2C3, kExp2C3}, f2{kExp2C2, kExp2C2});
+    p = fma2(p, f, f2{kExp2C1, kExp2C1});
+    p = fma2(p, f, f2{1.f, 1.f});
+    f2 r;
+    r.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
+    r.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+    return r;
+}
+
+// Orders later uses of registers written by tcgen05.ld after tcgen05.wait::ld
+// (the load's outputs are only valid once the wait has returned).
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* v) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(v[i]));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -18,7 +18,12 @@
 // A row's max is only raised when a score exceeds it by more than kTau (log2
 // units); O and the row sum are rescaled then, which after the first steps is
 // rare.  A warp whose 32 rows selected none of a step's pages skips that
-// step's exponentials.
+// step's exponentials.  Each softmax warp reads the bundle's page numbers and
+// its own 32-bit word of every page's row mask straight from the bundle
+// arrays, 32 entries at a time, one batch ahead; it waits for a V tile only
+// on a step whose page reaches kv_len (whose V rows past kv_len it zeroes).
+// bf16 P takes a quarter of its exponentials from a polynomial on the FMA pipe
+// (exp2_poly2) and the rest from the MUFU unit.
 //
 // Warp roles (256 threads):
 //   warps 0-3  softmax / epilogue: thread = TMEM lane = bundle row.  They
@@ -26,21 +31,20 @@
 //              Q tensor) into TMEM.
 //   warp 4     K producer: walks the bundle's page list, resolves physical
 //              pages (warp-parallel) and TMA-loads the K tiles.
-//   warp 6     V producer: the same walk for the V tiles; it also writes each
-//              step's page numbers and row masks, which live as long as the
-//              V slot (until the step's O update).
+//   warp 6     V producer: the same walk for the V tiles.
 //   warp 5     S issuer (one elected lane of a warp-uniform loop) and TMEM
 //              owner (512 columns): S(g) once K tile g has landed and the O
 //              update of step g - 2 has finished with S_b.
 //   warp 7     PV issuer: O += P_b V once P(g) and V tile g are ready.
 // The two issuers sit on different SM sub-partitions, each beside one softmax
-// warp and no other busy warp.
+// warp and no other busy warp; producers and issuers wait with suspended
+// try_waits, which leave the sub-partition's issue slots to the softmax.
 // TMEM columns: O [0,128); S_0 [128,256); S_1 [256,384); Q from 384 (bf16:
 // 64 columns, E4M3: 32; fp32 Q stays in shared memory).  P_b occupies the
 // first kPCols columns of S_b.
 // Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
 // FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
-// row with its own scale, P stored as E4M3 of 2^6 p).  Every MMA consumes 32
+// row with its own scale, P stored as E4M3 of 2^4 p).  Every MMA consumes 32
 // bytes of its K extent per row, so the descriptor arithmetic is shared.
 //
 // Every wait is bounded (ptx.cuh); on a timeout the CTA raises an abort flag,
@@ -62,13 +66,6 @@ constexpr int kTmemCols = 512;
 constexpr int kKProducerWarp = 4, kSWarp = 5, kVProducerWarp = 6, kPvWarp = 7;
 constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384;
 
-struct StageMeta {
-    int32_t upage[kMaxPPS];
-    uint32_t mask[kMaxPPS][4];
-    int32_t tok0;  // first token of the step inside its page (pages longer than a step)
-    int32_t pad[3];
-};
-
 template <int ES, int T>
 struct Geo {
     static constexpr int SPP = T > kST ? T / kST : 1;   // steps per page (not used: T <= 128)
@@ -88,13 +85,17 @@ struct Geo {
     static constexpr int kQCols = kD * ES / 4;          // TMEM columns of Q
     static_assert(!kQTmem || kColQ + kQCols <= kTmemCols, "TMEM budget");
     static_assert(kPCols <= 128, "P fits in its S buffer");
+    // exponentials on the FMA pipe by a polynomial: pairs (j / 2) % 8 < kPolyPairs of every 16
+    // columns; the rest go to the MUFU unit
+    static constexpr int kPolyPairs = ES == 2 ? 2 : 0;
     static_assert(PPS <= kMaxPPS, "pages per step");
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
-    static constexpr float kTau = ES == 1 ? 2.f : 8.f;  // lazy-rescale margin (log2 units)
-    // E4M3 P is stored as 2^kPLog2 p (p <= 2^kTau, so at most 256 < 448); the row sum carries
-    // the same factor, which cancels in O / l
-    static constexpr float kPLog2 = ES == 1 ? 6.f : 0.f;
+    static constexpr float kTau = ES == 1 ? 4.5f : 8.f;  // lazy-rescale margin (log2 units)
+    // E4M3 P is stored as 2^kPLog2 p (p <= 2^kTau, so at most 2^8.5 < 448, E4M3's largest
+    // finite value; a P below 2^-10 of its row's max is a subnormal of E4M3); the row sum
+    // carries the same factor, which cancels in O / l
+    static constexpr float kPLog2 = ES == 1 ? 4.f : 0.f;
 };
 
 struct SmemLayout {
@@ -113,7 +114,6 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     L.bars = off;
     off += 8u * (2u * (nsk + nsv) + 12u);
     L.meta = off;
-    off += (uint32_t)sizeof(StageMeta) * nsv;
     L.qsc = off;
     off += kRows * 4u;
     L.misc = off;
@@ -208,7 +208,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int NSK = p.nsk, NSV = p.nsv;
     const uint32_t sbase = smem_u32(smem);
     const Bars B{sbase + L.bars, NSK, NSV};
-    StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L.meta);
     float* qsc = reinterpret_cast<float*>(smem + L.qsc);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
@@ -285,10 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
                 const int idx = e0 + lane;
                 int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
-                uint4 mk = make_uint4(0, 0, 0, 0);
                 if (idx < it.nU) {
                     u = p.union_pages[it.ub + idx];
-                    if (isV) mk = reinterpret_cast<const uint4*>(p.row_mask)[it.ub + idx];
                     if (u < 0 || u >= p.num_logical_pages) {
                         atomicOr(p.err, QUP_ERR_PAGE_ID);
                         u = 0;
@@ -299,14 +296,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             phys = p.P_phys;
                         }
                     }
-                    if (phys == p.P_phys) mk = make_uint4(0, 0, 0, 0);
                 }
                 const int nst = min(32, n_ent - e0) / PPS;  // 32 is a multiple of PPS
                 for (int k = 0; k < nst; ++k, ++gs) {
                     const int slot = gs % NR;
                     int okv = 0;
                     if (lane == 0)
-                        okv = mbar_wait(isV ? B.vempty(slot) : B.kempty(slot), ((gs / NR) & 1) ^ 1, abort_flag,
+                        okv = mbar_wait_idle(isV ? B.vempty(slot) : B.kempty(slot), ((gs / NR) & 1) ^ 1, abort_flag,
                                         p.err, QUP_ERR_TIMEOUT, lim);
                     ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
                     if (!ok) break;
@@ -317,25 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int q = 0; q < PPS; ++q) {
                         const int src = k * PPS + q;
                         ph[q] = __shfl_sync(0xffffffffu, phys, src);
-                        if (isV) {
-                            const int uq = __shfl_sync(0xffffffffu, u, src);
-                            const uint32_t m0 = __shfl_sync(0xffffffffu, mk.x, src);
-                            const uint32_t m1 = __shfl_sync(0xffffffffu, mk.y, src);
-                            const uint32_t m2 = __shfl_sync(0xffffffffu, mk.z, src);
-                            const uint32_t m3 = __shfl_sync(0xffffffffu, mk.w, src);
-                            if (issue) {
-                                StageMeta& m = meta[slot];
-                                m.upage[q] = uq;
-                                m.mask[q][0] = m0;
-                                m.mask[q][1] = m1;
-                                m.mask[q][2] = m2;
-                                m.mask[q][3] = m3;
-                                m.tok0 = 0;
-                            }
-                        }
                     }
                     if (issue) {
-                        // the arrive releases the metadata stores; the copies complete the phase
                         const uint32_t fb = isV ? B.vfull(slot) : B.kfull(slot);
                         mbar_arrive_expect_tx(fb, G::kTile);
                         const uint32_t dst = ring + (uint32_t)slot * G::kTile;
@@ -388,13 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (f < 0) continue;
             const Item it = load_item<PPS>(p, nb_prefix, f);
             if (isS) {
-                ok = warp_ok(mbar_wait(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                ok = warp_ok(mbar_wait_idle(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                 if (!ok) break;
                 tc_fence_after();
                 for (int s = 0; s < it.nsteps; ++s) {
                     const int g = gs + s, b = g & 1;
-                    ok = warp_ok(mbar_wait(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 (g < 2 || mbar_wait(B.pvdone(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
+                    ok = warp_ok(mbar_wait_idle(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                 (g < 2 || mbar_wait_idle(B.pvdone(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
                                                      QUP_ERR_TIMEOUT, lim)));
                     if (!ok) break;
                     tc_fence_after();
@@ -424,8 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 for (int s = 0; s < it.nsteps; ++s) {
                     const int g = gs + s, b = g & 1;
-                    ok = warp_ok(mbar_wait(B.pfull(b), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 mbar_wait(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                    ok = warp_ok(mbar_wait_idle(B.pfull(b), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                 mbar_wait_idle(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
@@ -547,6 +526,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(B.qfull());
             float m_used = kNegInf, lsum = 0.f;
+            // a Q row of zeros (E4M3 scale 0) keeps a positive score scale: its scores are 0 anyway
+            cs = fmaxf(cs, 1e-30f);
+            const f2 cs2{cs, cs};
+            // The bundle's union entries, 32 at a time: lane j holds entry base + j, its logical
+            // page (-1 for padding or an entry the producers reject) and this warp's 32-bit word
+            // of the page's row mask.  The next 32 are loaded one batch ahead.
+            int cpage, npage;
+            uint32_t cmask, nmask;
+            int cbase = 0;
+            auto fetch = [&](int base, int& pg, uint32_t& mk) {
+                const int e = base + lane;
+                pg = -1;
+                mk = 0u;
+                if (e < it.nU) {
+                    const int u = p.union_pages[it.ub + e];
+                    const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + warp];
+                    if (u >= 0 && u < p.num_logical_pages) {
+                        const int ph = p.page_table[u];
+                        if (ph >= 0 && ph < p.P_phys) {
+                            pg = u;
+                            mk = m;
+                        }
+                    }
+                }
+            };
+            fetch(0, cpage, cmask);
+            fetch(32, npage, nmask);
+            // exponentials of one step: p = 2^(s*cs - m_used + kPLog2) into pk (or sv for fp32),
+            // and their sum
+            uint32_t sv[kST];
+            uint32_t pk[ES == 4 ? 1 : G::kPCols];
+            auto exps = [&](const int (&lim)[PPS]) -> float {
+                const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
+                f2 part[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token column
+#pragma unroll
+                for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
+                    // a page the row did not select gets an infinite offset: 2^-inf = 0
+                    const float off = lim[q] == 0 ? kPosInf : mb;
+                    const f2 noff{-off, -off};
+#pragma unroll
+                    for (int j = q * T; j < (q + 1) * T; j += 2) {
+                        const f2 y = fma2(f2{__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])}, cs2, noff);
+                        f2 e;
+                        if (((j >> 1) & 7) < G::kPolyPairs) {
+                            e = exp2_poly2(y);
+                        } else {
+                            e.x = ex2(y.x);
+                            e.y = ex2(y.y);
+                        }
+                        part[(j >> 1) & 3] = add2(part[(j >> 1) & 3], e);
+                        if constexpr (ES == 2) {
+                            pk[j / 2] = pack_bf16x2(e.x, e.y);
+                        } else if constexpr (ES == 4) {
+                            sv[j] = __float_as_uint(e.x);
+                            sv[j + 1] = __float_as_uint(e.y);
+                        } else {  // E4M3: four tokens per 32-bit column
+                            if (j & 2)
+                                pk[j / 4] = pack_e4m3x4(e_prev.x, e_prev.y, e.x, e.y);
+                            else
+                                e_prev = e;
+                        }
+                    }
+                }
+                const f2 ps = add2(add2(part[0], part[1]), add2(part[2], part[3]));
+                return ps.x + ps.y;
+            };
 
             for (int s = 0; s < it.nsteps; ++s) {
                 const int gstep = gs + s, b = gstep & 1, slot = vs;
@@ -555,25 +601,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     vs = 0;
                     vph ^= 1;
                 }
-                if (ok)
-                    ok = warp_ok(mbar_wait(B.vfull(slot), vphase, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 mbar_wait(B.sfull(b), (gstep >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                // this step's pages and mask words (PPS divides 32: a step never spans two batches)
+                const int e0 = s * PPS;
+                if (e0 >= cbase + 32) {
+                    cbase += 32;
+                    cpage = npage;
+                    cmask = nmask;
+                    fetch(cbase + 32, npage, nmask);
+                }
+                // row r sees token t of page q iff the page is in its own TopK row (its bit of the
+                // page's mask) and the token's position is < vis_end; a page that reaches kv_len
+                // may hold non-finite bytes past it (a tail step)
+                int lim_q[PPS];
+                bool live = false, partial = false, tail = false;
+#pragma unroll
+                for (int q = 0; q < PPS; ++q) {
+                    const int pg = __shfl_sync(0xffffffffu, cpage, e0 - cbase + q);
+                    const uint32_t mw = __shfl_sync(0xffffffffu, cmask, e0 - cbase + q);
+                    const bool mine = pg >= 0 && ((mw >> lane) & 1u);
+                    lim_q[q] = mine ? max(0, min(T, vis_end - pg * T)) : 0;
+                    live |= lim_q[q] > 0;
+                    partial |= lim_q[q] > 0 && lim_q[q] < T;
+                    tail |= pg >= 0 && pg * T + T > p.kv_len;
+                }
+                if (ok) ok = warp_ok(mbar_wait(B.sfull(b), (gstep >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                if (ok && tail) ok = warp_ok(mbar_wait(B.vfull(slot), vphase, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                 if (!ok) continue;
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_base + kColS + 128u * b;
-                uint32_t sv[kST];
 #pragma unroll
                 for (int i = 0; i < kST / 32; ++i)
                     tmem_ld32(s_addr + 32u * i, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * i));
-                const StageMeta& mt = meta[slot];
-                // a page of the step that reaches kv_len: its cache slots at or past kv_len may
-                // hold non-finite bytes, so those V rows are zeroed and the step's scores masked
-                bool tail = false;
-#pragma unroll
-                for (int q = 0; q < PPS; ++q) tail |= mt.upage[q] * T + T > p.kv_len;
-                if (tail) {  // thread r zeroes token row r of the step if it lies past kv_len
+                if (tail) {  // thread r zeroes V token row r of the step if it lies past kv_len
                     const int q = r / T;
-                    if (mt.upage[q] * T + (r - q * T) >= p.kv_len) {
+                    const int pg = __shfl_sync(0xffffffffu, cpage, e0 - cbase + q);
+                    if (pg >= 0 && pg * T + (r - q * T) >= p.kv_len) {
                         uint8_t* vt = smem + L.vst + (uint32_t)slot * G::kTile;
 #pragma unroll
                         for (int c = 0; c < G::kNChunk; ++c)
@@ -583,107 +645,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     make_uint4(0, 0, 0, 0);
                     }
                 }
-                // row r sees token t of page q iff the page is in its own TopK row (bit r of
-                // the page's mask) and the token's position is < vis_end
-                int lim_q[PPS];
-                bool live = false, partial = false;
-#pragma unroll
-                for (int q = 0; q < PPS; ++q) {
-                    const bool mine = (mt.mask[q][r >> 5] >> (r & 31)) & 1u;
-                    lim_q[q] = mine ? max(0, min(T, vis_end - mt.upage[q] * T)) : 0;
-                    live |= lim_q[q] > 0;
-                    partial |= lim_q[q] > 0 && lim_q[q] < T;
-                }
                 tmem_wait_ld();
+                reg_fence<kST>(sv);
                 const bool warp_live = __any_sync(0xffffffffu, live);
-                // Fast path (every page of the step fully seen or fully unseen by each row, no
-                // kv_len tail): the max is taken over the raw scores of seen pages (cs > 0) and
-                // each exponent is one FMA, an unseen page getting an infinite offset.
-                // Otherwise every score is scaled and masked first.
-                const bool slow = tail || __any_sync(0xffffffffu, partial);
-                float mloc = kNegInf;
-                if (warp_live) {
-                    if (!slow) {
+                // Raw scores of unseen tokens (past the row's causal limit or kv_len inside a page
+                // it selected) become -inf; pages the row did not select get an infinite offset in
+                // the exponent.  cs > 0, so the max of raw scores orders the scaled ones.
+                if (warp_live && (tail || __any_sync(0xffffffffu, partial))) {
 #pragma unroll
-                        for (int q = 0; q < PPS; ++q) {
-                            float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
-#pragma unroll
-                            for (int j = q * T; j < (q + 1) * T; ++j)
-                                mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(sv[j]));
-                            const float mq = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                            if (lim_q[q] > 0) mloc = fmaxf(mloc, mq * cs);
-                        }
-                    } else {
-                        float mx[8];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) mx[k] = kNegInf;
-#pragma unroll
-                        for (int j = 0; j < kST; ++j) {
-                            const int q = j / T, t = j - q * T;
-                            const float v = t < lim_q[q] ? __uint_as_float(sv[j]) * cs : kNegInf;
-                            sv[j] = __float_as_uint(v);
-                            mx[j & 7] = fmaxf(mx[j & 7], v);
-                        }
-                        mloc = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                    for (int j = 0; j < kST; ++j) {
+                        const int q = j / T, t = j - q * T;
+                        if (t >= lim_q[q]) sv[j] = __float_as_uint(kNegInf);
                     }
                 }
-                // lazy running max: raise it only when a score exceeds it by more than kTau
-                const bool need = mloc > m_used + G::kTau;
+                bool need = false;
                 float alpha = 1.f;
-                if (need) {
-                    alpha = ex2(m_used - mloc);  // 0 when m_used is -inf
-                    m_used = mloc;
-                    lsum *= alpha;
-                }
-                // packed P (fp32 P is written back into sv: it has the width of S)
-                uint32_t pk[ES == 4 ? 1 : G::kPCols];
                 if (warp_live) {
-                    // p = 2^(x - m + kPLog2); on the fast path an unseen page gets x - inf = -inf
-                    const float xs = slow ? 1.f : cs;
-                    const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
-                    float off[PPS];
+                    float mloc = kNegInf;
 #pragma unroll
-                    for (int q = 0; q < PPS; ++q) off[q] = (!slow && lim_q[q] == 0) ? kPosInf : mb;
-                    float part[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int q = 0; q < PPS; ++q) {
+                        float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-                    for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
-                        // (skipping the pages none of a warp's rows selected unbalances the four
-                        // warps, and each step waits for the slowest: measured slower)
-                        if constexpr (ES == 2) {
+                        for (int j = q * T; j < (q + 1) * T; j += 8) {
 #pragma unroll
-                            for (int j = q * T; j < (q + 1) * T; j += 2) {
-                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
-                                part[(j >> 1) & 3] += p0 + p1;
-                                pk[j / 2] = pack_bf16x2(p0, p1);
-                            }
-                        } else if constexpr (ES == 4) {
-#pragma unroll
-                            for (int j = q * T; j < (q + 1) * T; ++j) {
-                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                part[j & 3] += p0;
-                                sv[j] = __float_as_uint(p0);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = q * T; j < (q + 1) * T; j += 4) {
-                                const float p0 = ex2(fmaf(__uint_as_float(sv[j]), xs, -off[q]));
-                                const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), xs, -off[q]));
-                                const float p2 = ex2(fmaf(__uint_as_float(sv[j + 2]), xs, -off[q]));
-                                const float p3 = ex2(fmaf(__uint_as_float(sv[j + 3]), xs, -off[q]));
-                                part[(j >> 2) & 3] += (p0 + p1) + (p2 + p3);
-                                pk[j / 4] = pack_e4m3x4(p0, p1, p2, p3);
-                            }
+                            for (int k = 0; k < 4; ++k)
+                                mx[k] = max3f(mx[k], __uint_as_float(sv[j + 2 * k]), __uint_as_float(sv[j + 2 * k + 1]));
                         }
+                        const float mq = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                        if (lim_q[q] > 0) mloc = fmaxf(mloc, mq * cs);
                     }
-                    lsum += (part[0] + part[1]) + (part[2] + part[3]);
-                } else if constexpr (ES == 4) {
-#pragma unroll
-                    for (int j = 0; j < kST; ++j) sv[j] = 0u;
+                    // lazy running max: raise it only when a score exceeds it by more than kTau
+                    need = mloc > m_used + G::kTau;
+                    if (need) {
+                        alpha = ex2(m_used - mloc);  // 0 when m_used is -inf
+                        m_used = mloc;
+                        lsum *= alpha;
+                    }
+                    lsum += exps(lim_q);
                 } else {
+                    if constexpr (ES == 4) {
 #pragma unroll
-                    for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
+                        for (int j = 0; j < kST; ++j) sv[j] = 0u;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
+                    }
                 }
                 // O is rescaled only after every earlier O update has finished (rare)
                 if (s > 0 && __any_sync(0xffffffffu, need)) {
@@ -696,6 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t ov[32];
                         tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
                         tmem_wait_ld();
+                        reg_fence<32>(ov);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                         tmem_st_x32(tmem + lane_base + kColO + 32u * c, ov);
@@ -760,6 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     lsum > 0.f ? (m_used + __log2f(lsum) - G::kPLog2) * 0.69314718055994531f : kNegInf;
             tc_fence_before();
         }
+        tmem_wait_ld();  // a prefetched S load left behind by an aborted walk
     }
 
     // ---------------------------------------------------------------- teardown
@@ -779,6 +787,21 @@ static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, cons
     cudaError_t e = ensure_smem_attr((const void*)union_attn_kernel<ES, T>, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(union_attn_kernel<ES, T>, dim3(grid), dim3(kThreads), smem, stream, tmK, tmV, p);
+}
+
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const f2 r = exp2_poly2(f2{x[i], i + 1 < n ? x[i + 1] : 0.f});
+    y[i] = r.x;
+    if (i + 1 < n) y[i + 1] = r.y;
+}
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const int threads = 256, pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + threads - 1) / threads, threads, 0, stream>>>(x, y, n);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p,

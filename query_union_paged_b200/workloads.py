@@ -54,6 +54,7 @@ class Workload:
     q_pos: np.ndarray
     max_group: int = 8
     window: int = 64
+    bundle_window: int = 64
 
     @property
     def g(self) -> int:
