@@ -365,10 +365,10 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     // a pipeline step is 128 tokens: as many K and V tiles in flight as shared memory allows,
     // split between the K ring and the V ring (a V slot is held longer: through the softmax)
     int nt = 2 * qup::kMaxStages;
-    while (nt >= 2 && qup::attn_smem_bytes(es, nt / 2, nt - nt / 2, Hkv) > (size_t)ds->smem_optin) --nt;
+    while (nt >= 2 && qup::attn_smem_bytes(es, nt / 2, nt - nt / 2, Hkv, g) > (size_t)ds->smem_optin) --nt;
     if (nt < 2) return QUP_ERR_ARG;
     const int nsk = nt / 2, nsv = nt - nt / 2;
-    const size_t smem = qup::attn_smem_bytes(es, nsk, nsv, Hkv);
+    const size_t smem = qup::attn_smem_bytes(es, nsk, nsv, Hkv, g);
 
     qup::AttnParams p;
     std::memset(&p, 0, sizeof(p));

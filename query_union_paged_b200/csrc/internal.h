@@ -62,7 +62,7 @@ struct AttnParams {
 
 // dynamic shared memory of the attention kernel for (element size, K slots, V slots, KV heads),
 // and one K or V tile (one ring slot)
-size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv);
+size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g);
 size_t attn_tile_bytes(int es);
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,

@@ -25,13 +25,19 @@
 // bf16 P takes a quarter of its exponentials from a polynomial on the FMA pipe
 // (exp2_poly2) and the rest from the MUFU unit.
 //
+// Bundle boundaries: the V warp stages each bundle a few steps ahead (header,
+// query IDs and positions, and the bundle's Q rows by original query ID,
+// bulk-copied into shared memory); right after a bundle's last P the softmax
+// warps move the next bundle's Q rows into the other of two TMEM Q buffers,
+// so the next bundle's first S = Q K^T runs during this bundle's epilogue.
+//
 // Warp roles (256 threads):
 //   warps 0-3  softmax / epilogue: thread = TMEM lane = bundle row.  They
-//              also gather the rows of Q by original query ID (no reordered
-//              Q tensor) into TMEM.
+//              also move each bundle's Q rows (gathered by original query ID:
+//              no reordered Q tensor) into TMEM.
 //   warp 4     K producer: walks the bundle's page list, resolves physical
 //              pages (warp-parallel) and TMA-loads the K tiles.
-//   warp 6     V producer: the same walk for the V tiles.
+//   warp 6     V producer: the same walk for the V tiles; stages each bundle.
 //   warp 5     S issuer (one elected lane of a warp-uniform loop) and TMEM
 //              owner (512 columns): S(g) once K tile g has landed and the O
 //              update of step g - 2 has finished with S_b.
@@ -39,9 +45,9 @@
 // The two issuers sit on different SM sub-partitions, each beside one softmax
 // warp and no other busy warp; producers and issuers wait with suspended
 // try_waits, which leave the sub-partition's issue slots to the softmax.
-// TMEM columns: O [0,128); S_0 [128,256); S_1 [256,384); Q from 384 (bf16:
-// 64 columns, E4M3: 32; fp32 Q stays in shared memory).  P_b occupies the
-// first kPCols columns of S_b.
+// TMEM columns: O [0,128); S_0 [128,256); S_1 [256,384); two Q buffers from
+// 384 (bf16: 64 columns each, E4M3: 32; fp32 Q stays in shared memory).  P_b
+// occupies the first kPCols columns of S_b.
 // Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
 // FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
 // row with its own scale, P stored as E4M3 of 2^4 p).  Every MMA consumes 32
@@ -83,7 +89,7 @@ struct Geo {
     static constexpr int kPCols = kST * ES / 4;         // TMEM columns of P
     static constexpr bool kQTmem = ES != 4;             // Q as the TMEM A operand (bf16, E4M3)
     static constexpr int kQCols = kD * ES / 4;          // TMEM columns of Q
-    static_assert(!kQTmem || kColQ + kQCols <= kTmemCols, "TMEM budget");
+    static_assert(!kQTmem || kColQ + 2 * kQCols <= kTmemCols, "TMEM budget (two Q buffers)");
     static_assert(kPCols <= 128, "P fits in its S buffer");
     // exponentials on the FMA pipe by a polynomial: pairs (j / 2) % 8 < kPolyPairs of every 16
     // columns; the rest go to the MUFU unit
@@ -99,10 +105,15 @@ struct Geo {
 };
 
 struct SmemLayout {
-    uint32_t kst, vst, q, bars, meta, qsc, misc, total;
+    uint32_t kst, vst, q, qst, sinfo, bars, misc, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv) {
+// Stage of the next bundle (bf16 Q rows): query slot m holds the g rows of its query, 256 bytes
+// each, at m * qstage_stride(g); the 16-byte pad keeps row reads free of bank conflicts.
+__host__ __device__ inline uint32_t qstage_stride(int g) { return (uint32_t)g * 256u + 16u; }
+constexpr int kSinfoWords = 8;  // stage header: flat bundle, h, bi, ub, nU, nsteps, ok
+
+__host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv, int g) {
     SmemLayout L;
     uint32_t off = 0;
     L.kst = off;
@@ -111,11 +122,12 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     off += (uint32_t)nsv * kST * kD * es;
     L.q = off;
     if (es == 4) off += (uint32_t)kRows * kD * es;  // fp32 Q stays in shared memory
+    L.qst = off;
+    if (es != 4) off += (uint32_t)(kRows / g) * qstage_stride(g);
+    L.sinfo = off;
+    off += 4u * (kSinfoWords + 2 * kRows);  // header, qid[128 / g], q_pos[128 / g]
     L.bars = off;
     off += 8u * (2u * (nsk + nsv) + 12u);
-    L.meta = off;
-    L.qsc = off;
-    off += kRows * 4u;
     L.misc = off;
     off += 16u + 4u * (uint32_t)(Hkv + 1);
     L.total = off + 1024u;  // slack for aligning the dynamic base to 1024
@@ -137,6 +149,8 @@ struct Bars {
     __device__ __forceinline__ uint32_t qfull() const { return fixed(6); }
     __device__ __forceinline__ uint32_t drain() const { return fixed(7); }
     __device__ __forceinline__ uint32_t drain2() const { return fixed(8); }
+    __device__ __forceinline__ uint32_t stfull() const { return fixed(9); }
+    __device__ __forceinline__ uint32_t stempty() const { return fixed(10); }
 };
 
 struct Item {
@@ -204,11 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(ES, p.nsk, p.nsv, p.Hkv);
+    const SmemLayout L = smem_layout(ES, p.nsk, p.nsv, p.Hkv, p.g);
     const int NSK = p.nsk, NSV = p.nsv;
     const uint32_t sbase = smem_u32(smem);
     const Bars B{sbase + L.bars, NSK, NSV};
-    float* qsc = reinterpret_cast<float*>(smem + L.qsc);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
     int* nb_prefix = reinterpret_cast<int*>(smem + L.misc + 16);
@@ -235,6 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(B.qfull(), 4);
         mbar_init(B.drain(), 1);
         mbar_init(B.drain2(), 1);
+        mbar_init(B.stfull(), 1);
+        mbar_init(B.stempty(), 4);  // one arrive per softmax warp
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -273,13 +288,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int NR = isV ? NSV : NSK;
         const CUtensorMap* tm = isV ? &tmV : &tmK;
         const uint32_t ring = sbase + (isV ? L.vst : L.kst);
-        int gs = 0;
+        int gs = 0, n_staged = 0;
         bool ok = true;
         for (int rnd = 0; ok; ++rnd) {
             const int f = item_at(p, rnd, n_items);
             if (f == -1) break;
             if (f < 0) continue;
             const Item it = load_item<PPS>(p, nb_prefix, f);
+            if constexpr (ES != 4) {
+                // The V warp stages the bundle for the softmax warps (a few steps before they reach
+                // it): header, query IDs and positions of its query slots, and its Q rows (bulk
+                // copies by original query ID: the g rows of a query are contiguous in Q).
+                if (isV) {
+                    if (n_staged > 0) {  // the softmax warps have read the previous stage
+                        int okv = 0;
+                        if (lane == 0)
+                            okv = mbar_wait_idle(B.stempty(), (n_staged - 1) & 1, abort_flag, p.err,
+                                                 QUP_ERR_TIMEOUT, lim);
+                        ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
+                        if (!ok) break;
+                    }
+                    int* sinfo = reinterpret_cast<int*>(smem + L.sinfo);
+                    const int MQ = kRows / p.g;
+                    int nvalid = 0;
+                    for (int m0 = 0; m0 < MQ; m0 += 32) {
+                        const int m = m0 + lane;
+                        int qid = -1;
+                        if (m < MQ) {
+                            qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + m];
+                            if (qid >= p.Nq) {
+                                atomicOr(p.err, QUP_ERR_GROUP);
+                                qid = -1;
+                            }
+                            qid = max(qid, -1);
+                            sinfo[kSinfoWords + m] = qid;
+                            sinfo[kSinfoWords + kRows + m] = qid >= 0 ? p.q_pos[qid] : -1;
+                        }
+                        nvalid += __popc(__ballot_sync(0xffffffffu, qid >= 0));
+                    }
+                    if (lane == 0) {
+                        sinfo[0] = f;
+                        sinfo[1] = it.h;
+                        sinfo[2] = it.bi;
+                        sinfo[3] = it.ub;
+                        sinfo[4] = it.nU;
+                        sinfo[5] = it.nsteps;
+                        sinfo[6] = it.ok ? 1 : 0;
+                    }
+                    __syncwarp();
+                    const uint32_t qbytes = (uint32_t)p.g * kD * 2u;
+                    if (lane == 0) mbar_arrive_expect_tx(B.stfull(), (uint32_t)nvalid * qbytes);
+                    __syncwarp();
+                    for (int m = lane; m < MQ; m += 32) {
+                        const int qid = sinfo[kSinfoWords + m];
+                        if (qid >= 0)
+                            bulk_g2s(sbase + L.qst + (uint32_t)m * qstage_stride(p.g),
+                                     static_cast<const uint16_t*>(p.Q) + ((size_t)qid * p.Hq + (size_t)it.h * p.g) * kD,
+                                     qbytes, B.stfull());
+                    }
+                    ++n_staged;
+                }
+            }
             const int n_ent = it.nsteps * PPS;  // incl. padding of the last step
             for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
                 const int idx = e0 + lane;
@@ -335,8 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        // every issued load lands before the CTA may exit: the last NR stages of this ring
+        // every issued load lands before the CTA may exit: the last NR stages of this ring, and
+        // the last stage of Q rows
         if (lane == 0) {
+            if (n_staged > 0) mbar_wait_drain(B.stfull(), (n_staged - 1) & 1, lim);
             for (int i = max(0, gs - NR); i < gs; ++i) {
                 if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
                 mbar_wait_drain(isV ? B.vfull(i % NR) : B.kfull(i % NR), (i / NR) & 1, lim);
@@ -384,7 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < G::kNumMmaS; ++k) {
                             const uint32_t koff = ((k >> 2) * G::kChunkBytes + (k & 3) * 32) >> 4;
                             if constexpr (G::kQTmem) {
-                                tc_mma_ts<G::kKind>(tmem + kColS + 128u * b, tmem + kColQ + 8u * k, kdesc + koff,
+                                tc_mma_ts<G::kKind>(tmem + kColS + 128u * b,
+                                                    tmem + kColQ + (uint32_t)(item_no & 1) * G::kQCols + 8u * k, kdesc + koff,
                                                     idesc_s, k > 0);
                             } else {
                                 const uint32_t qoff = ((k >> 2) * G::kQChunkBytes + (k & 3) * 32) >> 4;
@@ -442,158 +514,198 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float kNegInf = -__int_as_float(0x7f800000);
         const float kPosInf = __int_as_float(0x7f800000);
         const int g = p.g, MQ = kRows / g;
+        const int* sinfo = reinterpret_cast<const int*>(smem + L.sinfo);
         int gs = 0, vs = 0, vph = 0;
         bool ok = true;
-        for (int rnd = 0;; ++rnd) {
-            const int f = item_at(p, rnd, n_items);
-            if (f == -1) break;
-            if (f < 0) {
-                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
-                continue;
+        // the row's bundle state: item, query (original ID), Q head, visible positions, score scale
+        Item it{};
+        int qid = -1, head = 0, vis_end = 0;
+        float cs = p.scale_log2;
+        float m_used = kNegInf, lsum = 0.f;
+        f2 cs2{cs, cs};
+        // The bundle's union entries, 32 at a time: lane j holds entry base + j, its logical
+        // page (-1 for padding or an entry the producers reject) and this warp's 32-bit word
+        // of the page's row mask.  The next 32 are loaded one batch ahead.
+        int cpage = -1, npage = -1;
+        uint32_t cmask = 0u, nmask = 0u;
+        int cbase = 0;
+        auto fetch = [&](int base, int& pg, uint32_t& mk) {
+            const int e = base + lane;
+            pg = -1;
+            mk = 0u;
+            if (e < it.nU) {
+                const int u = p.union_pages[it.ub + e];
+                const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + warp];
+                if (u >= 0 && u < p.num_logical_pages) {
+                    const int ph = p.page_table[u];
+                    if (ph >= 0 && ph < p.P_phys) {
+                        pg = u;
+                        mk = m;
+                    }
+                }
             }
-            const Item it = load_item<PPS>(p, nb_prefix, f);
+        };
+        // Take over flat bundle ff, the ino-th of this CTA: its header and this row's query
+        // (bf16 Q: from the stage the V warp filled; fp32 Q: from global memory), the first union
+        // entries, and this row of Q by original query ID into the bundle's TMEM Q buffer (fp32:
+        // the shared-memory Q tile).  Arrives on the Q barrier (and releases the stage).
+        auto take = [&](int ff, int ino) -> bool {
+            int qpos = -1;
+            if constexpr (ES != 4) {
+                if (!warp_ok(mbar_wait(B.stfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
+                it.h = sinfo[1];
+                it.bi = sinfo[2];
+                it.ub = sinfo[3];
+                it.nU = sinfo[4];
+                it.nsteps = sinfo[5];
+                it.ok = sinfo[6] != 0;
+                qid = sinfo[kSinfoWords + r / g];
+                qpos = sinfo[kSinfoWords + kRows + r / g];
+            } else {
+                it = load_item<PPS>(p, nb_prefix, ff);
+                qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
+                if (qid >= p.Nq) {
+                    atomicOr(p.err, QUP_ERR_GROUP);
+                    qid = -1;
+                }
+                qid = max(qid, -1);
+                qpos = qid >= 0 ? p.q_pos[qid] : -1;
+            }
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
-            // ---- this row's query (original ID) and head
-            int qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
-            if (qid >= p.Nq) {
-                atomicOr(p.err, QUP_ERR_GROUP);
-                qid = -1;
-            }
-            const int head = it.h * g + (r % g);
-            const int qpos = qid >= 0 ? p.q_pos[qid] : -1;
-            const int vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
-            float cs = p.scale_log2;                      // score scale (log2 domain) of this row
-            // ---- Q row by original ID -> TMEM (bf16, E4M3) or the shared-memory tile (fp32)
-            {
-                const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
-                if constexpr (ES == 2) {
-                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t qv[32];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint4 v = qid >= 0 ? src[half * 8 + c] : make_uint4(0, 0, 0, 0);
-                            qv[4 * c] = v.x;
-                            qv[4 * c + 1] = v.y;
-                            qv[4 * c + 2] = v.z;
-                            qv[4 * c + 3] = v.w;
-                        }
-                        tmem_st_x32(tmem + lane_base + kColQ + 32u * half, qv);
-                    }
-                } else if constexpr (ES == 4) {
-                    uint8_t* qt = smem + L.q;
-                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
-                    }
-                    fence_proxy_async_smem();
-                } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
-                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.Q) + row_off);
-                    uint4 raw[16];
-                    float amax = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        raw[c] = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                        const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
-                                                     fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
-                    }
-                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
-                    uint32_t qv[32];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
-                        const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-                        float x[8];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
-                            x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
-                        }
-                        qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-                        qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
-                    }
-                    tmem_st_x32(tmem + lane_base + kColQ, qv);
-                    cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
-                }
-                if constexpr (G::kQTmem) tmem_wait_st();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(B.qfull());
-            float m_used = kNegInf, lsum = 0.f;
-            // a Q row of zeros (E4M3 scale 0) keeps a positive score scale: its scores are 0 anyway
-            cs = fmaxf(cs, 1e-30f);
-            const f2 cs2{cs, cs};
-            // The bundle's union entries, 32 at a time: lane j holds entry base + j, its logical
-            // page (-1 for padding or an entry the producers reject) and this warp's 32-bit word
-            // of the page's row mask.  The next 32 are loaded one batch ahead.
-            int cpage, npage;
-            uint32_t cmask, nmask;
-            int cbase = 0;
-            auto fetch = [&](int base, int& pg, uint32_t& mk) {
-                const int e = base + lane;
-                pg = -1;
-                mk = 0u;
-                if (e < it.nU) {
-                    const int u = p.union_pages[it.ub + e];
-                    const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + warp];
-                    if (u >= 0 && u < p.num_logical_pages) {
-                        const int ph = p.page_table[u];
-                        if (ph >= 0 && ph < p.P_phys) {
-                            pg = u;
-                            mk = m;
-                        }
-                    }
-                }
-            };
+            head = it.h * g + (r % g);
+            vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
+            cs = p.scale_log2;                  // score scale (log2 domain) of this row
+            cbase = 0;
             fetch(0, cpage, cmask);
             fetch(32, npage, nmask);
-            // exponentials of one step: p = 2^(s*cs - m_used + kPLog2) into pk (or sv for fp32),
-            // and their sum
-            uint32_t sv[kST];
-            uint32_t pk[ES == 4 ? 1 : G::kPCols];
-            auto exps = [&](const int (&lim)[PPS]) -> float {
-                const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
-                f2 part[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-                f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token column
+            const uint32_t qcol = kColQ + (uint32_t)(ino & 1) * G::kQCols;
+            if constexpr (ES == 2) {
+                const uint8_t* row = smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
 #pragma unroll
-                for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
-                    // a page the row did not select gets an infinite offset: 2^-inf = 0
-                    const float off = lim[q] == 0 ? kPosInf : mb;
-                    const f2 noff{-off, -off};
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t qv[32];
 #pragma unroll
-                    for (int j = q * T; j < (q + 1) * T; j += 2) {
-                        const f2 y = fma2(f2{__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])}, cs2, noff);
-                        f2 e;
-                        if (((j >> 1) & 7) < G::kPolyPairs) {
-                            e = exp2_poly2(y);
-                        } else {
-                            e.x = ex2(y.x);
-                            e.y = ex2(y.y);
-                        }
-                        part[(j >> 1) & 3] = add2(part[(j >> 1) & 3], e);
-                        if constexpr (ES == 2) {
-                            pk[j / 2] = pack_bf16x2(e.x, e.y);
-                        } else if constexpr (ES == 4) {
-                            sv[j] = __float_as_uint(e.x);
-                            sv[j + 1] = __float_as_uint(e.y);
-                        } else {  // E4M3: four tokens per 32-bit column
-                            if (j & 2)
-                                pk[j / 4] = pack_e4m3x4(e_prev.x, e_prev.y, e.x, e.y);
-                            else
-                                e_prev = e;
-                        }
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v =
+                            qid >= 0 ? *reinterpret_cast<const uint4*>(row + half * 128 + c * 16) : make_uint4(0, 0, 0, 0);
+                        qv[4 * c] = v.x;
+                        qv[4 * c + 1] = v.y;
+                        qv[4 * c + 2] = v.z;
+                        qv[4 * c + 3] = v.w;
+                    }
+                    tmem_st_x32(tmem + lane_base + qcol + 32u * half, qv);
+                }
+            } else if constexpr (ES == 4) {
+                uint8_t* qt = smem + L.q;
+                const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+                const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
+                }
+                fence_proxy_async_smem();
+            } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
+                const uint8_t* row = smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
+                uint4 raw[16];
+                float amax = 0.f;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    raw[c] = qid >= 0 ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0, 0, 0, 0);
+                    const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                                 fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+                }
+                const float inv = amax > 0.f ? 448.f / amax : 0.f;
+                uint32_t qv[32];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
+                    const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
+                        x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
+                    }
+                    qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                    qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                }
+                tmem_st_x32(tmem + lane_base + qcol, qv);
+                cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
+            }
+            if constexpr (G::kQTmem) tmem_wait_st();
+            // a Q row of zeros (E4M3 scale 0) keeps a positive score scale: its scores are 0 anyway
+            cs = fmaxf(cs, 1e-30f);
+            cs2 = f2{cs, cs};
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(B.qfull());
+                if constexpr (ES != 4) mbar_arrive(B.stempty());
+            }
+            return true;
+        };
+        // the walk of bundles: -1 past the end; order entries that are bad are reported and skipped
+        auto walk = [&](int& rr) -> int {
+            int ff = item_at(p, rr, n_items);
+            while (ff == -2) {
+                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
+                ff = item_at(p, ++rr, n_items);
+            }
+            return ff;
+        };
+        // exponentials of one step: p = 2^(s*cs - m_used + kPLog2) into pk (or sv for fp32),
+        // and their sum
+        uint32_t sv[kST];
+        uint32_t pk[ES == 4 ? 1 : G::kPCols];
+        auto exps = [&](const int (&lim)[PPS]) -> float {
+            const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
+            f2 part[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token column
+#pragma unroll
+            for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
+                // a page the row did not select gets an infinite offset: 2^-inf = 0
+                const float off = lim[q] == 0 ? kPosInf : mb;
+                const f2 noff{-off, -off};
+#pragma unroll
+                for (int j = q * T; j < (q + 1) * T; j += 2) {
+                    const f2 y = fma2(f2{__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])}, cs2, noff);
+                    f2 e;
+                    if (((j >> 1) & 7) < G::kPolyPairs) {
+                        e = exp2_poly2(y);
+                    } else {
+                        e.x = ex2(y.x);
+                        e.y = ex2(y.y);
+                    }
+                    part[(j >> 1) & 3] = add2(part[(j >> 1) & 3], e);
+                    if constexpr (ES == 2) {
+                        pk[j / 2] = pack_bf16x2(e.x, e.y);
+                    } else if constexpr (ES == 4) {
+                        sv[j] = __float_as_uint(e.x);
+                        sv[j + 1] = __float_as_uint(e.y);
+                    } else {  // E4M3: four tokens per 32-bit column
+                        if (j & 2)
+                            pk[j / 4] = pack_e4m3x4(e_prev.x, e_prev.y, e.x, e.y);
+                        else
+                            e_prev = e;
                     }
                 }
-                const f2 ps = add2(add2(part[0], part[1]), add2(part[2], part[3]));
-                return ps.x + ps.y;
-            };
+            }
+            const f2 ps = add2(add2(part[0], part[1]), add2(part[2], part[3]));
+            return ps.x + ps.y;
+        };
 
+        int rnd = 0, item_no = 0;
+        int f = walk(rnd);
+        if (f >= 0) ok = take(f, 0);
+        while (f >= 0 && ok) {
+            // the next bundle's flat index: loaded now, used after this bundle's steps
+            int rnd2 = rnd + 1;
+            const int f2raw = item_at(p, rnd2, n_items);
+            m_used = kNegInf;
+            lsum = 0.f;
             for (int s = 0; s < it.nsteps; ++s) {
                 const int gstep = gs + s, b = gstep & 1, slot = vs;
                 const int vphase = vph;
@@ -720,29 +832,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(B.pfull(b));
             }
-            // ---- epilogue: O / l -> O[qid][head][:]
             gs += it.nsteps;
-            if (ok && it.nsteps > 0) {
+            const Item it_cur = it;
+            const int qid_cur = qid, head_cur = head;
+            const float lsum_cur = lsum, m_cur = m_used;
+            // The next bundle takes the other Q buffer before this bundle's epilogue, so its first
+            // S = Q K^T runs while the epilogue reads O.
+            int f2 = f2raw;
+            while (f2 == -2) {
+                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
+                f2 = item_at(p, ++rnd2, n_items);
+            }
+            if (ok && f2 >= 0) ok = take(f2, item_no + 1);
+            // ---- epilogue: O / l -> O[qid][head][:]
+            if (ok && it_cur.nsteps > 0) {
                 const int last = gs - 1;
                 ok = warp_ok(mbar_wait(B.pvdone(last & 1), (last >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
             }
             if (!ok) break;
             tc_fence_after();
             float vsc = 1.f;
-            if constexpr (ES == 1) vsc = p.v_scale[it.h];
-            const float inv = lsum > 0.f ? vsc / lsum : 0.f;
-            const size_t oi = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+            if constexpr (ES == 1) vsc = p.v_scale[it_cur.h];
+            const float inv = lsum_cur > 0.f ? vsc / lsum_cur : 0.f;
+            const size_t oi = ((size_t)(qid_cur >= 0 ? qid_cur : 0) * p.Hq + head_cur) * kD;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
-                if (it.nsteps > 0) {
+                if (it_cur.nsteps > 0) {
                     tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] = 0u;
                 }
-                if (qid >= 0) {
+                if (qid_cur >= 0) {
                     if constexpr (ES == 4) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi + 32 * c);
 #pragma unroll
@@ -762,10 +885,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (qid >= 0 && p.lse != nullptr)
-                p.lse[(size_t)qid * p.Hq + head] =
-                    lsum > 0.f ? (m_used + __log2f(lsum) - G::kPLog2) * 0.69314718055994531f : kNegInf;
+            if (qid_cur >= 0 && p.lse != nullptr)
+                p.lse[(size_t)qid_cur * p.Hq + head_cur] =
+                    lsum_cur > 0.f ? (m_cur + __log2f(lsum_cur) - G::kPLog2) * 0.69314718055994531f : kNegInf;
             tc_fence_before();
+            f = f2;
+            rnd = rnd2;
+            ++item_no;
         }
         tmem_wait_ld();  // a prefetched S load left behind by an aborted walk
     }
@@ -777,7 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kSWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv) { return smem_layout(es, nsk, nsv, Hkv).total; }
+size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g) { return smem_layout(es, nsk, nsv, Hkv, g).total; }
 
 size_t attn_tile_bytes(int es) { return (size_t)kST * kD * es; }
 
