@@ -741,9 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) continue;
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_base + kColS + 128u * b;
-#pragma unroll
-                for (int i = 0; i < kST / 32; ++i)
-                    tmem_ld32(s_addr + 32u * i, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * i));
+                tmem_ld128_wait(s_addr, sv);
                 if (tail) {  // thread r zeroes V token row r of the step if it lies past kv_len
                     const int q = r / T;
                     const int pg = __shfl_sync(0xffffffffu, cpage, e0 - cbase + q);
@@ -757,8 +755,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     make_uint4(0, 0, 0, 0);
                     }
                 }
-                tmem_wait_ld();
-                reg_fence<kST>(sv);
                 const bool warp_live = __any_sync(0xffffffffu, live);
                 // Raw scores of unseen tokens (past the row's causal limit or kv_len inside a page
                 // it selected) become -inf; pages the row did not select get an infinite offset in
@@ -812,9 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t ov[32];
-                        tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
-                        tmem_wait_ld();
-                        reg_fence<32>(ov);
+                        tmem_ld32_wait(tmem + lane_base + kColO + 32u * c, ov);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                         tmem_st_x32(tmem + lane_base + kColO + 32u * c, ov);
@@ -859,8 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
                 if (it_cur.nsteps > 0) {
-                    tmem_ld32(tmem + lane_base + kColO + 32u * c, ov);
-                    tmem_wait_ld();
+                    tmem_ld32_wait(tmem + lane_base + kColO + 32u * c, ov);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] = 0u;
@@ -893,7 +886,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             rnd = rnd2;
             ++item_no;
         }
-        tmem_wait_ld();  // a prefetched S load left behind by an aborted walk
     }
 
     // ---------------------------------------------------------------- teardown
