@@ -502,7 +502,11 @@ __device__ long long lookback(uint64_t* status, int f, long long agg, unsigned* 
 // status: visits, masked row slots, masked query slots, selected page edges.
 // The last window of a KV head adds up its head's windows after its look-back
 // (which implies every earlier window has published, and so written these).
-__global__ void __launch_bounds__(kFusedThreads, 2) grp_fused_kernel(
+// NT threads per CTA: 256 (two CTAs per SM), or 128 (four per SM) when the windows outnumber
+// the CTAs that fit at 256 threads (the greedy of a window of at most 64 queries is one warp's
+// work either way).
+template <int NT>
+__global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
     const int32_t* __restrict__ topk, int Hq, int Hkv, int Nq, int K, int P, int NW, int max_group, int W,
     int nwin, int32_t* __restrict__ group_ptr, int32_t* __restrict__ members, int32_t* __restrict__ n_groups,
     int32_t* __restrict__ union_ptr, int32_t* __restrict__ union_pages, uint64_t* __restrict__ row_mask,
@@ -513,39 +517,48 @@ __global__ void __launch_bounds__(kFusedThreads, 2) grp_fused_kernel(
     uint32_t* rb = sm_f1;  // [W][g][NW] page bitset of every TopK row of the window
     const WinSmem s = carve(sm_f1 + (size_t)W * g * NW, W, NW);
     __shared__ long long s_base;
-    __shared__ int s_red[kFusedWarps];
+    constexpr int kWarps = NT / 32;
+    __shared__ int s_red[kWarps];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     grid_dep_launch();  // the bundle kernel may take free SMs now; it waits for this grid
     const int items = Hkv * nwin;
     for (int f = blockIdx.x; f < items; f += gridDim.x) {
         const int h = f / nwin, w = f % nwin;
         const int w0 = w * W, nw = min(W, Nq - w0);
-        // ---- TopK rows -> row bitsets (-1 is padding, out-of-range IDs are reported and dropped)
+        // ---- TopK rows -> row bitsets (-1 is padding, out-of-range IDs are reported and dropped).
+        // One thread per (query, Q head) row owns that row's bitset words: no two threads update
+        // one word (rows that select the same pages would otherwise collide on shared-memory
+        // atomics), and the row's IDs are read with 16-byte loads when K allows it.
         for (int x = tid; x < nw * g * NW; x += blockDim.x) rb[x] = 0u;
         __syncthreads();
-        const int per_j = nw * K, n_ent = g * per_j;
-        constexpr int kBatch = 8;  // loads in flight per thread before their shared-memory updates
-        for (int x0 = tid; x0 < n_ent; x0 += kBatch * kFusedThreads) {
-            int pgv[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int x = x0 + u * kFusedThreads;
-                pgv[u] = -1;
-                if (x < n_ent) {
-                    const int j = x / per_j, rem = x - j * per_j;
-                    pgv[u] = topk[((size_t)(h * g + j) * Nq + w0) * K + rem];
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int x = x0 + u * kFusedThreads, pg = pgv[u];
-                if (x >= n_ent || pg == -1) continue;
+        for (int row = tid; row < nw * g; row += blockDim.x) {
+            const int i = row / g, j = row - i * g;
+            const int32_t* src = topk + ((size_t)(h * g + j) * Nq + w0 + i) * K;
+            uint32_t* dst = rb + ((size_t)i * g + j) * NW;
+            auto put = [&](int pg) {
+                if (pg == -1) return;
                 if (pg < 0 || pg >= P) {
                     atomicOr(err, QUP_ERR_PAGE_ID);
-                    continue;
+                    return;
                 }
-                const int j = x / per_j, i = (x - j * per_j) / K;
-                atomicOr(&rb[((size_t)i * g + j) * NW + (pg >> 5)], 1u << (pg & 31));
+                dst[pg >> 5] |= 1u << (pg & 31);
+            };
+            if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(topk) & 15) == 0) {
+                const int4* s4 = reinterpret_cast<const int4*>(src);
+                for (int k0 = 0; k0 < K / 4; k0 += 4) {
+                    int4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) v[u] = k0 + u < K / 4 ? s4[k0 + u] : make_int4(-1, -1, -1, -1);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        put(v[u].x);
+                        put(v[u].y);
+                        put(v[u].z);
+                        put(v[u].w);
+                    }
+                }
+            } else {
+                for (int k = 0; k < K; ++k) put(src[k]);
             }
         }
         __syncthreads();
@@ -599,7 +612,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) grp_fused_kernel(
             if (lane == 0) {
                 wcnt[f * 4 + 0] = carry;
                 int rb_total = 0;
-                for (int x = 0; x < kFusedWarps; ++x) rb_total += s_red[x];
+                for (int x = 0; x < kWarps; ++x) rb_total += s_red[x];
                 wcnt[f * 4 + 1] = mr - rb_total;
                 wcnt[f * 4 + 2] = mq;
                 wcnt[f * 4 + 3] = ed;
@@ -614,7 +627,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) grp_fused_kernel(
         if (tid == 0 && !fits) atomicOr(err, QUP_ERR_CAPACITY);
         const int gbase = w * (W / max_group);
         // ---- emit: one warp per group
-        for (int k = warp; k < ng; k += kFusedWarps) {
+        for (int k = warp; k < ng; k += kWarps) {
             const int m0 = s.gstart[k], cnt = s.gstart[k + 1] - m0, R = cnt * g;
             const int gi = gbase + k;
             for (int m = lane; m < cnt; m += 32) members[(size_t)h * Nq + w0 + m0 + m] = w0 + s.order[m0 + m];
@@ -1076,7 +1089,7 @@ size_t fused_bundle_smem(int WB, int NW, int Hkv) {
 // a look-back kernel never exceeds it (every window waited on must be running).
 // (cached per device, kernel and shared-memory size)
 template <typename Kern>
-static int resident_ctas(Kern kernel, size_t smem, int sms) {
+static int resident_ctas(Kern kernel, size_t smem, int sms, int threads = kFusedThreads) {
     struct Entry {
         int dev;
         const void* fn;
@@ -1095,7 +1108,7 @@ static int resident_ctas(Kern kernel, size_t smem, int sms) {
     int per_sm = 0;
     // the kernels want shared memory, not L1: ask for the largest carveout before counting
     cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     if (n < 64) table[n++] = Entry{dev, (const void*)kernel, smem, per_sm};
@@ -1106,11 +1119,20 @@ cudaError_t launch_group_fused(const GroupLaunch& a, uint32_t* gbits, int32_t* w
                                cudaStream_t stream) {
     const int g = a.Hq / a.Hkv;
     const size_t smem = fused_group_smem(a.W, g, a.NW);
-    cudaError_t e = ensure_smem_attr((const void*)grp_fused_kernel, smem);
-    if (e != cudaSuccess) return e;
     const int items = a.Hkv * a.nwin;
-    const int grid = std::min(items, resident_ctas(grp_fused_kernel, smem, a.sms));
-    grp_fused_kernel<<<grid, kFusedThreads, smem, stream>>>(
+    cudaError_t e = ensure_smem_attr((const void*)grp_fused_kernel<256>, smem);
+    if (e != cudaSuccess) return e;
+    int grid = std::min(items, resident_ctas(grp_fused_kernel<256>, smem, a.sms, 256));
+    if (items > grid && a.W <= 64) {  // more windows than CTAs: four smaller CTAs per SM
+        e = ensure_smem_attr((const void*)grp_fused_kernel<128>, smem);
+        if (e != cudaSuccess) return e;
+        grid = std::min(items, resident_ctas(grp_fused_kernel<128>, smem, a.sms, 128));
+        grp_fused_kernel<128><<<grid, 128, smem, stream>>>(
+            a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW, a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
+            a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, a.cap, a.err, 1u << 22);
+        return cudaGetLastError();
+    }
+    grp_fused_kernel<256><<<grid, 256, smem, stream>>>(
         a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW, a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
         a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, a.cap, a.err, 1u << 22);
     return cudaGetLastError();

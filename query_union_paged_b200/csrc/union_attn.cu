@@ -22,7 +22,7 @@
 // its own 32-bit word of every page's row mask straight from the bundle
 // arrays, 32 entries at a time, one batch ahead; it waits for a V tile only
 // on a step whose page reaches kv_len (whose V rows past kv_len it zeroes).
-// bf16 P takes a quarter of its exponentials from a polynomial on the FMA pipe
+// A quarter of the exponentials come from a polynomial on the FMA pipe
 // (exp2_poly2) and the rest from the MUFU unit.
 //
 // Bundle boundaries: the V warp stages each bundle a few steps ahead (header,
@@ -93,7 +93,7 @@ struct Geo {
     static_assert(kPCols <= 128, "P fits in its S buffer");
     // exponentials on the FMA pipe by a polynomial: pairs (j / 2) % 8 < kPolyPairs of every 16
     // columns; the rest go to the MUFU unit
-    static constexpr int kPolyPairs = ES == 2 ? 2 : 0;
+    static constexpr int kPolyPairs = 2;
     static_assert(PPS <= kMaxPPS, "pages per step");
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
