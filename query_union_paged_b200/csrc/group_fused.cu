@@ -162,25 +162,30 @@ __device__ void compact_window(const WinSmem& s, int n, int NW) {
     __syncthreads();
 }
 
-// Greedy (warp 0) with every set of a window of at most 64 items in registers:
-// lane l holds items l and l + 32.  Writes order / gstart / gus / gsum and the
-// group count.  The pick key is (new_pages << 9 | local_id); ties go to the
-// smallest ID.
-template <int NWR>
+// Greedy (warp 0) with every set of a window of at most 32 * CPL items in registers:
+// lane l holds items l, l + 32, ..., l + 32 * (CPL - 1).  Writes order / gstart / gus / gsum
+// and the group count.  The pick key is (new_pages << 9 | local_id); ties go to the smallest
+// ID.
+template <int NWR, int CPL>
 __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) {
     const int lane = threadIdx.x & 31;
-    uint32_t s0[NWR], s1[NWR], U[NWR];
+    uint32_t sc[CPL][NWR], U[NWR];
+    int sz[CPL];
     const int pitch = s.misc[7], NWC = s.misc[1];
+    unsigned taken = 0;
 #pragma unroll
-    for (int x = 0; x < NWR; ++x) {
-        s0[x] = (lane < n && x < NWC) ? s.cs[(size_t)lane * pitch + x] : 0u;
-        s1[x] = (lane + 32 < n && x < NWC) ? s.cs[(size_t)(lane + 32) * pitch + x] : 0u;
+    for (int k = 0; k < CPL; ++k) {
+        const int a = lane + 32 * k;
+#pragma unroll
+        for (int x = 0; x < NWR; ++x) sc[k][x] = (a < n && x < NWC) ? s.cs[(size_t)a * pitch + x] : 0u;
+        sz[k] = a < n ? s.ssize[a] : 0;
+        if (a >= n) taken |= 1u << k;
     }
-    const int sz0 = lane < n ? s.ssize[lane] : 0, sz1 = lane + 32 < n ? s.ssize[lane + 32] : 0;
-    unsigned taken = (lane < n ? 0u : 1u) | (lane + 32 < n ? 0u : 2u);
+    constexpr unsigned kAll = (1u << CPL) - 1u;
     int ng = 0, pos = 0;
     while (true) {
-        const unsigned my = !(taken & 1u) ? (unsigned)lane : (!(taken & 2u) ? (unsigned)lane + 32u : kNone);
+        const unsigned free_k = ~taken & kAll;
+        const unsigned my = free_k ? (unsigned)lane + 32u * (unsigned)(__ffs(free_k) - 1) : kNone;
         const unsigned seed = __reduce_min_sync(0xffffffffu, my);
         if (seed == kNone) break;
         int owner = (int)(seed & 31u), k = (int)(seed >> 5);
@@ -190,18 +195,25 @@ __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) 
             ing |= 1u << k;
         }
 #pragma unroll
-        for (int x = 0; x < NWR; ++x) U[x] = __shfl_sync(0xffffffffu, k ? s1[x] : s0[x], owner);
+        for (int x = 0; x < NWR; ++x) {
+            uint32_t v = sc[0][x];
+#pragma unroll
+            for (int kk = 1; kk < CPL; ++kk)
+                if (k == kk) v = sc[kk][x];
+            U[x] = __shfl_sync(0xffffffffu, v, owner);
+        }
         int cnt = 1;
         while (cnt < max_group) {
-            int c0 = 0, c1 = 0;
+            unsigned bestk = kNone;
 #pragma unroll
-            for (int x = 0; x < NWR; ++x) {
-                c0 += __popc(s0[x] & ~U[x]);
-                c1 += __popc(s1[x] & ~U[x]);
+            for (int kk = 0; kk < CPL; ++kk) {
+                int c = 0;
+#pragma unroll
+                for (int x = 0; x < NWR; ++x) c += __popc(sc[kk][x] & ~U[x]);
+                const unsigned key = (taken >> kk) & 1u ? kNone : (((unsigned)c << 9) | (unsigned)(lane + 32 * kk));
+                bestk = min(bestk, key);
             }
-            const unsigned k0 = (taken & 1u) ? kNone : (((unsigned)c0 << 9) | (unsigned)lane);
-            const unsigned k1 = (taken & 2u) ? kNone : (((unsigned)c1 << 9) | (unsigned)(lane + 32));
-            const unsigned best = __reduce_min_sync(0xffffffffu, min(k0, k1));
+            const unsigned best = __reduce_min_sync(0xffffffffu, bestk);
             if (best == kNone) break;
             const int c = (int)(best & 511u);
             owner = c & 31;
@@ -211,17 +223,31 @@ __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) 
                 ing |= 1u << k;
             }
 #pragma unroll
-            for (int x = 0; x < NWR; ++x) U[x] |= __shfl_sync(0xffffffffu, k ? s1[x] : s0[x], owner);
+            for (int x = 0; x < NWR; ++x) {
+                uint32_t v = sc[0][x];
+#pragma unroll
+                for (int kk = 1; kk < CPL; ++kk)
+                    if (k == kk) v = sc[kk][x];
+                U[x] |= __shfl_sync(0xffffffffu, v, owner);
+            }
             ++cnt;
         }
         int us = 0;
 #pragma unroll
         for (int x = 0; x < NWR; ++x) us += __popc(U[x]);
-        const int sum_s = __reduce_add_sync(0xffffffffu, ((ing & 1u) ? sz0 : 0) + ((ing & 2u) ? sz1 : 0));
-        const unsigned b0 = __ballot_sync(0xffffffffu, ing & 1u), b1 = __ballot_sync(0xffffffffu, ing & 2u);
+        int mysum = 0;
+#pragma unroll
+        for (int kk = 0; kk < CPL; ++kk) mysum += (ing >> kk) & 1u ? sz[kk] : 0;
+        const int sum_s = __reduce_add_sync(0xffffffffu, mysum);
+        // members in ascending ID: item lane + 32 kk ranks after every member of a lower kk
         const unsigned lt = (1u << lane) - 1u;
-        if (ing & 1u) s.order[pos + __popc(b0 & lt)] = lane;
-        if (ing & 2u) s.order[pos + __popc(b0) + __popc(b1 & lt)] = lane + 32;
+        int before = 0;
+#pragma unroll
+        for (int kk = 0; kk < CPL; ++kk) {
+            const unsigned bk = __ballot_sync(0xffffffffu, (ing >> kk) & 1u);
+            if ((ing >> kk) & 1u) s.order[pos + before + __popc(bk & lt)] = lane + 32 * kk;
+            before += __popc(bk);
+        }
         if (lane == 0) {
             s.gstart[ng] = pos;
             s.gus[ng] = us;
@@ -416,7 +442,9 @@ __device__ __noinline__ void greedy_block(const WinSmem& s, int n, int max_group
 // loop several times slower.
 __device__ __noinline__ void run_greedy(const WinSmem& s, int n, int max_group) {
     const int nwc = s.misc[1];
-    if (n > 64 && n <= (int)blockDim.x && blockDim.x <= 256 && nwc <= 8) {  // the whole CTA
+    // windows of 65..128 items with narrow compact sets: one warp, four items per lane
+    const bool reg4 = n > 64 && n <= 128 && nwc <= 16;
+    if (!reg4 && n > 64 && n <= (int)blockDim.x && blockDim.x <= 256 && nwc <= 8) {  // the whole CTA
         if (nwc <= 1) greedy_block<1>(s, n, max_group);
         else if (nwc <= 2) greedy_block<2>(s, n, max_group);
         else if (nwc <= 4) greedy_block<4>(s, n, max_group);
@@ -426,22 +454,29 @@ __device__ __noinline__ void run_greedy(const WinSmem& s, int n, int max_group) 
     }
     if (threadIdx.x < 32) {
         const int NWC = s.misc[1];
-        if (n <= 64 && NWC <= 32) {
+        if (reg4) {
+            if (NWC <= 2) greedy_reg<2, 4>(s, n, max_group);
+            else if (NWC <= 4) greedy_reg<4, 4>(s, n, max_group);
+            else if (NWC <= 6) greedy_reg<6, 4>(s, n, max_group);
+            else if (NWC <= 8) greedy_reg<8, 4>(s, n, max_group);
+            else if (NWC <= 12) greedy_reg<12, 4>(s, n, max_group);
+            else greedy_reg<16, 4>(s, n, max_group);
+        } else if (n <= 64 && NWC <= 32) {
             switch (NWC) {  // exact widths up to 8 words, then 12, 16, 24, 32
                 case 0:
-                case 1: greedy_reg<1>(s, n, max_group); break;
-                case 2: greedy_reg<2>(s, n, max_group); break;
-                case 3: greedy_reg<3>(s, n, max_group); break;
-                case 4: greedy_reg<4>(s, n, max_group); break;
-                case 5: greedy_reg<5>(s, n, max_group); break;
-                case 6: greedy_reg<6>(s, n, max_group); break;
-                case 7: greedy_reg<7>(s, n, max_group); break;
-                case 8: greedy_reg<8>(s, n, max_group); break;
+                case 1: greedy_reg<1, 2>(s, n, max_group); break;
+                case 2: greedy_reg<2, 2>(s, n, max_group); break;
+                case 3: greedy_reg<3, 2>(s, n, max_group); break;
+                case 4: greedy_reg<4, 2>(s, n, max_group); break;
+                case 5: greedy_reg<5, 2>(s, n, max_group); break;
+                case 6: greedy_reg<6, 2>(s, n, max_group); break;
+                case 7: greedy_reg<7, 2>(s, n, max_group); break;
+                case 8: greedy_reg<8, 2>(s, n, max_group); break;
                 default:
-                    if (NWC <= 12) greedy_reg<12>(s, n, max_group);
-                    else if (NWC <= 16) greedy_reg<16>(s, n, max_group);
-                    else if (NWC <= 24) greedy_reg<24>(s, n, max_group);
-                    else greedy_reg<32>(s, n, max_group);
+                    if (NWC <= 12) greedy_reg<12, 2>(s, n, max_group);
+                    else if (NWC <= 16) greedy_reg<16, 2>(s, n, max_group);
+                    else if (NWC <= 24) greedy_reg<24, 2>(s, n, max_group);
+                    else greedy_reg<32, 2>(s, n, max_group);
             }
         } else {
             greedy_smem(s, n, max_group);

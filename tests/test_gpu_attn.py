@@ -28,8 +28,10 @@ def _attn(w, dev, groups, want_lse=False):
     return (O, lse) if want_lse else O
 
 
-def _gpu_groups(w, dev, max_group=8, window=64):
-    return qup.sparse_group(dev["topk"], w.Hq, w.Hkv, w.num_logical_pages, max_group, window)
+def _gpu_groups(w, dev, max_group=8, window=None):
+    """Groups as the bench forms them: the workload's own window unless one is given."""
+    return qup.sparse_group(dev["topk"], w.Hq, w.Hkv, w.num_logical_pages, max_group,
+                            w.window if window is None else window)
 
 
 def _perm_groups(w, seed, max_group=8):

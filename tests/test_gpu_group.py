@@ -39,7 +39,7 @@ def test_random_small_bitexact(seed):
 
 
 @pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c", "5"])
-@pytest.mark.parametrize("window", [64, 8, 256])
+@pytest.mark.parametrize("window", [64, 8, 128, 256])
 def test_workload_bitexact(cfg, window):
     w = W.make(cfg)
     got = _run(w.topk, w.Hq, w.Hkv, w.num_logical_pages, 8, window)
