@@ -397,8 +397,9 @@ int oracle_group(const int32_t* topk, int Hq, int Hkv, int Nq, int K, int P,
  * Bundles (an execution-level packing with no counterpart on the pages): per
  * KV head, the groups in order are cut into windows of wb groups; inside a
  * window a bundle is seeded with the first unbundled group and grown, up to
- * `slots` groups, by the group whose union adds the fewest pages to the
- * bundle union (ties: smallest index).  Groups of a bundle are listed
+ * `slots` groups, by the group with the smallest  new - 2 * shared , new
+ * being the pages its union adds to the bundle union and shared the pages
+ * of its union already in it (ties: smallest index).  Groups of a bundle are listed
  * ascending (slot order).  Row of slot j, member rank m, head offset jj:
  * j*rs + m*g + jj.  The 128-bit mask of a bundle page has the group's row
  * mask of that page at bit offset j*rs.
@@ -458,7 +459,9 @@ int oracle_bundle(int Hq, int Hkv, int Nq, int max_group, int bundle_window,
                     for (int c = seed + 1; c < nw; ++c) {
                         if (taken[c]) continue;
                         iset sc = { (int32_t*)union_pages + up[w0 + c], up[w0 + c + 1] - up[w0 + c] };
-                        int nc = set_minus_count(&sc, &u);
+                        /* new pages counted against pages already shared with the bundle union:
+                         * new - 2 * shared = 3 * new - 2 * |S(c)| */
+                        int nc = 3 * set_minus_count(&sc, &u) - 2 * sc.n;
                         if (best < 0 || nc < bestc) { best = c; bestc = nc; }
                     }
                     if (best < 0) break;

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restr
                                                           int32_t* __restrict__ ws_usize,
                                                           int32_t* __restrict__ ws_wtot,
                                                           int32_t* __restrict__ ws_wcnt,
-                                                          int64_t* __restrict__ out_count) {
+                                                          int64_t* __restrict__ out_count, int bundle) {
     extern __shared__ uint32_t sm_gr[];
     const int NWp = NW | 1;  // odd row pitch: lanes reading different queries hit different banks
     uint32_t* S = sm_gr;
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(128) grp_greedy_kernel(const uint32_t* __restr
                 const uint32_t* sa = S + a * NWp;
                 int nc = 0;
                 for (int wd = 0; wd < NW; ++wd) nc += __popc(sa[wd] & ~U[wd]);
-                key = min(key, ((unsigned)nc << 9) | (unsigned)a);
+                key = min(key, (pick_value(nc, ssize[a], bundle != 0) << 9) | (unsigned)a);
             }
             const unsigned best = __reduce_min_sync(0xffffffffu, key);
             if (best == 0xffffffffu) break;
@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(128) grp_greedy_reg_kernel(const uint32_t* __r
                                                               int32_t* __restrict__ ws_usize,
                                                               int32_t* __restrict__ ws_wtot,
                                                               int32_t* __restrict__ ws_wcnt,
-                                                              int64_t* __restrict__ out_count) {
+                                                              int64_t* __restrict__ out_count, int bundle) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int item = blockIdx.x * 4 + warp;
     if (item >= nwin * Hkv) return;
@@ -601,13 +601,13 @@ __global__ void __launch_bounds__(128) grp_greedy_reg_kernel(const uint32_t* __r
                 int nc = 0;
 #pragma unroll
                 for (int x = 0; x < NWR; ++x) nc += __popc(s0[x] & ~U[x]);
-                key = ((unsigned)nc << 9) | (unsigned)lane;
+                key = (pick_value(nc, sz0, bundle != 0) << 9) | (unsigned)lane;
             }
             if (!(taken & 2u)) {
                 int nc = 0;
 #pragma unroll
                 for (int x = 0; x < NWR; ++x) nc += __popc(s1[x] & ~U[x]);
-                key = min(key, ((unsigned)nc << 9) | (unsigned)(lane + 32));
+                key = min(key, (pick_value(nc, sz1, bundle != 0) << 9) | (unsigned)(lane + 32));
             }
             const unsigned best = __reduce_min_sync(0xffffffffu, key);
             if (best == kNone) break;
@@ -661,13 +661,13 @@ __global__ void __launch_bounds__(128) grp_greedy_reg_kernel(const uint32_t* __r
 static cudaError_t launch_greedy(const uint32_t* sets, int sets_per_item, int Hkv, int Nq, const int32_t* n_items_dev,
                                  int NW, int max_group, int W, int nwin, int32_t* group_ptr, int32_t* members,
                                  int32_t* n_groups, int32_t* ws_usize, int32_t* ws_wtot, int32_t* ws_wcnt,
-                                 int64_t* out_count, cudaStream_t stream) {
+                                 int64_t* out_count, bool bundle, cudaStream_t stream) {
     if (W <= 64 && NW <= 32) {
         const int items = nwin * Hkv, grid = (items + 3) / 4;
 #define QUP_GREEDY_REG(N)                                                                                        \
     grp_greedy_reg_kernel<N><<<grid, 128, 0, stream>>>(sets, sets_per_item, Hkv, Nq, n_items_dev, NW, max_group, \
                                                        W, nwin, group_ptr, members, n_groups, ws_usize, ws_wtot, \
-                                                       ws_wcnt, out_count)
+                                                       ws_wcnt, out_count, bundle ? 1 : 0)
         if (NW <= 4) QUP_GREEDY_REG(4);
         else if (NW <= 8) QUP_GREEDY_REG(8);
         else if (NW <= 12) QUP_GREEDY_REG(12);
@@ -682,7 +682,7 @@ static cudaError_t launch_greedy(const uint32_t* sets, int sets_per_item, int Hk
     if (e != cudaSuccess) return e;
     grp_greedy_kernel<<<dim3(nwin, Hkv), 128, sm, stream>>>(sets, sets_per_item, Hkv, Nq, n_items_dev, NW, max_group,
                                                              W, nwin, group_ptr, members, n_groups, ws_usize, ws_wtot,
-                                                             ws_wcnt, out_count);
+                                                             ws_wcnt, out_count, bundle ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -705,7 +705,7 @@ cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
                                                        a.rowbits, a.counters, a.err);
     const dim3 grid2(a.nwin, a.Hkv);
     if ((e = launch_greedy(a.rowbits, a.Hq / a.Hkv, a.Hkv, a.Nq, nullptr, a.NW, a.max_group, a.W, a.nwin,
-                           a.group_ptr, a.members, a.n_groups, a.ws_usize, a.ws_wtot, a.ws_wcnt, nullptr,
+                           a.group_ptr, a.members, a.n_groups, a.ws_usize, a.ws_wtot, a.ws_wcnt, nullptr, false,
                            stream)) != cudaSuccess)
         return e;
     grp_emit_kernel<<<grid2, 256, sm1, stream>>>(a.rowbits, a.Hq, a.Hkv, a.Nq, a.NW, a.max_group, a.W,
@@ -834,7 +834,7 @@ cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream) {
                                                   a.gbits, a.bcounters, a.err);
     const dim3 grid2(a.nwin, a.Hkv);
     if ((e = launch_greedy(a.gbits, 1, a.Hkv, a.Nq, a.n_groups, a.NW, a.slots, a.WB, a.nwin, a.bundle_ptr,
-                           a.bundle_groups, a.n_bundles, a.ws_usize, a.ws_wtot, a.ws_wcnt, a.bcounters, stream)) !=
+                           a.bundle_groups, a.n_bundles, a.ws_usize, a.ws_wtot, a.ws_wcnt, a.bcounters, true, stream)) !=
         cudaSuccess)
         return e;
     bnd_emit_kernel<<<grid2, 256, smw, stream>>>(a.gbits, a.Hkv, a.Nq, a.NW, a.g, a.RS, a.slots, a.WB, a.nwin,

@@ -164,10 +164,11 @@ __device__ void compact_window(const WinSmem& s, int n, int NW) {
 
 // Greedy (warp 0) with every set of a window of at most 32 * CPL items in registers:
 // lane l holds items l, l + 32, ..., l + 32 * (CPL - 1).  Writes order / gstart / gus / gsum
-// and the group count.  The pick key is (new_pages << 9 | local_id); ties go to the smallest
-// ID.
-template <int NWR, int CPL>
+// and the group count.  The pick key is (value << 9 | local_id), value = pick_value (the new
+// page count for groups); ties go to the smallest ID.
+template <int NWR, int CPL, bool BUNDLE>
 __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) {
+    constexpr bool bundle = BUNDLE;
     const int lane = threadIdx.x & 31;
     uint32_t sc[CPL][NWR], U[NWR];
     int sz[CPL];
@@ -210,7 +211,8 @@ __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) 
                 int c = 0;
 #pragma unroll
                 for (int x = 0; x < NWR; ++x) c += __popc(sc[kk][x] & ~U[x]);
-                const unsigned key = (taken >> kk) & 1u ? kNone : (((unsigned)c << 9) | (unsigned)(lane + 32 * kk));
+                const unsigned key =
+                    (taken >> kk) & 1u ? kNone : ((pick_value(c, sz[kk], bundle) << 9) | (unsigned)(lane + 32 * kk));
                 bestk = min(bestk, key);
             }
             const unsigned best = __reduce_min_sync(0xffffffffu, bestk);
@@ -264,7 +266,7 @@ __device__ __noinline__ void greedy_reg(const WinSmem& s, int n, int max_group) 
 
 // Greedy (warp 0) for any window (n <= 256) and any compact width: sets and
 // the running union stay in shared memory.
-__device__ __noinline__ void greedy_smem(const WinSmem& s, int n, int max_group) {
+__device__ __noinline__ void greedy_smem(const WinSmem& s, int n, int max_group, bool bundle) {
     const int lane = threadIdx.x & 31;
     const int NWC = s.misc[1], pitch = s.misc[7];
     const int CPL = (n + 31) >> 5;
@@ -294,7 +296,7 @@ __device__ __noinline__ void greedy_smem(const WinSmem& s, int n, int max_group)
                 const uint32_t* sa = s.cs + (size_t)a * pitch;
                 int nc = 0;
                 for (int wd = 0; wd < NWC; ++wd) nc += __popc(sa[wd] & ~s.Ug[wd]);
-                key = min(key, ((unsigned)nc << 9) | (unsigned)a);
+                key = min(key, (pick_value(nc, s.ssize[a], bundle) << 9) | (unsigned)a);
             }
             const unsigned best = __reduce_min_sync(0xffffffffu, key);
             if (best == kNone) break;
@@ -339,9 +341,10 @@ __device__ __noinline__ void greedy_smem(const WinSmem& s, int n, int max_group)
 // scores its item, each warp's best lane posts its key and set to shared memory
 // (double-buffered by pick parity), one barrier, and every thread reduces the
 // posted keys and ORs the winner's set into its copy of the running union.
-// Same keys (new_pages << 9 | local_id) and so the same picks as greedy_reg.
-template <int NWR>
+// Same keys (pick_value << 9 | local_id) and so the same picks as greedy_reg.
+template <int NWR, bool BUNDLE>
 __device__ __noinline__ void greedy_block(const WinSmem& s, int n, int max_group) {
+    constexpr bool bundle = BUNDLE;
     uint32_t* post = s.post;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarp = blockDim.x >> 5;
@@ -392,7 +395,8 @@ __device__ __noinline__ void greedy_block(const WinSmem& s, int n, int max_group
             int nc = 0;
 #pragma unroll
             for (int x = 0; x < NWR; ++x) nc += __popc(sv[x] & ~U[x]);
-            const unsigned best = block_pick(taken ? kNone : (((unsigned)nc << 9) | (unsigned)tid), win);
+            const unsigned best =
+                block_pick(taken ? kNone : ((pick_value(nc, sz, bundle) << 9) | (unsigned)tid), win);
             if (best == kNone) break;
             if ((int)(best & 511u) == tid) {
                 taken = true;
@@ -440,49 +444,58 @@ __device__ __noinline__ void greedy_block(const WinSmem& s, int n, int max_group
 // sets), the whole CTA for larger windows of narrow sets; the CTA waits.  The greedy
 // functions stay out of line: inlined into the kernel body they compiled to a
 // loop several times slower.
-__device__ __noinline__ void run_greedy(const WinSmem& s, int n, int max_group) {
+template <bool BUNDLE>
+__device__ __noinline__ void run_greedy_t(const WinSmem& s, int n, int max_group) {
     const int nwc = s.misc[1];
     // windows of 65..128 items with narrow compact sets: one warp, four items per lane
     const bool reg4 = n > 64 && n <= 128 && nwc <= 16;
     if (!reg4 && n > 64 && n <= (int)blockDim.x && blockDim.x <= 256 && nwc <= 8) {  // the whole CTA
-        if (nwc <= 1) greedy_block<1>(s, n, max_group);
-        else if (nwc <= 2) greedy_block<2>(s, n, max_group);
-        else if (nwc <= 4) greedy_block<4>(s, n, max_group);
-        else greedy_block<8>(s, n, max_group);
+        if (nwc <= 1) greedy_block<1, BUNDLE>(s, n, max_group);
+        else if (nwc <= 2) greedy_block<2, BUNDLE>(s, n, max_group);
+        else if (nwc <= 4) greedy_block<4, BUNDLE>(s, n, max_group);
+        else greedy_block<8, BUNDLE>(s, n, max_group);
         __syncthreads();
         return;
     }
     if (threadIdx.x < 32) {
         const int NWC = s.misc[1];
         if (reg4) {
-            if (NWC <= 2) greedy_reg<2, 4>(s, n, max_group);
-            else if (NWC <= 4) greedy_reg<4, 4>(s, n, max_group);
-            else if (NWC <= 6) greedy_reg<6, 4>(s, n, max_group);
-            else if (NWC <= 8) greedy_reg<8, 4>(s, n, max_group);
-            else if (NWC <= 12) greedy_reg<12, 4>(s, n, max_group);
-            else greedy_reg<16, 4>(s, n, max_group);
+            if (NWC <= 2) greedy_reg<2, 4, BUNDLE>(s, n, max_group);
+            else if (NWC <= 4) greedy_reg<4, 4, BUNDLE>(s, n, max_group);
+            else if (NWC <= 6) greedy_reg<6, 4, BUNDLE>(s, n, max_group);
+            else if (NWC <= 8) greedy_reg<8, 4, BUNDLE>(s, n, max_group);
+            else if (NWC <= 12) greedy_reg<12, 4, BUNDLE>(s, n, max_group);
+            else greedy_reg<16, 4, BUNDLE>(s, n, max_group);
         } else if (n <= 64 && NWC <= 32) {
             switch (NWC) {  // exact widths up to 8 words, then 12, 16, 24, 32
                 case 0:
-                case 1: greedy_reg<1, 2>(s, n, max_group); break;
-                case 2: greedy_reg<2, 2>(s, n, max_group); break;
-                case 3: greedy_reg<3, 2>(s, n, max_group); break;
-                case 4: greedy_reg<4, 2>(s, n, max_group); break;
-                case 5: greedy_reg<5, 2>(s, n, max_group); break;
-                case 6: greedy_reg<6, 2>(s, n, max_group); break;
-                case 7: greedy_reg<7, 2>(s, n, max_group); break;
-                case 8: greedy_reg<8, 2>(s, n, max_group); break;
+                case 1: greedy_reg<1, 2, BUNDLE>(s, n, max_group); break;
+                case 2: greedy_reg<2, 2, BUNDLE>(s, n, max_group); break;
+                case 3: greedy_reg<3, 2, BUNDLE>(s, n, max_group); break;
+                case 4: greedy_reg<4, 2, BUNDLE>(s, n, max_group); break;
+                case 5: greedy_reg<5, 2, BUNDLE>(s, n, max_group); break;
+                case 6: greedy_reg<6, 2, BUNDLE>(s, n, max_group); break;
+                case 7: greedy_reg<7, 2, BUNDLE>(s, n, max_group); break;
+                case 8: greedy_reg<8, 2, BUNDLE>(s, n, max_group); break;
                 default:
-                    if (NWC <= 12) greedy_reg<12, 2>(s, n, max_group);
-                    else if (NWC <= 16) greedy_reg<16, 2>(s, n, max_group);
-                    else if (NWC <= 24) greedy_reg<24, 2>(s, n, max_group);
-                    else greedy_reg<32, 2>(s, n, max_group);
+                    if (NWC <= 12) greedy_reg<12, 2, BUNDLE>(s, n, max_group);
+                    else if (NWC <= 16) greedy_reg<16, 2, BUNDLE>(s, n, max_group);
+                    else if (NWC <= 24) greedy_reg<24, 2, BUNDLE>(s, n, max_group);
+                    else greedy_reg<32, 2, BUNDLE>(s, n, max_group);
             }
         } else {
-            greedy_smem(s, n, max_group);
+            greedy_smem(s, n, max_group, BUNDLE);
         }
     }
     __syncthreads();
+}
+
+// The greedy on the compact sets of a window: groups (bundle = false) or bundles (true).
+__device__ __forceinline__ void run_greedy(const WinSmem& s, int n, int max_group, bool bundle) {
+    if (bundle)
+        run_greedy_t<true>(s, n, max_group);
+    else
+        run_greedy_t<false>(s, n, max_group);
 }
 
 // Decoupled look-back (warp 0): publishes `agg` for item f and returns the sum
@@ -613,7 +626,7 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
         if (lane == 0) s_red[warp] = rbits;
         __syncthreads();
         compact_window(s, nw, NW);
-        run_greedy(s, nw, max_group);
+        run_greedy(s, nw, max_group, false);
         const int ng = s.misc[0];
         // ---- offsets: group prefix inside the window, window prefix by look-back
         if (warp == 0) {
@@ -942,7 +955,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) bnd_fused_kernel(
         int ng = 0;
         if (nw > 0) {
             compact_window(s, nw, NW);
-            run_greedy(s, nw, slots);
+            run_greedy(s, nw, slots, true);
             ng = s.misc[0];
         }
         if (warp == 0) {

@@ -71,6 +71,16 @@ cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUten
 // the softmax's polynomial 2^x over n floats (test hook)
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 
+// Pick value of the bundling greedy (groups packed into bundles; execution-level, no counterpart
+// on the pages): new pages counted against the pages a candidate already shares with the bundle
+// union, new - 2 * shared = 3 * new - 2 * |S(c)|, biased non-negative (exact for windows whose
+// universe is below 2^20 pages).  The pick key is (value << 9 | local_id), as for groups, whose
+// value is the new page count alone.
+constexpr int kBundleKeyBias = 1 << 21;
+__host__ __device__ inline unsigned pick_value(int new_pages, int set_size, bool bundle) {
+    return bundle ? (unsigned)(3 * new_pages - 2 * set_size + kBundleKeyBias) : (unsigned)new_pages;
+}
+
 struct GroupLaunch {
     const int32_t* topk;
     int Hq, Hkv, Nq, K, P, NW, max_group, W, nwin;

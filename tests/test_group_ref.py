@@ -192,7 +192,8 @@ def test_block_union_workload_groups_align_with_query_blocks():
 # ----------------------------------------------------------- bundles
 
 def py_bundle(out, Hq, Hkv, Nq, max_group, wb=64):
-    """The bundling rule written with Python sets: greedy over group unions."""
+    """The bundling rule written with Python sets: greedy over group unions (pick key: new pages
+    minus twice the shared pages, ties to the smallest index)."""
     g = Hq // Hkv
     rs = 1
     while rs < max_group * g:
@@ -209,7 +210,8 @@ def py_bundle(out, Hq, Hkv, Nq, max_group, wb=64):
                 seed = left.pop(0)
                 U, b = set(groups[seed][1]), [seed]
                 while len(b) < slots and left:
-                    c = min(left, key=lambda q: (len(set(groups[q][1]) - U), q))
+                    # fewest new pages, counted against the pages already shared with the bundle
+                    c = min(left, key=lambda q: (len(set(groups[q][1]) - U) - 2 * len(set(groups[q][1]) & U), q))
                     left.remove(c)
                     b.append(c)
                     U |= set(groups[c][1])
