@@ -67,6 +67,24 @@ def unique_kv_pages(w) -> int:
     return n
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(total_ms: float, world: int, device) -> float:
+    """The slowest rank's device time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return total_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flop_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processed its own chunk in the slowest rank's time."""
+    return world * flop_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ environment helpers
 
 def measured_peaks():
@@ -275,11 +293,7 @@ def main():
     t_group = [evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)]
     t_attn = [evs[k][1].elapsed_time(evs[k][2]) for k in range(args.steps)]
     t_step = [a + b for a, b in zip(t_group, t_attn)]
-    total_ms = sum(t_step)
-    if world > 1:
-        tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(t_step), world, "cuda")
 
     # ---- work accounting
     E = int(selected_edges_per_row(w).sum())
@@ -289,7 +303,7 @@ def main():
     ctr = groups.counters.cpu().numpy().sum(axis=0)
     bctr = groups.bcounters.cpu().numpy().sum(axis=0)
     ms_per_step = total_ms / args.steps
-    value = world * flop / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flop, world, ms_per_step)
     attn_ms = statistics.mean(t_attn)
     peaks = measured_peaks()
     # contraction dtype: bf16 MMAs for bf16 KV, tf32 for fp32, fp8 for E4M3 (nominal 2x bf16)
