@@ -73,9 +73,11 @@ extern "C" {
  *
  * Bundles (the attention kernel's work items; no counterpart on the pages,
  * which share a page between the two CTAs of one Union8 group instead):
- * the groups of one KV head are packed, by the same greedy page-affinity
- * rule applied to group unions inside windows of bundle_window groups, into
- * bundles of up to 128 / rows_per_group groups.  A bundle's query rows are
+ * the groups of one KV head are packed, inside windows of bundle_window
+ * groups, into bundles of up to 128 / rows_per_group groups by a greedy on
+ * group unions: seeded with the first unbundled group, grown by the group
+ * with the smallest (new pages - 2 * pages already shared with the bundle
+ * union), ties to the smallest index.  A bundle's query rows are
  * laid out slot by slot: row = slot*rows_per_group + rank*g + j, with
  * rows_per_group = max_group*g rounded up to a power of two (<= 32).
  *   bundle_ptr[h*(Nq+1)+b] .. [+b+1]  indexes bundle_groups[h*Nq + ...]

@@ -10,7 +10,9 @@
 //      smallest unassigned query, add the candidate with the fewest pages
 //      outside the union (ties to the smallest ID) until max_group members or
 //      the window is exhausted.  The argmin is one warp reduction of the
-//      packed key (new_pages << 9 | local_id).
+//      packed key (value << 9 | local_id), value = pick_value: the new page
+//      count for groups; for bundles (the same kernels run on group unions)
+//      new - 2 * shared pages.
 //   3. emit:    one CTA per (window, KV head) sums the union sizes of all
 //      earlier windows for its absolute offset, then one warp per group
 //      writes the sorted union pages and per-page row masks from the bitsets.

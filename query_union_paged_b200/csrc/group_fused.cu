@@ -5,15 +5,18 @@
 // Same rule and same outputs as the multi-kernel path in group.cu, with the
 // intermediate state kept in shared memory:
 //   grp_fused_kernel  one CTA per (query window, KV head): the window's TopK
-//                     rows -> per-row page bitsets -> per-query sets (OR over
-//                     the g heads of the KV group) -> greedy groups -> union
-//                     pages and row masks of every group, written at offsets
-//                     found by a look-back over the earlier windows.
+//                     rows -> per-row page bitsets (one thread per row) ->
+//                     per-query sets (OR over the g heads of the KV group) ->
+//                     greedy groups (pick: fewest new pages) -> union pages and
+//                     row masks of every group, written at offsets found by a
+//                     look-back over the earlier windows.  256 threads, or 128
+//                     (four CTAs per SM) when the windows outnumber the CTAs.
 //   bnd_fused_kernel  one CTA per (window of groups, KV head): the groups'
 //                     union bitsets -> greedy bundles of up to `slots` groups
-//                     -> bundle unions, 128-bit row masks and the row ->
-//                     query table; the CTA that finishes last also sorts the
-//                     bundles by union size for the attention kernel.
+//                     (pick: smallest new - 2 * shared pages, pick_value) ->
+//                     bundle unions, 128-bit row masks and the row -> query
+//                     table; the CTA that finishes last also sorts the bundles
+//                     by union size for the attention kernel.
 //
 // The greedy runs on sets compacted to the window's own pages: page p of the
 // window universe becomes bit rank(p), so |S(c) \ U| is computed over a few
