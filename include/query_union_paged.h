@@ -114,7 +114,7 @@ typedef struct {
     int64_t* bcounters;    /* [Hkv][2] */
     int32_t* bundle_order; /* [Hkv*Nq] */
     int32_t rows_per_group;/* set by qup_sparse_group / qup_build_bundles */
-    int32_t bundle_window; /* groups per bundling window (0: default 64) */
+    int32_t bundle_window; /* groups per bundling window: 0 (default 64) .. 256, else QUP_ERR_ARG */
 } qup_groups;
 
 /*

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -27,8 +28,8 @@ struct DevState {
 
 std::mutex g_mu;
 DevState g_dev[kMaxDevices];
-int g_wait_limit_ms = 0;   // 0: default
-int g_skip_stage = -1;
+std::atomic<int> g_wait_limit_ms{0};  // 0: default
+std::atomic<int> g_skip_stage{-1};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -235,6 +236,7 @@ int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
     if (!g || !g->n_groups || !g->group_ptr || !g->members || !g->union_ptr || !g->union_pages || !g->row_mask ||
         !bundle_fields_ok(g))
         return QUP_ERR_ARG;
+    if (g->bundle_window < 0 || g->bundle_window > 256) return QUP_ERR_ARG;
     if (!ws || ws_bytes < need) return QUP_ERR_CAPACITY;
     DevState* ds = nullptr;
     if ((rc = device_state(&ds))) return rc;
@@ -250,6 +252,7 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
     if (!out || !out->n_groups || !out->group_ptr || !out->members || !out->union_ptr || !out->union_pages ||
         !out->row_mask || !out->counters || !bundle_fields_ok(out))
         return QUP_ERR_ARG;
+    if (out->bundle_window < 0 || out->bundle_window > 256) return QUP_ERR_ARG;
     if ((Nq > 0 && Ksel > 0 && !topk) || (!ws && need > 0)) return QUP_ERR_ARG;
     if (ws_bytes < need) return QUP_ERR_CAPACITY;
     if (out->cap_union < cap) return QUP_ERR_CAPACITY;
@@ -398,8 +401,9 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.nsk = nsk;
     p.nsv = nsv;
-    p.wait_limit_ns = (unsigned long long)(g_wait_limit_ms > 0 ? g_wait_limit_ms : 2000) * 1000000ull;
-    p.dbg_skip_stage = g_skip_stage;
+    const int wait_ms = g_wait_limit_ms.load();
+    p.wait_limit_ns = (unsigned long long)(wait_ms > 0 ? wait_ms : 2000) * 1000000ull;
+    p.dbg_skip_stage = g_skip_stage.load();
     const cudaError_t e =
         qup::launch_union_attn(es, T, tm[0], tm[1], p, ds->sms, smem, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;

@@ -64,3 +64,16 @@ def test_generator_is_deterministic():
     w = W.gqa_chunk_bf16()
     assert w.topk.shape == (32, 2048, 16) and w.kv_len == 16384 + 2048
     assert np.all(w.topk[0] == w.topk[3]) and not np.all(w.topk[0] == w.topk[4])
+
+
+def test_bundle_window_out_of_range_is_rejected_before_any_device_work(lib):
+    # every buffer pointer is non-null but fake: the argument checks run before the device is touched
+    fake = [ctypes.c_void_p(0x1000 + 0x100 * i).value for i in range(len(qup._GROUP_KEYS) + len(qup._BUNDLE_KEYS))]
+    for bw, want in ((300, qup.ERR["ARG"]), (-1, qup.ERR["ARG"])):
+        cs = qup._Groups(*fake[:len(qup._GROUP_KEYS)], 1 << 20, *fake[len(qup._GROUP_KEYS):], 0, bw)
+        qup.load()
+        rc = qup._lib.qup_sparse_group(ctypes.c_void_p(0x2000), 32, 8, 2048, 16, 288, 8, 64, ctypes.byref(cs),
+                                       ctypes.c_void_p(0x3000), 1 << 30, None)
+        assert rc == want, (bw, rc)
+        rc = qup._lib.qup_build_bundles(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30, None)
+        assert rc == want, (bw, rc)
