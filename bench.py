@@ -42,9 +42,9 @@ CONFIG_DEFAULT = "2"
 
 # ------------------------------------------------------------------ workload accounting
 
-def selected_edges_per_row(w) -> np.ndarray:
+def selected_edges_per_row(w, topk=None) -> np.ndarray:
     """|A_i| for every (Q head, query): tokens of the row's distinct pages with t < kv_len, t <= q_pos."""
-    topk = w.topk
+    topk = w.topk if topk is None else topk
     Hq, Nq, K = topk.shape
     E = np.zeros((Hq, Nq), np.int64)
     srt = np.sort(topk, axis=2)
@@ -65,6 +65,23 @@ def unique_kv_pages(w) -> int:
         rows = w.topk[h * g:(h + 1) * g].reshape(-1)
         n += np.unique(rows[rows >= 0]).size
     return n
+
+
+def union_topk(w, groups) -> np.ndarray:
+    """[Hq][Nq][Kmax] TopK rows holding each query's group union (host copy of the groups)."""
+    n_groups = groups.n_groups.cpu().numpy()
+    gp_all, up_all = groups.group_ptr.cpu().numpy(), groups.union_ptr.cpu().numpy()
+    members, pages = groups.members.cpu().numpy(), groups.union_pages.cpu().numpy()
+    g = w.Hq // w.Hkv
+    kmax = max(1, max(int(np.diff(up_all[h, :n_groups[h] + 1]).max(initial=0)) for h in range(w.Hkv)))
+    out = np.full((w.Hq, w.Nq, kmax), -1, np.int32)
+    for h in range(w.Hkv):
+        gp, up = gp_all[h], up_all[h]
+        for k in range(int(n_groups[h])):
+            u = pages[up[k]:up[k + 1]]
+            for m in members[h, gp[k]:gp[k + 1]]:
+                out[h * g:(h + 1) * g, m, :u.size] = u
+    return out
 
 
 # ------------------------------------------------------------------ ranks
@@ -217,6 +234,8 @@ def main():
     ap.add_argument("--window", type=int, default=None)
     ap.add_argument("--max-group", type=int, default=None)
     ap.add_argument("--bundle-window", type=int, default=None)
+    ap.add_argument("--union-support", action="store_true",
+                    help="every row of a group attends to its group's whole union (qup_union_support)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -259,6 +278,8 @@ def main():
         if ev is not None:
             ev[0].record(stream)
         qup.sparse_group(topk, w.Hq, w.Hkv, w.num_logical_pages, max_group, window, out=groups)
+        if args.union_support:
+            qup.union_support(groups, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, max_group)
         if ev is not None:
             ev[1].record(stream)
         qup.sparse_prefill_attn(dev["Q"], dev["K"], dev["V"], page_table, groups, q_pos, w.kv_len,
@@ -295,8 +316,8 @@ def main():
     t_step = [a + b for a, b in zip(t_group, t_attn)]
     total_ms = max_over_ranks(sum(t_step), world, "cuda")
 
-    # ---- work accounting
-    E = int(selected_edges_per_row(w).sum())
+    # ---- work accounting (with union support, a row's edges are those of its group's union)
+    E = int(selected_edges_per_row(w, union_topk(w, groups) if args.union_support else None).sum())
     flop = 4.0 * w.d * E
     n_uniq = unique_kv_pages(w)
     uniq_bytes = n_uniq * w.kv_page_bytes()
@@ -312,7 +333,7 @@ def main():
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
 
     # ---- end to end through host buffers (pinned), copies inside the timed region
-    e2e = run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O)
+    e2e = run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O, flop)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -322,7 +343,8 @@ def main():
         "data": "synthetic (seeded; shapes of the pages' prefill chunks)",
         "config": {"workload": w.name, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "d": w.d,
                    "page_tokens": w.T, "topk": w.K, "kv_len": w.kv_len, "max_group": max_group,
-                   "window": window, "bundle_window": bundle_window, "l2": "flushed before every timed step (2x L2 write)",
+                   "window": window, "bundle_window": bundle_window,
+                   "support": "group union" if args.union_support else "own TopK row", "l2": "flushed before every timed step (2x L2 write)",
                    "parallelism": f"replicas x{world} (independent chunks)"},
         "us_per_call": {"group": round(statistics.median(t_group) * 1e3, 2),
                         "attn": round(statistics.median(t_attn) * 1e3, 2),
@@ -357,7 +379,7 @@ def main():
         dist.destroy_process_group()
 
 
-def run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O_ref):
+def run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O_ref, flop):
     """Same metric through the public calls with host (pinned) inputs and output.
 
     Every step copies its inputs (Q, TopK, q_pos, page table) from pinned host memory and reads
@@ -392,6 +414,8 @@ def run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O_ref)
         di = d_in[b]
         qup.sparse_group(di["topk"], w.Hq, w.Hkv, w.num_logical_pages, max_group, window, out=groups,
                          stream=s_comp)
+        if args.union_support:
+            qup.union_support(groups, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, max_group, stream=s_comp)
         qup.sparse_prefill_attn(di["Q"], dev["K"], dev["V"], di["page_table"], groups, di["q_pos"],
                                 w.kv_len, k_scale=ks, v_scale=vs, topk=di["topk"], out=O[b],
                                 num_logical_pages=w.num_logical_pages, stream=s_comp)
@@ -419,7 +443,6 @@ def run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O_ref)
     # the output read back through host memory is the device path's output
     if not torch.equal(O_host[(n - 1) & 1], O_ref.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
-    flop = 4.0 * w.d * float(selected_edges_per_row(w).sum())
     return {"value": round(flop / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "pipelined": "copies in, compute and read-back on three streams, two buffers each"}

@@ -176,6 +176,20 @@ int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Union as support (CompactAttention: Accelerating Chunked Prefill with
+ * Block-Union KV Selection, where each query block attends to the whole union
+ * table of its KV group): rewrites the row masks of the groups in `g` so that
+ * every row of a group sees every page of the group's union, then rebuilds the
+ * bundles (as qup_build_bundles).  qup_sparse_prefill_attn on the result
+ * computes attention over the group unions instead of each query's own TopK
+ * rows.  The group counters keep describing the original selection.
+ *   g, ws, sizes: as for qup_build_bundles; groups of more than 64 rows or
+ *   union offsets past cap_union raise QUP_ERR_GROUP on the device.
+ */
+int qup_union_support(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * ID-aware union attention (Abstract; Figure 1; Figure 3).  One persistent
  * kernel: per bundle (up to 128 query rows of one KV head) it gathers the
  * rows of Q by original ID into shared memory, streams each page of the

@@ -19,7 +19,7 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host",
+__all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host", "union_support",
            "get_error", "set_debug", "load",
            "QupError", "F32", "BF16", "E4M3", "ERR"]
 
@@ -70,8 +70,9 @@ def load():
     lib.qup_set_debug.argtypes = [I, I]
     lib.qup_num_sms.argtypes = []
     lib.qup_exp2_poly.argtypes = [P, P, I, P]
+    lib.qup_union_support.argtypes = [ctypes.POINTER(_Groups), I, I, I, I, I, P, SZ, P]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
-               "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly"):
+               "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -189,6 +190,19 @@ def build_bundles(gr: Groups, Hq: int, Hkv: int, Nq: int, num_logical_pages: int
     _check(lib.qup_build_bundles(ctypes.byref(cs), Hq, Hkv, Nq, num_logical_pages, max_group,
                                  _p(gr.workspace), gr.workspace.numel(), _stream_ptr(stream)),
            "qup_build_bundles")
+    gr._after(cs)
+    return gr
+
+
+def union_support(gr: Groups, Hq: int, Hkv: int, Nq: int, num_logical_pages: int, max_group: int = 8,
+                  stream=None) -> Groups:
+    """Every row of a group sees every page of its group's union (qup_union_support); the
+    bundles are rebuilt.  Attention on the result uses the group unions as supports."""
+    lib = load()
+    cs = gr.c_struct()
+    _check(lib.qup_union_support(ctypes.byref(cs), Hq, Hkv, Nq, num_logical_pages, max_group,
+                                 _p(gr.workspace), gr.workspace.numel(), _stream_ptr(stream)),
+           "qup_union_support")
     gr._after(cs)
     return gr
 

@@ -243,6 +243,26 @@ int qup_build_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
     return run_bundles(g, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, static_cast<cudaStream_t>(stream));
 }
 
+int qup_union_support(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, int max_group, void* ws,
+                      size_t ws_bytes, void* stream) {
+    size_t need = 0;
+    int64_t cap = 0;
+    int rc = qup_group_workspace(Hq, Hkv, Nq, 1, num_logical_pages, max_group, max_group, &need, &cap);
+    if (rc) return rc;
+    if (!g || !g->n_groups || !g->group_ptr || !g->members || !g->union_ptr || !g->union_pages || !g->row_mask ||
+        !bundle_fields_ok(g))
+        return QUP_ERR_ARG;
+    if (g->bundle_window < 0 || g->bundle_window > 256) return QUP_ERR_ARG;
+    if (!ws || ws_bytes < need) return QUP_ERR_CAPACITY;
+    DevState* ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (qup::launch_union_support(g->n_groups, g->group_ptr, g->union_ptr, g->row_mask, Hkv, Nq, Hq / Hkv,
+                                  g->cap_union, ds->err, ds->sms, st) != cudaSuccess)
+        return QUP_ERR_CUDA;
+    return run_bundles(g, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st);
+}
+
 int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int max_group,
                      int window, qup_groups* out, void* ws, size_t ws_bytes, void* stream) {
     size_t need = 0;

@@ -810,6 +810,45 @@ __global__ void __launch_bounds__(1024) bnd_order_kernel(const int32_t* __restri
 
 namespace qup {
 
+// Union as support (CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+// Selection, where a query block attends to its whole union table): every row of a group sees
+// every page of the group's union.  One warp per group sets each union entry's row mask to the
+// group's rows (bits 0 .. members * g - 1).
+__global__ void __launch_bounds__(256) grp_union_support_kernel(const int32_t* __restrict__ n_groups,
+                                                               const int32_t* __restrict__ group_ptr,
+                                                               const int32_t* __restrict__ union_ptr,
+                                                               uint64_t* __restrict__ row_mask, int Hkv, int Nq,
+                                                               int g, long long cap, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long x = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); x < (long long)Hkv * Nq;
+         x += nwarps) {
+        const int h = (int)(x / Nq), k = (int)(x % Nq);
+        if (k >= n_groups[h]) continue;
+        const size_t gp = (size_t)h * (Nq + 1) + k;
+        const int cnt = group_ptr[gp + 1] - group_ptr[gp];
+        const long long e0 = union_ptr[gp], e1 = union_ptr[gp + 1];
+        if (cnt < 1 || cnt * g > 64 || e0 < 0 || e1 < e0 || e1 > cap) {
+            if (lane == 0) atomicOr(err, QUP_ERR_GROUP);
+            continue;
+        }
+        const int R = cnt * g;
+        const uint64_t full = R == 64 ? ~0ull : ((1ull << R) - 1ull);
+        for (long long e = e0 + lane; e < e1; e += 32) row_mask[e] = full;
+    }
+}
+
+cudaError_t launch_union_support(const int32_t* n_groups, const int32_t* group_ptr, const int32_t* union_ptr,
+                                 uint64_t* row_mask, int Hkv, int Nq, int g, long long cap, unsigned* err, int sms,
+                                 cudaStream_t stream) {
+    const long long items = (long long)Hkv * Nq;
+    if (items == 0) return cudaSuccess;
+    const int grid = (int)std::min<long long>((items + 7) / 8, (long long)sms * 8);
+    grp_union_support_kernel<<<grid, 256, 0, stream>>>(n_groups, group_ptr, union_ptr, row_mask, Hkv, Nq, g, cap,
+                                                       err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gbits(const BundleLaunch& a, cudaStream_t stream) {
     const size_t smw = sizeof(uint32_t) * 8 * (size_t)a.NW;
     cudaError_t e = cudaFuncSetAttribute(bnd_gbits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smw);
