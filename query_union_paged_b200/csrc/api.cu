@@ -13,6 +13,14 @@
 #include "internal.h"
 #include "query_union_paged.h"
 
+namespace qup {
+// group.cu: every row of each group sees every page of the group's union (row masks set to the
+// group's rows)
+cudaError_t launch_union_support(const int32_t* n_groups, const int32_t* group_ptr, const int32_t* union_ptr,
+                                 uint64_t* row_mask, int Hkv, int Nq, int g, long long cap, unsigned* err, int sms,
+                                 cudaStream_t stream);
+}  // namespace qup
+
 namespace {
 
 __device__ unsigned g_err_word;  // ORed device error bits, read and cleared by qup_get_error

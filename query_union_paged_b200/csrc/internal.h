@@ -142,9 +142,5 @@ cudaError_t launch_bundles_fused(const BundleLaunch& a, int32_t* wcnt, uint64_t*
                                  cudaStream_t stream);
 // group union lists -> group bitsets (a.gbits), for bundles of a caller-given partition
 cudaError_t launch_gbits(const BundleLaunch& a, cudaStream_t stream);
-// every row of each group sees every page of the group's union (row masks set to the group's rows)
-cudaError_t launch_union_support(const int32_t* n_groups, const int32_t* group_ptr, const int32_t* union_ptr,
-                                 uint64_t* row_mask, int Hkv, int Nq, int g, long long cap, unsigned* err, int sms,
-                                 cudaStream_t stream);
 
 }  // namespace qup
