@@ -114,11 +114,23 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(src: str) -> str:
+    """Source text without // comments and blank lines: what the compiler turns into the kernel."""
+    lines = []
+    for line in src.splitlines():
+        code = re.sub(r"//.*$", "", line).rstrip()
+        if code.strip():
+            lines.append(code)
+    return "\n".join(lines)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the attention kernel's code (comments excluded): a recorded ncu capture counts only
+    while it matches."""
     h = hashlib.sha256()
     for name in ("union_attn.cu", "ptx.cuh", "internal.h"):
-        with open(os.path.join(ROOT, "query_union_paged_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "query_union_paged_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

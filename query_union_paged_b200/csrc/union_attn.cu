@@ -282,8 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kKProducerWarp || warp == kVProducerWarp) {
         // ============================================================ producers (whole warp each)
         // Both walk the same bundles and pages; the K warp fills the K ring, the V warp the
-        // V ring and the step metadata (indexed by V slot: it is read by the softmax of the
-        // step, which precedes the step's O update and so the slot's release).
+        // V ring (and stages each bundle for the softmax warps).
         const bool isV = warp == kVProducerWarp;
         const int NR = isV ? NSV : NSK;
         const CUtensorMap* tm = isV ? &tmV : &tmK;
