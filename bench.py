@@ -149,8 +149,10 @@ def profiled_traffic(workload_name: str):
 
 
 # kernels of one step: the fused grouping kernel, the fused bundling kernel (which also orders
-# the bundles), union attention (a memset of the look-back status words precedes them)
+# the bundles), union attention (a memset of the look-back status words precedes them); union
+# support adds its mask rewrite and the bundle rebuild (bitset and bundling kernels)
 LAUNCHES_PER_STEP = 3
+LAUNCHES_UNION_SUPPORT = 3
 
 
 class ClockSampler:
@@ -376,7 +378,7 @@ def main():
                      ("" if w.kv_dtype == W.DT_BF16 else " x nominal dtype ratio"),
                      "unique_kv_gbs": round(uniq_bytes / (attn_ms * 1e-3) / 1e9, 1),
                      "hbm_frac_unique_kv": round(uniq_bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (LAUNCHES_UNION_SUPPORT if args.union_support else 0)) * args.steps,
         "e2e": e2e,
     }
     if rank == 0:
