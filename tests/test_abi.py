@@ -77,3 +77,16 @@ def test_bundle_window_out_of_range_is_rejected_before_any_device_work(lib):
         assert rc == want, (bw, rc)
         rc = qup._lib.qup_build_bundles(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30, None)
         assert rc == want, (bw, rc)
+
+
+def test_union_support_rejects_bad_arguments_before_any_device_work(lib):
+    fake = [ctypes.c_void_p(0x1000 + 0x100 * i).value for i in range(len(qup._GROUP_KEYS) + len(qup._BUNDLE_KEYS))]
+    cs = qup._Groups(*fake[:len(qup._GROUP_KEYS)], 1 << 20, *fake[len(qup._GROUP_KEYS):], 0, 0)
+    qup.load()
+    # max_group 9, a missing workspace and an out-of-range bundle window are all refused on the host
+    assert qup._lib.qup_union_support(ctypes.byref(cs), 32, 8, 2048, 288, 9, ctypes.c_void_p(0x3000), 1 << 30,
+                                      None) == qup.ERR["ARG"]
+    assert qup._lib.qup_union_support(ctypes.byref(cs), 32, 8, 2048, 288, 8, None, 0, None) == qup.ERR["CAPACITY"]
+    cs.bundle_window = 512
+    assert qup._lib.qup_union_support(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30,
+                                      None) == qup.ERR["ARG"]
