@@ -1,7 +1,7 @@
 """Benchmark of the complete sparse-prefill call: page-affinity grouping followed by
 union attention, on one seeded synthetic prefill chunk per GPU.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4b] [--impl reference]
 
 A step = qup_sparse_group + qup_sparse_prefill_attn over the whole chunk (inputs
 resident in HBM). Each timed step is bracketed by CUDA events on the launching
@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 from query_union_paged_b200 import workloads as W  # noqa: E402
 
 METRIC = "selected-edge TFLOP/s of the complete sparse-prefill call (group + union attention)"
-CONFIG_DEFAULT = "2"
+CONFIG_DEFAULT = "4b"
 
 
 # ------------------------------------------------------------------ workload accounting

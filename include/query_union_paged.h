@@ -127,8 +127,8 @@ int qup_group_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages
                         int window, size_t* ws_bytes, int64_t* cap_union);
 
 /*
- * Bounded page-affinity grouping (Abstract: "a bounded GPU search produces
- * query IDs" from selected-page affinity; Figure 2).  Per KV head h, S(i) is
+ * Bounded page-affinity grouping (Abstract: a GPU search of bounded cost
+ * turns selected-page affinity into query-ID lists; Figure 2).  Per KV head h, S(i) is
  * the set of distinct valid pages of the g rows topk[h*g+j][i]; inside fixed
  * windows [w*window, (w+1)*window) of query IDs a group is seeded with the
  * smallest unassigned ID and grown, up to max_group members, by the candidate
@@ -156,7 +156,8 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
  *    for these sizes exceeds QUP_STATIC_GROUP_SCRATCH_BYTES; nothing is launched.
  *  - The first call on a device looks up the array's device address (a host
  *    query, with that device current); make that first call before capturing
- *    a stream.
+ *    a stream.  The address is cached per device context: after a device reset
+ *    (or in another context) the next call looks it up again.
  *  - Every call on one device shares the one array: two calls in flight at the
  *    same time (other streams, other host threads) race on it and corrupt each
  *    other's groups.  Order them on one stream.
@@ -203,9 +204,11 @@ int qup_union_support(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
  *   k_scale, v_scale  device fp32 [Hkv], > 0, required iff kv_dtype == QUP_E4M3
  *   page_table        device int32 [num_logical_pages]
  *   T                 page tokens: 16, 32, 64 or 128
- *   topk, Ksel        accepted for the problem statement's signature; the
- *                     groups' row masks carry each query's support and this
- *                     call does not read topk (may be NULL)
+ *   topk, Ksel        device int32 [Hq][Nq][Ksel] or NULL.  The groups' row
+ *                     masks carry each query's support: the kernel computes
+ *                     from them alone.  topk is read only in checked mode
+ *                     (qup_set_checked), which verifies the masks against it
+ *                     first.
  *   groups            output of qup_sparse_group (or qup_build_bundles on
  *                     any partition); the kernel walks its bundles
  *   q_pos, kv_len     device int32 [Nq]; tokens >= kv_len are never attended
@@ -237,6 +240,19 @@ const char* qup_error_string(int code);
  * is raised and every CTA exits cleanly.
  */
 int qup_set_debug(int wait_limit_ms, int skip_stage);
+
+/*
+ * Checked mode (process-wide, off by default; on = nonzero).  While it is on,
+ * qup_sparse_prefill_attn given a non-NULL topk first runs one extra kernel on
+ * the stream that checks every bundle row against its own TopK row: a mask
+ * bit is set exactly for the union pages the row selected (a set: duplicates
+ * and -1 dropped), every page of the row is in the bundle union, and rows of
+ * empty slots carry no bits.  A mismatch raises QUP_ERR_GROUP (a TopK ID out
+ * of range QUP_ERR_PAGE_ID) in the device error word; the attention call
+ * still runs.  Ksel < 0 is then QUP_ERR_ARG.  Meant for groups a caller builds
+ * itself; qup_sparse_group's groups satisfy it by construction.
+ */
+int qup_set_checked(int on);
 
 /* Number of SMs the persistent attention kernel is sized for on the current device. */
 int qup_num_sms(void);

@@ -21,9 +21,9 @@
  * kernel for any grouping.
  *
  * The grouping reference implements the bounded page-affinity rule read from
- * the Abstract ("a bounded GPU search produces query IDs" from
- * "selected-page affinity") and Figure 2 (logical page visits and masked
- * query-page slots), with sets held as sorted integer arrays:
+ * the Abstract (a search of bounded cost on the GPU turns the affinity of the
+ * queries' selected pages into lists of query IDs) and Figure 2 (logical page
+ * visits and masked query-page slots), with sets held as sorted integer arrays:
  *   per KV head h and query i, S(i) = sorted distinct valid pages of the g
  *   rows topk[h*g + j][i][:];  fixed windows [w*W, (w+1)*W) of query IDs;
  *   inside a window: seed = smallest unassigned ID, U = S(seed); while the

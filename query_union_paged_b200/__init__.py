@@ -20,7 +20,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host", "union_support",
-           "get_error", "set_debug", "load",
+           "get_error", "set_debug", "set_checked", "load",
            "QupError", "F32", "BF16", "E4M3", "ERR"]
 
 F32, BF16, E4M3 = 0, 1, 2
@@ -71,8 +71,10 @@ def load():
     lib.qup_num_sms.argtypes = []
     lib.qup_exp2_poly.argtypes = [P, P, I, P]
     lib.qup_union_support.argtypes = [ctypes.POINTER(_Groups), I, I, I, I, I, P, SZ, P]
+    lib.qup_set_checked.argtypes = [I]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
-               "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support"):
+               "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support",
+               "qup_set_checked"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -296,6 +298,12 @@ def get_error(stream=None) -> int:
 
 def set_debug(wait_limit_ms: int = 0, skip_stage: int = -1):
     _check(load().qup_set_debug(wait_limit_ms, skip_stage), "qup_set_debug")
+
+
+def set_checked(on: bool):
+    """Checked mode (qup_set_checked): attention calls given topk first verify every bundle row's
+    page mask against its TopK row and raise the GROUP error bit on a mismatch."""
+    _check(load().qup_set_checked(1 if on else 0), "qup_set_checked")
 
 
 def num_sms() -> int:

@@ -28,8 +28,8 @@ __device__ unsigned g_err_word;  // ORed device error bits, read and cleared by 
 constexpr int kMaxDevices = 64;
 
 struct DevState {
-    bool ready = false;
-    unsigned* err = nullptr;  // device address of g_err_word on this device
+    unsigned long long ctx = 0;  // context the fields below were looked up in (0: not yet)
+    unsigned* err = nullptr;     // device address of g_err_word in that context
     int sms = 0;
     int smem_optin = 0;
 };
@@ -38,6 +38,7 @@ std::mutex g_mu;
 DevState g_dev[kMaxDevices];
 std::atomic<int> g_wait_limit_ms{0};  // 0: default
 std::atomic<int> g_skip_stage{-1};
+std::atomic<int> g_checked{0};  // checked mode: attention validates the row masks against topk
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -47,9 +48,11 @@ EncodeTiledFn g_encode = nullptr;
 int device_state(DevState** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QUP_ERR_CUDA;
+    const unsigned long long ctx = qup::context_id();
+    if (ctx == 0) return QUP_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
     DevState& s = g_dev[dev];
-    if (!s.ready) {
+    if (s.ctx != ctx) {  // first call in this context (a reset or another context starts over)
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return QUP_ERR_CUDA;
         s.err = static_cast<unsigned*>(p);
@@ -65,7 +68,7 @@ int device_state(DevState** out) {
                 return QUP_ERR_CUDA;
             g_encode = reinterpret_cast<EncodeTiledFn>(fn);
         }
-        s.ready = true;
+        s.ctx = ctx;
     }
     *out = &s;
     return QUP_OK;
@@ -351,8 +354,6 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                             int num_logical_pages, int P_phys, int T, const int32_t* topk, int Ksel,
                             const qup_groups* groups, const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq,
                             int d, float softmax_scale, void* O, float* lse, void* stream) {
-    (void)topk;
-    (void)Ksel;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || d != qup::kHeadDim) return QUP_ERR_ARG;
     if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
     // supported (dtype, page size) pairs: bf16 16/32/64/128, E4M3 64/128, fp32 32/64
@@ -372,9 +373,16 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(groups->bunion_mask)) & 15) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
     if (128 % g != 0 || groups->rows_per_group % g != 0) return QUP_ERR_ARG;
+    const bool checked = g_checked.load() != 0 && topk != nullptr;
+    if (checked && Ksel < 0) return QUP_ERR_ARG;
     DevState* ds = nullptr;
     int rc = device_state(&ds);
     if (rc) return rc;
+    if (checked && qup::launch_check_support(topk, Ksel, Hkv, Nq, g, num_logical_pages, groups->n_bundles,
+                                             groups->bunion_ptr, groups->bunion_pages, groups->bunion_mask,
+                                             groups->bundle_qid, groups->cap_union, ds->err, ds->sms,
+                                             static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return QUP_ERR_CUDA;
 
     // K / V cache tensor maps: dims (d, T, Hkv, P_phys), box (128 bytes of d, T, 1, 1), 128B swizzle
     CUtensorMap tm[2];
@@ -472,6 +480,11 @@ int qup_set_debug(int wait_limit_ms, int skip_stage) {
     return QUP_OK;
 }
 
+int qup_set_checked(int on) {
+    g_checked = on ? 1 : 0;
+    return QUP_OK;
+}
+
 int qup_num_sms(void) {
     DevState* ds = nullptr;
     return device_state(&ds) == QUP_OK ? ds->sms : 0;
@@ -486,28 +499,60 @@ int qup_exp2_poly(const float* x, float* y, int n, void* stream) {
 
 namespace qup {
 
+unsigned long long context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext*);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext c = nullptr;
+    if (get_current(&c) != CUDA_SUCCESS) return 0;
+    if (c == nullptr) {  // no context on this thread yet: cudaSetDevice makes the primary one current
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return 0;
+        if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+    }
+    unsigned long long id = 0;
+    if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id + 1;  // never 0
+}
+
 cudaError_t ensure_smem_attr(const void* fn, size_t smem) {
     struct Entry {
-        int dev;
+        unsigned long long ctx;
         const void* fn;
         size_t smem;
     };
     static std::mutex mu;
     static Entry table[256];
     static int n = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
+    const unsigned long long ctx = context_id();
+    if (ctx == 0) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < n; ++i)
-        if (table[i].dev == dev && table[i].fn == fn) {
+        if (table[i].ctx == ctx && table[i].fn == fn) {
             if (table[i].smem >= smem) return cudaSuccess;
-            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e == cudaSuccess) table[i].smem = smem;
             return e;
         }
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess && n < 256) table[n++] = Entry{dev, fn, smem};
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) {
+        if (n < 256) table[n++] = Entry{ctx, fn, smem};
+        else table[(size_t)(ctx + (uintptr_t)fn) % 256] = Entry{ctx, fn, smem};  // full: overwrite one
+    }
     return e;
 }
 

@@ -1,6 +1,6 @@
-// group.cu -- bounded page-affinity grouping (PageWeaver, Abstract: "a bounded
-// GPU search produces query IDs" from selected-page affinity; Figure 2:
-// logical page visits and masked query-page slots).
+// group.cu -- bounded page-affinity grouping (PageWeaver, Abstract: a GPU
+// search of bounded cost turns selected-page affinity into query-ID lists;
+// Figure 2: logical page visits and masked query-page slots).
 //
 // Three kernels, all deterministic:
 //   1. rowbits: one warp per TopK row builds the row's page bitset (duplicates

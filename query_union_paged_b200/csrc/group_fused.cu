@@ -1,6 +1,7 @@
 // group_fused.cu -- the grouping call in two fused kernels (PageWeaver,
-// Abstract: "a bounded GPU search produces query IDs" from selected-page
-// affinity; Figure 2: logical page visits and masked query-page slots).
+// Abstract: a GPU search of bounded cost turns the affinity of the queries'
+// selected pages into query-ID lists; Figure 2: logical page visits and masked
+// query-page slots).
 //
 // Same rule and same outputs as the multi-kernel path in group.cu, with the
 // intermediate state kept in shared memory:

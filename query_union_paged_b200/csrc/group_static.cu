@@ -14,6 +14,7 @@
 
 #include <mutex>
 
+#include "internal.h"
 #include "query_union_paged.h"
 
 namespace {
@@ -25,19 +26,28 @@ __device__ __align__(256) unsigned char g_group_scratch[QUP_STATIC_GROUP_SCRATCH
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices];  // device address of g_group_scratch, per device
+struct ScratchAddr {
+    unsigned long long ctx;  // context the address was looked up in (0: not yet)
+    void* ptr;               // device address of g_group_scratch in that context
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Looks the symbol up once per device, with that device current.
+// Looks the symbol up once per device context, with that device current: a device reset or a
+// non-primary context gets a new context ID and a fresh lookup, so a stale address is never used.
 int scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QUP_ERR_CUDA;
+    const unsigned long long ctx = qup::context_id();
+    if (ctx == 0) return QUP_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    ScratchAddr& a = g_scratch[dev];
+    if (a.ctx != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_group_scratch) != cudaSuccess || p == nullptr) return QUP_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
+        a.ptr = p;
+        a.ctx = ctx;
     }
-    *out = g_scratch_ptr[dev];
+    *out = a.ptr;
     return QUP_OK;
 }
 

@@ -14,9 +14,15 @@ constexpr int kHeadDim = 128;
 constexpr int kMaxPPS = 8;      // pages per 128-token step at T = 16
 constexpr int kMaxStages = 16;
 
-// Raises a kernel's dynamic shared-memory limit to `smem` once per device (the
+// Raises a kernel's dynamic shared-memory limit to `smem` once per device context (the
 // attribute is a maximum: later launches with less need no call).
 cudaError_t ensure_smem_attr(const void* fn, size_t smem);
+
+// Unique ID (over the life of the process) of the CUDA context current on this thread, the
+// primary context of the current device being made current first if none is.  Caches of
+// device addresses and kernel attributes are keyed on it: a device reset or another context
+// gets a new ID, so nothing looked up in an earlier context is reused.  0 on failure.
+unsigned long long context_id();
 
 // Launch with programmatic stream serialization: the kernel may start while the
 // previous kernel of the stream finishes; it calls grid_dep_wait() before it
@@ -67,6 +73,12 @@ size_t attn_tile_bytes(int es);
 
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);
+
+// checked mode: every bundle row's page mask against its own TopK row (QUP_ERR_GROUP on a mismatch)
+cudaError_t launch_check_support(const int32_t* topk, int K, int Hkv, int Nq, int g, int P, const int32_t* n_bundles,
+                                 const int32_t* bunion_ptr, const int32_t* bunion_pages,
+                                 const uint32_t* bunion_mask, const int32_t* bundle_qid, long long cap,
+                                 unsigned* err, int sms, cudaStream_t stream);
 
 // the softmax's polynomial 2^x over n floats (test hook)
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);

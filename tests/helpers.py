@@ -1,7 +1,26 @@
 """Shared test utilities: move a seeded workload to the GPU and compare results."""
+import dataclasses
+import functools
+
 import numpy as np
 
 from query_union_paged_b200 import workloads as W
+
+
+@functools.lru_cache(maxsize=None)
+def workload(cfg: str):
+    """The named full-size workload, generated once per test session (callers must not modify it)."""
+    return W.make(cfg)
+
+
+def permute_queries(w, perm, q_pos=None, name_suffix="perm"):
+    """The same problem with query IDs renumbered: new query i is old query perm[i] (its Q row, its
+    TopK rows and its position move with it).  q_pos, if given, replaces the permuted positions."""
+    perm = np.asarray(perm)
+    pos = w.q_pos[perm] if q_pos is None else np.asarray(q_pos, np.int32)
+    return dataclasses.replace(w, name=f"{w.name}_{name_suffix}", Q=np.ascontiguousarray(w.Q[perm]),
+                               topk=np.ascontiguousarray(w.topk[:, perm]),
+                               q_pos=np.ascontiguousarray(pos, dtype=np.int32))
 
 
 def to_device(w, device="cuda"):
@@ -99,10 +118,13 @@ def out_to_f64(O):
 TOL = {W.DT_F32: (2e-2, 2e-3), W.DT_BF16: (2e-2, 2e-3), W.DT_E4M3: (6e-2, 6e-3)}
 
 
-def check_close(got, ref, kv_dtype, what=""):
+def check_close(got, ref, kv_dtype, what="", report=False):
     err = np.abs(got - ref)
     mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
     tmax, tmean = TOL[kv_dtype]
+    if report:  # one parseable line per comparison (shown with pytest -s)
+        print(f"PARITY {what} elements={err.size} max_abs={mx:.3e} (bound {tmax}) "
+              f"mean_abs={mean:.3e} (bound {tmean})", flush=True)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     assert mx <= tmax and mean <= tmean, f"{what}: max abs {mx:.3e} (<= {tmax}), mean abs {mean:.3e} (<= {tmean})"
     return mx, mean

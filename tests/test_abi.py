@@ -4,6 +4,7 @@ the workload generator is deterministic."""
 import ctypes
 import os
 import re
+import textwrap
 
 import numpy as np
 import pytest
@@ -66,23 +67,44 @@ def test_generator_is_deterministic():
     assert np.all(w.topk[0] == w.topk[3]) and not np.all(w.topk[0] == w.topk[4])
 
 
+def _run_without_devices(code: str):
+    """Run `code` in a fresh interpreter that sees no CUDA device.  The argument checks below pass
+    made-up non-null buffer addresses: with no device visible, a check that stopped answering
+    first would end in QUP_ERR_CUDA, never in a kernel launch on those addresses."""
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    prog = f"import sys; sys.path.insert(0, {ROOT!r})\n" + textwrap.dedent(code)
+    res = subprocess.run([sys.executable, "-c", prog], env=env, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stdout + res.stderr
+
+
+_FAKE_GROUPS = """
+    import ctypes
+    import query_union_paged_b200 as qup
+    qup.load()
+    fake = [0x1000 + 0x100 * i for i in range(len(qup._GROUP_KEYS) + len(qup._BUNDLE_KEYS))]
+    def groups(bw):
+        return qup._Groups(*fake[:len(qup._GROUP_KEYS)], 1 << 20, *fake[len(qup._GROUP_KEYS):], 0, bw)
+"""
+
+
 def test_bundle_window_out_of_range_is_rejected_before_any_device_work(lib):
-    # every buffer pointer is non-null but fake: the argument checks run before the device is touched
-    fake = [ctypes.c_void_p(0x1000 + 0x100 * i).value for i in range(len(qup._GROUP_KEYS) + len(qup._BUNDLE_KEYS))]
-    for bw, want in ((300, qup.ERR["ARG"]), (-1, qup.ERR["ARG"])):
-        cs = qup._Groups(*fake[:len(qup._GROUP_KEYS)], 1 << 20, *fake[len(qup._GROUP_KEYS):], 0, bw)
-        qup.load()
+    _run_without_devices(_FAKE_GROUPS + """
+    for bw in (300, -1):
+        cs = groups(bw)
         rc = qup._lib.qup_sparse_group(ctypes.c_void_p(0x2000), 32, 8, 2048, 16, 288, 8, 64, ctypes.byref(cs),
                                        ctypes.c_void_p(0x3000), 1 << 30, None)
-        assert rc == want, (bw, rc)
-        rc = qup._lib.qup_build_bundles(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30, None)
-        assert rc == want, (bw, rc)
+        assert rc == qup.ERR["ARG"], (bw, rc)
+        rc = qup._lib.qup_build_bundles(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30,
+                                        None)
+        assert rc == qup.ERR["ARG"], (bw, rc)
+""")
 
 
 def test_union_support_rejects_bad_arguments_before_any_device_work(lib):
-    fake = [ctypes.c_void_p(0x1000 + 0x100 * i).value for i in range(len(qup._GROUP_KEYS) + len(qup._BUNDLE_KEYS))]
-    cs = qup._Groups(*fake[:len(qup._GROUP_KEYS)], 1 << 20, *fake[len(qup._GROUP_KEYS):], 0, 0)
-    qup.load()
+    _run_without_devices(_FAKE_GROUPS + """
+    cs = groups(0)
     # max_group 9, a missing workspace and an out-of-range bundle window are all refused on the host
     assert qup._lib.qup_union_support(ctypes.byref(cs), 32, 8, 2048, 288, 9, ctypes.c_void_p(0x3000), 1 << 30,
                                       None) == qup.ERR["ARG"]
@@ -90,3 +112,26 @@ def test_union_support_rejects_bad_arguments_before_any_device_work(lib):
     cs.bundle_window = 512
     assert qup._lib.qup_union_support(ctypes.byref(cs), 32, 8, 2048, 288, 8, ctypes.c_void_p(0x3000), 1 << 30,
                                       None) == qup.ERR["ARG"]
+""")
+
+
+def test_checked_mode_argument_and_no_device_answer(lib):
+    _run_without_devices(_FAKE_GROUPS + """
+    assert qup._lib.qup_set_checked(1) == 0
+    cs = groups(0)
+    cs.rows_per_group = 32
+    # Ksel < 0 with topk given is an argument error in checked mode, found before the device
+    rc = qup._lib.qup_sparse_prefill_attn(ctypes.c_void_p(0x10000), 1, ctypes.c_void_p(0x20000),
+                                          ctypes.c_void_p(0x30000), 1, None, None, ctypes.c_void_p(0x4000), 288,
+                                          288, 64, ctypes.c_void_p(0x5000), -1, ctypes.byref(cs),
+                                          ctypes.c_void_p(0x6000), 18432, 32, 8, 2048, 128, 0.088,
+                                          ctypes.c_void_p(0x70000), None, None)
+    assert rc == qup.ERR["ARG"], rc
+    # valid arguments reach the device lookup, which answers that there is no device
+    rc = qup._lib.qup_sparse_prefill_attn(ctypes.c_void_p(0x10000), 1, ctypes.c_void_p(0x20000),
+                                          ctypes.c_void_p(0x30000), 1, None, None, ctypes.c_void_p(0x4000), 288,
+                                          288, 64, ctypes.c_void_p(0x5000), 16, ctypes.byref(cs),
+                                          ctypes.c_void_p(0x6000), 18432, 32, 8, 2048, 128, 0.088,
+                                          ctypes.c_void_p(0x70000), None, None)
+    assert rc == qup.ERR["CUDA"], rc
+""")

@@ -1,9 +1,8 @@
 """GPU union attention (qup_sparse_prefill_attn through the C ABI) vs the fp64 oracle.
 
 Bounds (max abs, mean abs): bf16 and fp32 inputs 2e-2 / 2e-3; E4M3 KV 6e-2 / 6e-3.
-Small cases are compared on every output element; full-size workloads in the
-launch configuration the bench times are compared on sampled rows the oracle
-computes one by one.
+Every case, the full-size workloads in the launch configuration the bench
+times included, is compared on every output element.
 """
 import numpy as np
 import pytest
@@ -12,7 +11,7 @@ import oracle
 import query_union_paged_b200 as qup
 from query_union_paged_b200 import workloads as W
 
-from helpers import check_close, out_to_f64, to_device
+from helpers import check_close, out_to_f64, permute_queries, to_device, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -131,27 +130,73 @@ def test_identity_page_table_and_single_member_groups():
     check_close(got, ref, w.kv_dtype, "groups of one")
 
 
-def _sampled(w, n, seed):
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(w.Hq * w.Nq, size=min(n, w.Hq * w.Nq), replace=False)).astype(np.int64)
-    return rows
-
-
 @pytest.mark.parametrize("cfg", ["2", "3", "4a", "4b", "4c", "5"])
-def test_full_size_sampled_rows(cfg):
-    w = W.make(cfg)
+def test_full_size_every_element(cfg):
+    """The whole output of each full-size workload, grouped as the bench groups it."""
+    w = workload(cfg)
     dev = to_device(w)
     O = out_to_f64(_attn(w, dev, _gpu_groups(w, dev)))
-    assert np.all(np.isfinite(O))
-    rows = _sampled(w, 384, 17)
-    ref = oracle.sparse_attn_workload(w, rows=rows)
-    hq, i = rows // w.Nq, rows % w.Nq
-    check_close(O[i, hq], ref, w.kv_dtype, w.name)
+    ref = oracle.sparse_attn_workload(w)
+    check_close(O, ref, w.kv_dtype, w.name, report=True)
+
+
+def _shuffled_positions(w, seed, max_back):
+    """Query IDs in random order, and each position moved back by up to max_back tokens (gaps,
+    repeats, out of order): rows may then hold pages past their query, which the causal limit
+    empties."""
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(w.Nq)
+    pos = np.maximum(w.q_pos[perm] - rng.integers(0, max_back + 1, size=w.Nq), 0)
+    return permute_queries(w, perm, q_pos=pos, name_suffix=f"shuffled{seed}")
+
+
+SHUFFLED = [
+    dict(seed=20),
+    dict(seed=21, T=128, prefix=700, Nq=150, kv_dtype=W.DT_E4M3),
+    dict(seed=22, T=32, prefix=1000, Hq=8, Hkv=2),
+    dict(seed=23, q_dtype=W.DT_F32, kv_dtype=W.DT_F32, T=64),
+]
+
+
+@pytest.mark.parametrize("kw", SHUFFLED, ids=lambda k: f"s{k['seed']}")
+def test_positions_out_of_id_order(kw):
+    """Positions carried by the query IDs in any order (shuffled, gapped, repeated)."""
+    w = _shuffled_positions(W.random_small(**kw), kw["seed"], 3 * W.random_small(**kw).T)
+    ref = oracle.sparse_attn_workload(w)
+    dev = to_device(w)
+    for name, gr in (("online", _gpu_groups(w, dev)), ("fixed", _gpu_groups(w, dev, w.max_group, w.max_group))):
+        check_close(out_to_f64(_attn(w, dev, gr)), ref, w.kv_dtype, f"{w.name}/{name}", report=True)
+
+
+@pytest.mark.parametrize("cfg", ["2", "4b"])
+def test_full_size_positions_out_of_id_order(cfg):
+    """A full-size workload with its query IDs shuffled and positions moved back by up to a page."""
+    w0 = workload(cfg)
+    w = _shuffled_positions(w0, 31, w0.T)
+    dev = to_device(w)
+    O = out_to_f64(_attn(w, dev, _gpu_groups(w, dev)))
+    ref = oracle.sparse_attn_workload(w)
+    check_close(O, ref, w.kv_dtype, w.name, report=True)
+
+
+@pytest.mark.parametrize("T", [64, 128])
+def test_e4m3_ragged_kv_len_with_nan_bytes(T):
+    """E4M3 KV with the last page partly filled and NaN bytes (0x7F) past kv_len."""
+    w = W.random_small(40 + T, kv_dtype=W.DT_E4M3, T=T, prefix=1000, Nq=77, Hq=8, Hkv=2)
+    fill = w.kv_len % w.T
+    assert fill != 0
+    last_phys = w.page_table[w.num_logical_pages - 1]
+    w.Kc[last_phys, :, fill:, :] = 0x7F
+    w.Vc[last_phys, :, fill:, :] = 0x7F
+    ref = oracle.sparse_attn_workload(w)
+    dev = to_device(w)
+    got = out_to_f64(_attn(w, dev, _gpu_groups(w, dev)))
+    check_close(got, ref, w.kv_dtype, f"e4m3 nan tail T={T}", report=True)
 
 
 @pytest.mark.parametrize("cfg", ["2", "4b"])
 def test_outputs_do_not_depend_on_grouping(cfg):
-    w = W.make(cfg)
+    w = workload(cfg)
     dev = to_device(w)
     a = out_to_f64(_attn(w, dev, _gpu_groups(w, dev, 8, 64)))
     b = out_to_f64(_attn(w, dev, _gpu_groups(w, dev, 8, 8)))

@@ -6,7 +6,7 @@ import oracle
 import query_union_paged_b200 as qup
 from query_union_paged_b200 import workloads as W
 
-from helpers import assert_bundles_equal, assert_groups_equal, groups_to_host
+from helpers import assert_bundles_equal, assert_groups_equal, groups_to_host, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def test_random_small_bitexact(seed):
 @pytest.mark.parametrize("cfg", ["1", "2", "3", "4a", "4b", "4c", "5"])
 @pytest.mark.parametrize("window", [64, 8, 128, 256])
 def test_workload_bitexact(cfg, window):
-    w = W.make(cfg)
+    w = workload(cfg)
     got = _run(w.topk, w.Hq, w.Hkv, w.num_logical_pages, 8, window)
     ref = oracle.group(w.topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, 8, window)
     assert_groups_equal(got, ref)

@@ -11,7 +11,7 @@ import oracle
 import query_union_paged_b200 as qup
 from query_union_paged_b200 import workloads as W
 
-from helpers import check_close, groups_to_host, out_to_f64, to_device
+from helpers import check_close, groups_to_host, out_to_f64, to_device, workload
 
 pytestmark = pytest.mark.gpu
 
@@ -57,10 +57,10 @@ def test_union_support_small_full_output():
 
 
 def test_union_support_block_union_workload_sampled_rows():
-    w = W.make("5")
+    w = workload("5")
     got, wu = _run(w, w.window)
     rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(w.Hq * w.Nq, size=256, replace=False)).astype(np.int64)
+    rows = np.sort(rng.choice(w.Hq * w.Nq, size=2048, replace=False)).astype(np.int64)
     ref = oracle.sparse_attn_workload(wu, rows=rows)
     hq, i = rows // w.Nq, rows % w.Nq
     check_close(got[i, hq], ref, w.kv_dtype, "union support, block-union workload")

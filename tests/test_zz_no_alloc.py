@@ -1,7 +1,8 @@
 """qup_sparse_group_static (grouping with its scratch in the library's own fixed
 device array) vs qup_sparse_group (caller workspace): identical groups and
 bundles, over two calls in a row with different problems, called through the
-C ABI.  Runs alone or after every other test file.
+C ABI; the second call of each problem changes neither torch's allocated bytes
+nor the device's free memory.  Runs alone or after every other test file.
 """
 import ctypes
 
@@ -26,10 +27,8 @@ def _lib():
     return lib
 
 
-def _static_group(topk, Hq, Hkv, P, max_group, window):
+def _static_group_into(out, topk, Hq, Hkv, P, max_group, window):
     Hq_, Nq, K = topk.shape
-    ws_bytes, cap = qup.group_workspace(Hq, Hkv, Nq, K, P, max_group, window)
-    out = qup.alloc_groups(Hq, Hkv, Nq, cap, 0, topk.device)  # outputs only, no workspace
     cs = out.c_struct()
     rc = _lib().qup_sparse_group_static(ctypes.c_void_p(topk.data_ptr()), Hq, Hkv, Nq, K, P, max_group,
                                         window, ctypes.byref(cs), None)
@@ -53,8 +52,18 @@ def test_static_scratch_matches_workspace_entry_point_two_calls_in_a_row():
         ws_bytes, _ = qup.group_workspace(Hq, Hkv, topk.shape[1], topk.shape[2], P, mg, win)
         assert ws_bytes <= STATIC_LIMIT
         ref = groups_to_host(qup.sparse_group(topk, Hq, Hkv, P, mg, win))
-        for _ in range(2):
-            got = groups_to_host(_static_group(topk, Hq, Hkv, P, mg, win))
+        for call in range(2):
+            Hq_, Nq, K = topk.shape
+            _, cap = qup.group_workspace(Hq, Hkv, Nq, K, P, mg, win)
+            out = qup.alloc_groups(Hq, Hkv, Nq, cap, 0, topk.device)  # outputs only, no workspace
+            torch.cuda.synchronize()
+            before = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+            _static_group_into(out, topk, Hq, Hkv, P, mg, win)
+            torch.cuda.synchronize()
+            after = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+            if call == 1:  # the first call may still load the library's module; the second allocates nothing
+                assert after == before, (before, after)
+            got = groups_to_host(out)
             assert qup.get_error() == 0
             assert_groups_equal(got, ref)
             assert_bundles_equal(got, ref)
