@@ -401,6 +401,20 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QUP_ERR_ARG;
     }
+    // Q rows for the bf16 kernel's Q operand: dims (d, Hq, Nq), box (64 elements, g heads, 1 query),
+    // 128-byte swizzle (the operand's K-major layout); a query coordinate of Nq reads zeros
+    CUtensorMap tmq;
+    std::memset(&tmq, 0, sizeof(tmq));
+    if (es == 2) {
+        const cuuint64_t qdims[3] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)Nq};
+        const cuuint64_t qstrides[2] = {(cuuint64_t)d * 2, (cuuint64_t)Hq * d * 2};
+        const cuuint32_t qbox[3] = {64, (cuuint32_t)g, 1};
+        const cuuint32_t qestr[3] = {1, 1, 1};
+        if (g_encode(&tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(Q), qdims, qstrides, qbox, qestr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QUP_ERR_ARG;
+    }
     // a pipeline step is 128 tokens: as many K and V tiles in flight as shared memory allows,
     // split between the K ring and the V ring (a V slot is held longer: through the softmax)
     int nt = 2 * qup::kMaxStages;
@@ -441,7 +455,7 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.wait_limit_ns = (unsigned long long)(wait_ms > 0 ? wait_ms : 2000) * 1000000ull;
     p.dbg_skip_stage = g_skip_stage.load();
     const cudaError_t e =
-        qup::launch_union_attn(es, T, tm[0], tm[1], p, ds->sms, smem, static_cast<cudaStream_t>(stream));
+        qup::launch_union_attn(es, T, tm[0], tm[1], tmq, p, ds->sms, smem, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
 }
 

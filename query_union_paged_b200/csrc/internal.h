@@ -71,7 +71,9 @@ struct AttnParams {
 size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g);
 size_t attn_tile_bytes(int es);
 
-cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV,
+// tmQ: Q [Nq][Hq][d] bf16 with a box of (64 elements, g heads, 1 query) and 128-byte swizzle
+// (read by the bf16 kernel only)
+cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);
 
 // checked mode: every bundle row's page mask against its own TopK row (QUP_ERR_GROUP on a mismatch)

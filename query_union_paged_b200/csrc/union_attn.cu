@@ -5,56 +5,64 @@
 // page-affine groups of one KV head, see qup_groups).  Pages of the bundle
 // union are streamed once per bundle in steps of 128 tokens (one 128-token
 // page, or 128 / T smaller pages) through two TMA rings, one of K tiles and
-// one of V tiles.  Per step g, with b = g & 1:
-//      S_b  = Q K^T     M = 128 rows, N = 128 tokens, K = d  (Q from TMEM, K from smem)
-//      P_b  = masked online softmax of S_b, written over S_b  (TMEM -> registers -> TMEM)
-//      O   += P_b V     M = 128 rows, N = d, K = 128 tokens   (P from TMEM, V from smem)
-// One warpgroup runs the softmax: thread = TMEM lane = bundle row, so the row
-// max and the row sum never leave the thread, and each SM sub-partition holds
-// one softmax warp (two busy softmax warps on one sub-partition starve each
-// other's latency-bound phases).  While it works on step g the tensor pipe
-// runs O += P(g-1) V and then S(g+1) = Q K^T: P is written over the S buffer
-// it came from, so S(g+2) waits for the O update of step g.
+// one of V tiles.  Step s of a bundle belongs to softmax warpgroup w = s % 2,
+// which owns S buffer w and O accumulator w in TMEM:
+//      S_w  = Q K^T     M = 128 rows, N = 128 tokens, K = d  (Q and K from shared memory)
+//      P_w  = masked online softmax of S_w, written over S_w  (TMEM -> registers -> TMEM)
+//      O_w += P_w V     M = 128 rows, N = d, K = 128 tokens   (P from TMEM, V from shared memory)
+// Thread = TMEM lane = bundle row in both warpgroups, so a row's running max
+// and sum never leave its thread; each warpgroup keeps its own for its steps.
+// While one warpgroup computes the exponentials of step s, the other works on
+// step s + 1 and the tensor pipe runs the O update of step s - 1 and S of step
+// s + 2: the serial chain of one warp (TMEM load, row max, exponentials, P
+// store) is hidden behind the other warp of its SM sub-partition.  The
+// epilogue merges the two partial results of each row (O_0, O_1 with their
+// maxima and sums) and writes the row to O[qid][h'].
 // A row's max is only raised when a score exceeds it by more than kTau (log2
-// units); O and the row sum are rescaled then, which after the first steps is
-// rare.  A warp whose 32 rows selected none of a step's pages skips that
+// units); O_w and the row sum are rescaled then, which after the first steps
+// is rare.  A warp whose 32 rows selected none of a step's pages skips that
 // step's exponentials.  Each softmax warp reads the bundle's page numbers and
 // its own 32-bit word of every page's row mask straight from the bundle
-// arrays, 32 entries at a time, one batch ahead; it waits for a V tile only
-// on a step whose page reaches kv_len (whose V rows past kv_len it zeroes).
-// A quarter of the exponentials come from a polynomial on the FMA pipe
+// arrays, 32 entries at a time, one batch ahead; it waits for a V tile only on
+// a step whose page reaches kv_len (whose V rows past kv_len it zeroes).  A
+// quarter of the exponentials come from a polynomial on the FMA pipe
 // (exp2_poly2) and the rest from the MUFU unit.
 //
-// Bundle boundaries: the V warp stages each bundle a few steps ahead (header,
-// query IDs and positions, and the bundle's Q rows by original query ID,
-// bulk-copied into shared memory); right after a bundle's last P the softmax
-// warps move the next bundle's Q rows into the other of two TMEM Q buffers,
-// so the next bundle's first S = Q K^T runs during this bundle's epilogue.
+// Q: the bundle's rows, gathered by original query ID (no reordered Q tensor),
+// sit in shared memory as the A operand of S in the 128-byte-swizzled K-major
+// layout.  bf16: the V producer loads them by TMA (one box of g heads x 64
+// elements per query and half of d; empty query slots read zeros from outside
+// the tensor) once every S of the previous bundle has completed.  E4M3: the V
+// producer bulk-copies the bf16 rows into a stage, and softmax warpgroup 0
+// quantises each row to E4M3 with its own scale into the operand.  fp32: the
+// same warpgroup copies the rows from global memory.
 //
-// Warp roles (256 threads):
-//   warps 0-3  softmax / epilogue: thread = TMEM lane = bundle row.  They
-//              also move each bundle's Q rows (gathered by original query ID:
-//              no reordered Q tensor) into TMEM.
-//   warp 4     K producer: walks the bundle's page list, resolves physical
-//              pages (warp-parallel) and TMA-loads the K tiles.
-//   warp 6     V producer: the same walk for the V tiles; stages each bundle.
-//   warp 5     S issuer (one elected lane of a warp-uniform loop) and TMEM
-//              owner (512 columns): S(g) once K tile g has landed and the O
-//              update of step g - 2 has finished with S_b.
-//   warp 7     PV issuer: O += P_b V once P(g) and V tile g are ready.
-// The two issuers sit on different SM sub-partitions, each beside one softmax
-// warp and no other busy warp; producers and issuers wait with suspended
-// try_waits, which leave the sub-partition's issue slots to the softmax.
-// TMEM columns: O [0,128); S_0 [128,256); S_1 [256,384); two Q buffers from
-// 384 (bf16: 64 columns each, E4M3: 32; fp32 Q stays in shared memory).  P_b
-// occupies the first kPCols columns of S_b.
-// Operand types: bf16 (kind::f16), fp32 (kind::tf32, Q in shared memory),
-// FP8 E4M3 (kind::f8f6f4: K and V straight from the cache, Q quantised per
-// row with its own scale, P stored as E4M3 of 2^4 p).  Every MMA consumes 32
-// bytes of its K extent per row, so the descriptor arithmetic is shared.
+// Warp roles (384 threads; warp w runs on SM sub-partition w % 4):
+//   warps 0-3   softmax warpgroup 0 (even steps), warps 4-7 warpgroup 1 (odd
+//               steps); both run the epilogue, each for half of the columns.
+//   warp 8      K producer: walks the bundle's page list, resolves physical
+//               pages (warp-parallel) and TMA-loads the K tiles.
+//   warp 10     V producer: the same walk for the V tiles; writes each
+//               bundle's header (query IDs and positions of its rows) and
+//               loads or stages its Q rows.
+//   warp 9      S issuer (one elected lane of a warp-uniform loop) and TMEM
+//               owner (512 columns): S(s) once K tile s has landed and the O
+//               update that last read P from S_w has finished.
+//   warp 11     PV issuer: O_w += P_w V once P(s) and V tile s are ready.
+// Producers and issuers wait with suspended try_waits, which leave the
+// sub-partition's issue slots to the softmax warps, and give registers to
+// them (setmaxnreg).
+// TMEM columns: O_0 [0,128); O_1 [128,256); S_0 [256,384); S_1 [384,512).
+// P_w occupies the first kPCols columns of S_w.
+// Operand types: bf16 (kind::f16), fp32 (kind::tf32), FP8 E4M3
+// (kind::f8f6f4: K and V straight from the cache, Q quantised per row with
+// its own scale, P stored as E4M3 of 2^4 p).  Every MMA consumes 32 bytes of
+// its K extent per row, so the descriptor arithmetic is shared.
 //
 // Every wait is bounded (ptx.cuh); on a timeout the CTA raises an abort flag,
-// drains its in-flight TMA loads and MMAs, frees TMEM and exits.
+// drains its in-flight TMA loads and MMAs, frees TMEM and exits.  The two
+// softmax warpgroups meet only on mbarriers (bounded waits), never on a
+// named barrier.
 #include <cstdint>
 #include <cuda.h>
 
@@ -64,17 +72,22 @@
 
 namespace qup {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kRows = 128;
 constexpr int kD = kHeadDim;
 constexpr int kST = 128;  // tokens per pipeline step
 constexpr int kTmemCols = 512;
-constexpr int kKProducerWarp = 4, kSWarp = 5, kVProducerWarp = 6, kPvWarp = 7;
-constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kKProducerWarp = 8, kSWarp = 9, kVProducerWarp = 10, kPvWarp = 11;
+constexpr uint32_t kColO = 0, kColS = 256;  // O_w at kColO + 128 w, S_w at kColS + 128 w
+// Register split: the launch gives every thread kLaunchRegs (384 x 168 = 64,512 of the SM's
+// 65,536); the producer and issuer warpgroup gives back down to kOtherRegs and the two softmax
+// warpgroups take kSoftmaxRegs: 256 x 224 + 128 x 56 = 64,512, exactly the launch's total.
+constexpr int kLaunchRegs = 168, kSoftmaxRegs = 224, kOtherRegs = 56;
+static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 
 template <int ES, int T>
 struct Geo {
-    static constexpr int SPP = T > kST ? T / kST : 1;   // steps per page (not used: T <= 128)
     static constexpr int PPS = T < kST ? kST / T : 1;   // pages per step
     static constexpr int BOXR = T < 64 ? T : 64;        // token rows per TMA box
     static constexpr int BPP = T / BOXR;                // boxes per page (along tokens)
@@ -82,14 +95,12 @@ struct Geo {
     static constexpr int kChunkElems = 128 / ES;        // elements per 128-byte swizzle row
     static constexpr int kNChunk = kD * ES / 128;       // 128-byte chunks along d
     static constexpr int kChunkBytes = kST * 128;       // one chunk column of a K or V tile
-    static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of a shared-memory Q tile
+    static constexpr int kQBytes = kRows * kD * ES;     // the Q operand of a bundle
+    static constexpr int kQChunkBytes = kRows * 128;    // one chunk column of the Q operand
     static constexpr int kMmaK = 32 / ES;               // K elements per MMA instruction
     static constexpr int kNumMmaS = kD * ES / 32;       // MMAs per S (K = d)
     static constexpr int kNumMmaPV = kST * ES / 32;     // MMAs per O update (K = 128 tokens)
     static constexpr int kPCols = kST * ES / 4;         // TMEM columns of P
-    static constexpr bool kQTmem = ES != 4;             // Q as the TMEM A operand (bf16, E4M3)
-    static constexpr int kQCols = kD * ES / 4;          // TMEM columns of Q
-    static_assert(!kQTmem || kColQ + 2 * kQCols <= kTmemCols, "TMEM budget (two Q buffers)");
     static_assert(kPCols <= 128, "P fits in its S buffer");
     // exponentials on the FMA pipe by a polynomial: pairs (j / 2) % 8 < kPolyPairs of every 16
     // columns; the rest go to the MUFU unit
@@ -105,29 +116,36 @@ struct Geo {
 };
 
 struct SmemLayout {
-    uint32_t kst, vst, q, qst, sinfo, bars, misc, total;
+    uint32_t kst, vst, q, qst, sinfo, mrg, qsc, bars, misc, total;
 };
 
-// Stage of the next bundle (bf16 Q rows): query slot m holds the g rows of its query, 256 bytes
-// each, at m * qstage_stride(g); the 16-byte pad keeps row reads free of bank conflicts.
+// Stage of the next bundle (E4M3: its bf16 Q rows): query slot m holds the g rows of its query,
+// 256 bytes each, at m * qstage_stride(g); the 16-byte pad keeps row reads free of bank conflicts.
 __host__ __device__ inline uint32_t qstage_stride(int g) { return (uint32_t)g * 256u + 16u; }
-constexpr int kSinfoWords = 8;  // stage header: flat bundle, h, bi, ub, nU, nsteps, ok
+constexpr int kSinfoWords = 8;  // bundle header: flat bundle, h, bi, ub, nU, nsteps, ok
+constexpr int kFixedBars = 14;
 
 __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv, int g) {
     SmemLayout L;
+    const uint32_t MQ = (uint32_t)(kRows / g);
     uint32_t off = 0;
     L.kst = off;
     off += (uint32_t)nsk * kST * kD * es;
     L.vst = off;
     off += (uint32_t)nsv * kST * kD * es;
-    L.q = off;
-    if (es == 4) off += (uint32_t)kRows * kD * es;  // fp32 Q stays in shared memory
+    L.q = off;  // 1024-aligned: every tile above is a multiple of 16 KB
+    off += (uint32_t)kRows * kD * es;
     L.qst = off;
-    if (es != 4) off += (uint32_t)(kRows / g) * qstage_stride(g);
+    if (es == 1) off += MQ * qstage_stride(g);
     L.sinfo = off;
-    off += 4u * (kSinfoWords + 2 * kRows);  // header, qid[128 / g], q_pos[128 / g]
+    off += 4u * (kSinfoWords + 2u * MQ);  // header, qid[MQ], q_pos[MQ]
+    L.mrg = off;
+    off += 2u * kRows * 8u;  // per warpgroup and row: running max and sum (float2)
+    L.qsc = off;
+    if (es == 1) off += 4u * kRows;  // E4M3: per-row score scale of the quantised Q
+    off = (off + 7u) & ~7u;
     L.bars = off;
-    off += 8u * (2u * (nsk + nsv) + 12u);
+    off += 8u * (2u * (nsk + nsv) + kFixedBars);
     L.misc = off;
     off += 16u + 4u * (uint32_t)(Hkv + 1);
     L.total = off + 1024u;  // slack for aligning the dynamic base to 1024
@@ -143,14 +161,17 @@ struct Bars {
     __device__ __forceinline__ uint32_t vfull(int s) const { return base + 8u * (2 * nsk + s); }
     __device__ __forceinline__ uint32_t vempty(int s) const { return base + 8u * (2 * nsk + nsv + s); }
     __device__ __forceinline__ uint32_t fixed(int i) const { return base + 8u * (2 * (nsk + nsv) + i); }
-    __device__ __forceinline__ uint32_t sfull(int i) const { return fixed(i); }
-    __device__ __forceinline__ uint32_t pfull(int i) const { return fixed(2 + i); }
-    __device__ __forceinline__ uint32_t pvdone(int i) const { return fixed(4 + i); }
-    __device__ __forceinline__ uint32_t qfull() const { return fixed(6); }
-    __device__ __forceinline__ uint32_t drain() const { return fixed(7); }
-    __device__ __forceinline__ uint32_t drain2() const { return fixed(8); }
-    __device__ __forceinline__ uint32_t stfull() const { return fixed(9); }
-    __device__ __forceinline__ uint32_t stempty() const { return fixed(10); }
+    __device__ __forceinline__ uint32_t sfull(int w) const { return fixed(w); }       // S_w computed
+    __device__ __forceinline__ uint32_t pfull(int w) const { return fixed(2 + w); }   // P_w stored
+    __device__ __forceinline__ uint32_t pvdone(int w) const { return fixed(4 + w); }  // O_w += P_w V done
+    __device__ __forceinline__ uint32_t qfull() const { return fixed(6); }   // the bundle's Q operand is in place
+    __device__ __forceinline__ uint32_t qfree() const { return fixed(7); }   // every S of the bundle completed
+    __device__ __forceinline__ uint32_t stfull() const { return fixed(8); }  // header (and E4M3 stage) written
+    __device__ __forceinline__ uint32_t stempty() const { return fixed(9); } // header read by every softmax warp
+    __device__ __forceinline__ uint32_t ep1() const { return fixed(10); }    // both row states published
+    __device__ __forceinline__ uint32_t ep2() const { return fixed(11); }    // both halves of O read
+    __device__ __forceinline__ uint32_t drain() const { return fixed(12); }
+    __device__ __forceinline__ uint32_t drain2() const { return fixed(13); }
 };
 
 struct Item {
@@ -212,7 +233,7 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
 template <int ES, int T>
 __global__ void __launch_bounds__(kThreads, 1)
     union_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                      const __grid_constant__ AttnParams p) {
+                      const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ AttnParams p) {
     using G = Geo<ES, T>;
     constexpr int PPS = G::PPS, BOXR = G::BOXR, BPP = G::BPP;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -227,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* nb_prefix = reinterpret_cast<int*>(smem + L.misc + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t lim = p.wait_limit_ns;
+    const int g = p.g, MQ = kRows / g;
 
     // ---------------------------------------------------------------- setup
     // barriers, TMEM and the tensor maps first; the kernel ahead in the stream may
@@ -240,21 +262,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(B.vfull(s), 1);
             mbar_init(B.vempty(s), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(B.sfull(i), 1);
-            mbar_init(B.pfull(i), 4);  // one arrive per softmax warp
-            mbar_init(B.pvdone(i), 1);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(B.sfull(w), 1);
+            mbar_init(B.pfull(w), 4);  // one arrive per warp of softmax warpgroup w
+            mbar_init(B.pvdone(w), 1);
         }
-        mbar_init(B.qfull(), 4);
+        mbar_init(B.qfull(), ES == 2 ? 1 : 4);  // bf16: the TMA transactions; else warpgroup 0's warps
+        mbar_init(B.qfree(), 1);
+        mbar_init(B.stfull(), 1);
+        mbar_init(B.stempty(), kSoftmaxWarps);
+        mbar_init(B.ep1(), kSoftmaxWarps);
+        mbar_init(B.ep2(), kSoftmaxWarps);
         mbar_init(B.drain(), 1);
         mbar_init(B.drain2(), 1);
-        mbar_init(B.stfull(), 1);
-        mbar_init(B.stempty(), 4);  // one arrive per softmax warp
         fence_mbar_init();
         *abort_flag = 0;
     }
     if (threadIdx.x == kKProducerWarp * 32) prefetch_tensormap(&tmK);
-    if (threadIdx.x == kVProducerWarp * 32) prefetch_tensormap(&tmV);
+    if (threadIdx.x == kVProducerWarp * 32) {
+        prefetch_tensormap(&tmV);
+        if constexpr (ES == 2) prefetch_tensormap(&tmQ);
+    }
     if (warp == kSWarp) {
         tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
         tmem_relinquish();
@@ -279,36 +307,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_items = nb_prefix[p.Hkv];
 
-    if (warp == kKProducerWarp || warp == kVProducerWarp) {
-        // ============================================================ producers (whole warp each)
-        // Both walk the same bundles and pages; the K warp fills the K ring, the V warp the
-        // V ring (and stages each bundle for the softmax warps).
-        const bool isV = warp == kVProducerWarp;
-        const int NR = isV ? NSV : NSK;
-        const CUtensorMap* tm = isV ? &tmV : &tmK;
-        const uint32_t ring = sbase + (isV ? L.vst : L.kst);
-        int gs = 0, n_staged = 0;
-        bool ok = true;
-        for (int rnd = 0; ok; ++rnd) {
-            const int f = item_at(p, rnd, n_items);
-            if (f == -1) break;
-            if (f < 0) continue;
-            const Item it = load_item<PPS>(p, nb_prefix, f);
-            if constexpr (ES != 4) {
-                // The V warp stages the bundle for the softmax warps (a few steps before they reach
-                // it): header, query IDs and positions of its query slots, and its Q rows (bulk
-                // copies by original query ID: the g rows of a query are contiguous in Q).
+    if (warp >= kSoftmaxWarps) {
+        regs_decrease<kOtherRegs>();
+        if (warp == kKProducerWarp || warp == kVProducerWarp) {
+            // ======================================================== producers (whole warp each)
+            // Both walk the same bundles and pages; the K warp fills the K ring, the V warp the V
+            // ring, writes each bundle's header and loads (bf16) or stages (E4M3) its Q rows.
+            const bool isV = warp == kVProducerWarp;
+            const int NR = isV ? NSV : NSK;
+            const CUtensorMap* tm = isV ? &tmV : &tmK;
+            const uint32_t ring = sbase + (isV ? L.vst : L.kst);
+            int gs = 0, n_done = 0;
+            bool ok = true;
+            for (int rnd = 0; ok; ++rnd) {
+                const int f = item_at(p, rnd, n_items);
+                if (f == -1) break;
+                if (f < 0) continue;
+                const Item it = load_item<PPS>(p, nb_prefix, f);
                 if (isV) {
-                    if (n_staged > 0) {  // the softmax warps have read the previous stage
+                    // the header, once every softmax warp has read the previous bundle's
+                    if (n_done > 0) {
                         int okv = 0;
                         if (lane == 0)
-                            okv = mbar_wait_idle(B.stempty(), (n_staged - 1) & 1, abort_flag, p.err,
-                                                 QUP_ERR_TIMEOUT, lim);
+                            okv = mbar_wait_idle(B.stempty(), (n_done - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
+                                                 lim);
                         ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
                         if (!ok) break;
                     }
                     int* sinfo = reinterpret_cast<int*>(smem + L.sinfo);
-                    const int MQ = kRows / p.g;
                     int nvalid = 0;
                     for (int m0 = 0; m0 < MQ; m0 += 32) {
                         const int m = m0 + lane;
@@ -321,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             qid = max(qid, -1);
                             sinfo[kSinfoWords + m] = qid;
-                            sinfo[kSinfoWords + kRows + m] = qid >= 0 ? p.q_pos[qid] : -1;
+                            sinfo[kSinfoWords + MQ + m] = qid >= 0 ? p.q_pos[qid] : -1;
                         }
                         nvalid += __popc(__ballot_sync(0xffffffffu, qid >= 0));
                     }
@@ -335,186 +361,252 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sinfo[6] = it.ok ? 1 : 0;
                     }
                     __syncwarp();
-                    const uint32_t qbytes = (uint32_t)p.g * kD * 2u;
-                    if (lane == 0) mbar_arrive_expect_tx(B.stfull(), (uint32_t)nvalid * qbytes);
-                    __syncwarp();
-                    for (int m = lane; m < MQ; m += 32) {
-                        const int qid = sinfo[kSinfoWords + m];
-                        if (qid >= 0)
-                            bulk_g2s(sbase + L.qst + (uint32_t)m * qstage_stride(p.g),
-                                     static_cast<const uint16_t*>(p.Q) + ((size_t)qid * p.Hq + (size_t)it.h * p.g) * kD,
-                                     qbytes, B.stfull());
-                    }
-                    ++n_staged;
-                }
-            }
-            const int n_ent = it.nsteps * PPS;  // incl. padding of the last step
-            for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
-                const int idx = e0 + lane;
-                int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
-                if (idx < it.nU) {
-                    u = p.union_pages[it.ub + idx];
-                    if (u < 0 || u >= p.num_logical_pages) {
-                        atomicOr(p.err, QUP_ERR_PAGE_ID);
-                        u = 0;
+                    if constexpr (ES == 1) {
+                        // the bf16 Q rows, by query ID (the g rows of a query are contiguous in Q)
+                        const uint32_t qbytes = (uint32_t)g * kD * 2u;
+                        if (lane == 0) mbar_arrive_expect_tx(B.stfull(), (uint32_t)nvalid * qbytes);
+                        __syncwarp();
+                        for (int m = lane; m < MQ; m += 32) {
+                            const int qid = sinfo[kSinfoWords + m];
+                            if (qid >= 0)
+                                bulk_g2s(sbase + L.qst + (uint32_t)m * qstage_stride(g),
+                                         static_cast<const uint16_t*>(p.Q) + ((size_t)qid * p.Hq + (size_t)it.h * g) * kD,
+                                         qbytes, B.stfull());
+                        }
                     } else {
-                        phys = p.page_table[u];
-                        if (phys < 0 || phys >= p.P_phys) {
-                            atomicOr(p.err, QUP_ERR_PHYS_PAGE);
-                            phys = p.P_phys;
+                        if (lane == 0) mbar_arrive(B.stfull());
+                    }
+                    if constexpr (ES == 2) {
+                        // the Q operand by TMA, once every S of the previous bundle has completed: per
+                        // query slot and half of d one box of g rows; an empty slot reads zeros from
+                        // outside the tensor
+                        if (n_done > 0) {
+                            int okv = 0;
+                            if (lane == 0)
+                                okv = mbar_wait_idle(B.qfree(), (n_done - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT,
+                                                     lim);
+                            ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
+                            if (!ok) break;
+                        }
+                        if (lane == 0) mbar_arrive_expect_tx(B.qfull(), (uint32_t)G::kQBytes);
+                        __syncwarp();
+                        for (int m = lane; m < MQ; m += 32) {
+                            const int qid = sinfo[kSinfoWords + m];
+                            const int qc = qid >= 0 ? qid : p.Nq;
+#pragma unroll
+                            for (int kb = 0; kb < 2; ++kb)
+                                tma_load_3d(sbase + L.q + (uint32_t)kb * G::kQChunkBytes + (uint32_t)(m * g) * 128u, &tmQ,
+                                            B.qfull(), kb * 64, it.h * g, qc);
                         }
                     }
+                    ++n_done;
                 }
-                const int nst = min(32, n_ent - e0) / PPS;  // 32 is a multiple of PPS
-                for (int k = 0; k < nst; ++k, ++gs) {
-                    const int slot = gs % NR;
-                    int okv = 0;
-                    if (lane == 0)
-                        okv = mbar_wait_idle(isV ? B.vempty(slot) : B.kempty(slot), ((gs / NR) & 1) ^ 1, abort_flag,
-                                        p.err, QUP_ERR_TIMEOUT, lim);
-                    ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
-                    if (!ok) break;
-                    const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
-                                                      gs == p.dbg_skip_stage);
-                    int ph[PPS];
-#pragma unroll
-                    for (int q = 0; q < PPS; ++q) {
-                        const int src = k * PPS + q;
-                        ph[q] = __shfl_sync(0xffffffffu, phys, src);
+                const int n_ent = it.nsteps * PPS;  // incl. padding of the last step
+                for (int e0 = 0; e0 < n_ent && ok; e0 += 32) {
+                    const int idx = e0 + lane;
+                    int u = 0, phys = p.P_phys;  // P_phys: outside the tensor, TMA fills zeros
+                    if (idx < it.nU) {
+                        u = p.union_pages[it.ub + idx];
+                        if (u < 0 || u >= p.num_logical_pages) {
+                            atomicOr(p.err, QUP_ERR_PAGE_ID);
+                            u = 0;
+                        } else {
+                            phys = p.page_table[u];
+                            if (phys < 0 || phys >= p.P_phys) {
+                                atomicOr(p.err, QUP_ERR_PHYS_PAGE);
+                                phys = p.P_phys;
+                            }
+                        }
                     }
-                    if (issue) {
-                        const uint32_t fb = isV ? B.vfull(slot) : B.kfull(slot);
-                        mbar_arrive_expect_tx(fb, G::kTile);
-                        const uint32_t dst = ring + (uint32_t)slot * G::kTile;
+                    const int nst = min(32, n_ent - e0) / PPS;  // 32 is a multiple of PPS
+                    for (int k = 0; k < nst; ++k, ++gs) {
+                        const int slot = gs % NR;
+                        int okv = 0;
+                        if (lane == 0)
+                            okv = mbar_wait_idle(isV ? B.vempty(slot) : B.kempty(slot), ((gs / NR) & 1) ^ 1,
+                                                 abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
+                        ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
+                        if (!ok) break;
+                        const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
+                                                          gs == p.dbg_skip_stage);
+                        int ph[PPS];
 #pragma unroll
-                        for (int q = 0; q < PPS; ++q) {
+                        for (int q = 0; q < PPS; ++q) ph[q] = __shfl_sync(0xffffffffu, phys, k * PPS + q);
+                        if (issue) {
+                            const uint32_t fb = isV ? B.vfull(slot) : B.kfull(slot);
+                            mbar_arrive_expect_tx(fb, G::kTile);
+                            const uint32_t dst = ring + (uint32_t)slot * G::kTile;
 #pragma unroll
-                            for (int bb = 0; bb < BPP; ++bb) {
+                            for (int q = 0; q < PPS; ++q) {
 #pragma unroll
-                                for (int c = 0; c < G::kNChunk; ++c) {
-                                    const uint32_t off =
-                                        (uint32_t)c * G::kChunkBytes + (uint32_t)(q * T + bb * BOXR) * 128u;
-                                    tma_load_4d(dst + off, tm, fb, c * G::kChunkElems, bb * BOXR, it.h, ph[q]);
+                                for (int bb = 0; bb < BPP; ++bb) {
+#pragma unroll
+                                    for (int c = 0; c < G::kNChunk; ++c) {
+                                        const uint32_t off =
+                                            (uint32_t)c * G::kChunkBytes + (uint32_t)(q * T + bb * BOXR) * 128u;
+                                        tma_load_4d(dst + off, tm, fb, c * G::kChunkElems, bb * BOXR, it.h, ph[q]);
+                                    }
                                 }
                             }
                         }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
-        }
-        // every issued load lands before the CTA may exit: the last NR stages of this ring, and
-        // the last stage of Q rows
-        if (lane == 0) {
-            if (n_staged > 0) mbar_wait_drain(B.stfull(), (n_staged - 1) & 1, lim);
-            for (int i = max(0, gs - NR); i < gs; ++i) {
-                if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
-                mbar_wait_drain(isV ? B.vfull(i % NR) : B.kfull(i % NR), (i / NR) & 1, lim);
+            // every issued load lands before the CTA may exit: the last NR stages of this ring,
+            // and the last bundle's staged or loaded Q rows
+            if (lane == 0) {
+                if (isV && n_done > 0) {
+                    if constexpr (ES == 1) mbar_wait_drain(B.stfull(), (n_done - 1) & 1, lim);
+                    if constexpr (ES == 2) mbar_wait_drain(B.qfull(), (n_done - 1) & 1, lim);
+                }
+                for (int i = max(0, gs - NR); i < gs; ++i) {
+                    if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
+                    mbar_wait_drain(isV ? B.vfull(i % NR) : B.kfull(i % NR), (i / NR) & 1, lim);
+                }
             }
-        }
-        __syncwarp();
-    } else if (warp == kSWarp || warp == kPvWarp) {
-        // ============================================================ MMA issuers (whole warp, one elected lane)
-        //   S warp:  S(g) = Q K^T into S_b: needs K tile g, and the O update of step g - 2
-        //            (which read P from S_b) finished; commits S-full(b) and the K slot.
-        //   PV warp: O += P_b V: needs P(g) and V tile g; commits PV-done(b) and the V slot.
-        // The PV warp needs no Q barrier: P(g) of a bundle's first step is written after the
-        // softmax warps have finished the previous bundle's epilogue (its reads of O).
-        const bool isS = warp == kSWarp;
-        const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, kST, kRows);
-        const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
-        // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
-        // has only the 128-byte swizzle with 32-byte atoms (layout 1, 4-row atoms)
-        constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
-        constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
-        const uint32_t qbase = sbase + L.q;
-        int gs = 0, item_no = 0;
-        int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slot and phase of step gs
-        bool ok = true;
-        for (int rnd = 0; ok; ++rnd) {
-            const int f = item_at(p, rnd, n_items);
-            if (f == -1) break;
-            if (f < 0) continue;
-            const Item it = load_item<PPS>(p, nb_prefix, f);
-            if (isS) {
-                ok = warp_ok(mbar_wait_idle(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-                if (!ok) break;
-                tc_fence_after();
-                for (int s = 0; s < it.nsteps; ++s) {
-                    const int g = gs + s, b = g & 1;
-                    ok = warp_ok(mbar_wait_idle(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 (g < 2 || mbar_wait_idle(B.pvdone(b), ((g - 2) >> 1) & 1, abort_flag, p.err,
-                                                     QUP_ERR_TIMEOUT, lim)));
+            __syncwarp();
+        } else {
+            // ======================================================== MMA issuers (whole warp, one elected lane)
+            //   S warp:  S_w = Q K^T for step s (w = s % 2): needs the bundle's Q operand, K tile s,
+            //            and the O update that last read P from S_w finished; commits S-full(w) and
+            //            the K slot, and after the bundle's last S the Q-free barrier.
+            //   PV warp: O_w += P_w V: needs P(s) and V tile s; commits PV-done(w) and the V slot.
+            // The first O update of each accumulator in a bundle overwrites it; its P is stored
+            // after both warpgroups have read the previous bundle's O (the epilogue's barrier).
+            const bool isS = warp == kSWarp;
+            const uint32_t idesc_s = instr_desc(G::kFmt, 0, 0, kST, kRows);
+            const uint32_t idesc_o = instr_desc(G::kFmt, 0, 1, kD, kRows);
+            // V as the MN-major B operand (N = d): 128-byte swizzle with 8-row atoms; tf32
+            // has only the 128-byte swizzle with 32-byte atoms (layout 1, 4-row atoms)
+            constexpr uint32_t vlayout = ES == 4 ? 1u : 2u;
+            constexpr uint32_t vsbo = ES == 4 ? 512u : 1024u;
+            const uint64_t qdesc = smem_desc(sbase + L.q, 16, 1024, 2);
+            int use[2] = {0, 0}, item_no = 0;
+            int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slot and phase of the next step
+            bool ok = true;
+            for (int rnd = 0; ok; ++rnd) {
+                const int f = item_at(p, rnd, n_items);
+                if (f == -1) break;
+                if (f < 0) continue;
+                const Item it = load_item<PPS>(p, nb_prefix, f);
+                if (isS) {
+                    ok = warp_ok(mbar_wait_idle(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t kdesc = smem_desc(sbase + L.kst + (uint32_t)ks * G::kTile, 16, 1024, 2);
-                    const uint64_t qdesc = smem_desc(qbase, 16, 1024, 2);
-                    if (elect_one_sync()) {
+                    for (int s = 0; s < it.nsteps; ++s) {
+                        const int w = s & 1, k = use[w];
+                        ok = warp_ok(mbar_wait_idle(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                     (k < 1 || mbar_wait_idle(B.pvdone(w), (k - 1) & 1, abort_flag, p.err,
+                                                              QUP_ERR_TIMEOUT, lim)));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t kdesc = smem_desc(sbase + L.kst + (uint32_t)ks * G::kTile, 16, 1024, 2);
+                        if (elect_one_sync()) {
 #pragma unroll
-                        for (int k = 0; k < G::kNumMmaS; ++k) {
-                            const uint32_t koff = ((k >> 2) * G::kChunkBytes + (k & 3) * 32) >> 4;
-                            if constexpr (G::kQTmem) {
-                                tc_mma_ts<G::kKind>(tmem + kColS + 128u * b,
-                                                    tmem + kColQ + (uint32_t)(item_no & 1) * G::kQCols + 8u * k, kdesc + koff,
-                                                    idesc_s, k > 0);
-                            } else {
-                                const uint32_t qoff = ((k >> 2) * G::kQChunkBytes + (k & 3) * 32) >> 4;
-                                tc_mma<G::kKind>(tmem + kColS + 128u * b, qdesc + qoff, kdesc + koff, idesc_s, k > 0);
+                            for (int kk = 0; kk < G::kNumMmaS; ++kk) {
+                                const uint32_t koff = ((kk >> 2) * G::kChunkBytes + (kk & 3) * 32) >> 4;
+                                const uint32_t qoff = ((kk >> 2) * G::kQChunkBytes + (kk & 3) * 32) >> 4;
+                                tc_mma<G::kKind>(tmem + kColS + 128u * w, qdesc + qoff, kdesc + koff, idesc_s, kk > 0);
                             }
+                            tc_commit(B.sfull(w));
+                            tc_commit(B.kempty(ks));
                         }
-                        tc_commit(B.sfull(b));
-                        tc_commit(B.kempty(ks));
+                        __syncwarp();
+                        ++use[w];
+                        if (++ks == NSK) {
+                            ks = 0;
+                            kph ^= 1;
+                        }
                     }
-                    __syncwarp();
-                    if (++ks == NSK) {
-                        ks = 0;
-                        kph ^= 1;
-                    }
-                }
-            } else {
-                for (int s = 0; s < it.nsteps; ++s) {
-                    const int g = gs + s, b = g & 1;
-                    ok = warp_ok(mbar_wait_idle(B.pfull(b), (g >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                 mbar_wait_idle(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                     if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
-                                                     (uint32_t)G::kChunkBytes, vsbo, vlayout);
-                    if (elect_one_sync()) {
-#pragma unroll
-                        for (int k = 0; k < G::kNumMmaPV; ++k) {
-                            // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
-                            tc_mma_ts<G::kKind>(tmem + kColO, tmem + kColS + 128u * b + 8u * k,
-                                                vdesc + ((k * G::kMmaK * 128) >> 4), idesc_o, s > 0 || k > 0);
-                        }
-                        tc_commit(B.pvdone(b));
-                        tc_commit(B.vempty(vs));
-                    }
+                    if (elect_one_sync()) tc_commit(B.qfree());
                     __syncwarp();
-                    if (++vs == NSV) {
-                        vs = 0;
-                        vph ^= 1;
+                } else {
+                    // The bundle's union entries, 32 at a time (lane j: entry cb + j); a page that
+                    // reaches past kv_len may hold non-finite bytes there: its V rows past kv_len
+                    // are zeroed before the O update reads the tile (P is 0 there, but 0 * NaN is not)
+                    int cb = -32, cpg = -1;
+                    for (int s = 0; s < it.nsteps; ++s) {
+                        const int w = s & 1, k = use[w];
+                        const int e0 = s * PPS;
+                        if (e0 >= cb + 32) {
+                            cb = e0 - (e0 & 31);
+                            const int e = cb + lane;
+                            cpg = e < it.nU ? p.union_pages[it.ub + e] : -1;
+                            if (cpg >= p.num_logical_pages) cpg = -1;
+                        }
+                        bool tail = false;
+#pragma unroll
+                        for (int q = 0; q < PPS; ++q) {
+                            const int pg = __shfl_sync(0xffffffffu, cpg, e0 - cb + q);
+                            tail |= pg >= 0 && pg * T + T > p.kv_len;
+                        }
+                        ok = warp_ok(mbar_wait_idle(B.pfull(w), k & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
+                                     mbar_wait_idle(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                        if (!ok) break;
+                        if (tail) {
+                            uint8_t* vt = smem + L.vst + (uint32_t)vs * G::kTile;
+#pragma unroll 1
+                            for (int q = 0; q < PPS; ++q) {
+                                const int pg = __shfl_sync(0xffffffffu, cpg, e0 - cb + q);
+                                if (pg < 0 || pg * T + T <= p.kv_len) continue;
+                                const int t0 = max(0, p.kv_len - pg * T);  // first token row past kv_len
+                                const int nwords = (T - t0) * G::kNChunk * 8;  // 16-byte words to clear
+                                for (int i = lane; i < nwords; i += 32) {
+                                    const int row = q * T + t0 + i / (G::kNChunk * 8);
+                                    const int rest = i % (G::kNChunk * 8);
+                                    *reinterpret_cast<uint4*>(vt + (rest >> 3) * G::kChunkBytes + row * 128 +
+                                                              (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
+                                }
+                            }
+                            fence_proxy_async_smem();  // zeroed rows -> the tensor core
+                            __syncwarp();
+                        }
+                        tc_fence_after();
+                        const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
+                                                         (uint32_t)G::kChunkBytes, vsbo, vlayout);
+                        if (elect_one_sync()) {
+#pragma unroll
+                            for (int kk = 0; kk < G::kNumMmaPV; ++kk) {
+                                // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
+                                tc_mma_ts<G::kKind>(tmem + kColO + 128u * w, tmem + kColS + 128u * w + 8u * kk,
+                                                    vdesc + ((kk * G::kMmaK * 128) >> 4), idesc_o, s >= 2 || kk > 0);
+                            }
+                            tc_commit(B.pvdone(w));
+                            tc_commit(B.vempty(vs));
+                        }
+                        __syncwarp();
+                        ++use[w];
+                        if (++vs == NSV) {
+                            vs = 0;
+                            vph ^= 1;
+                        }
                     }
                 }
+                ++item_no;
             }
-            gs += it.nsteps;
-            ++item_no;
+            // every MMA this warp issued completes before TMEM is freed
+            const uint32_t dbar = isS ? B.drain() : B.drain2();
+            if (elect_one_sync()) tc_commit(dbar);
+            __syncwarp();
+            mbar_wait_drain(dbar, 0, lim);
+            __syncwarp();
         }
-        // every MMA this warp issued completes before TMEM is freed
-        const uint32_t dbar = isS ? B.drain() : B.drain2();
-        if (elect_one_sync()) tc_commit(dbar);
-        __syncwarp();
-        mbar_wait_drain(dbar, 0, lim);
-        __syncwarp();
     } else {
-        // ============================================================ softmax / epilogue (warps 0-3)
-        const int r = warp * 32 + lane;  // bundle row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        regs_increase<kSoftmaxRegs>();
+        // ============================================================ softmax / epilogue (warps 0-7)
+        const int w = warp >> 2;          // warpgroup: the steps s with s % 2 == w
+        const int wq = warp & 3;          // TMEM lane quarter of this warp
+        const int r = wq * 32 + lane;     // bundle row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const uint32_t colS = kColS + 128u * w, colO = kColO + 128u * w;
         const float kNegInf = -__int_as_float(0x7f800000);
         const float kPosInf = __int_as_float(0x7f800000);
-        const int g = p.g, MQ = kRows / g;
         const int* sinfo = reinterpret_cast<const int*>(smem + L.sinfo);
-        int gs = 0, vs = 0, vph = 0;
+        float2* mrg = reinterpret_cast<float2*>(smem + L.mrg);  // [2][kRows]
+        float* qsc = reinterpret_cast<float*>(smem + L.qsc);
+        int use = 0;  // this warpgroup's uses of S_w and O_w so far
         bool ok = true;
         // the row's bundle state: item, query (original ID), Q head, visible positions, score scale
         Item it{};
@@ -534,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mk = 0u;
             if (e < it.nU) {
                 const int u = p.union_pages[it.ub + e];
-                const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + warp];
+                const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + wq];
                 if (u >= 0 && u < p.num_logical_pages) {
                     const int ph = p.page_table[u];
                     if (ph >= 0 && ph < p.P_phys) {
@@ -544,32 +636,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        // Take over flat bundle ff, the ino-th of this CTA: its header and this row's query
-        // (bf16 Q: from the stage the V warp filled; fp32 Q: from global memory), the first union
-        // entries, and this row of Q by original query ID into the bundle's TMEM Q buffer (fp32:
-        // the shared-memory Q tile).  Arrives on the Q barrier (and releases the stage).
-        auto take = [&](int ff, int ino) -> bool {
-            int qpos = -1;
-            if constexpr (ES != 4) {
-                if (!warp_ok(mbar_wait(B.stfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
-                it.h = sinfo[1];
-                it.bi = sinfo[2];
-                it.ub = sinfo[3];
-                it.nU = sinfo[4];
-                it.nsteps = sinfo[5];
-                it.ok = sinfo[6] != 0;
-                qid = sinfo[kSinfoWords + r / g];
-                qpos = sinfo[kSinfoWords + kRows + r / g];
-            } else {
-                it = load_item<PPS>(p, nb_prefix, ff);
-                qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + r / g];
-                if (qid >= p.Nq) {
-                    atomicOr(p.err, QUP_ERR_GROUP);
-                    qid = -1;
-                }
-                qid = max(qid, -1);
-                qpos = qid >= 0 ? p.q_pos[qid] : -1;
-            }
+        // Take over the ino-th bundle of this CTA from the header the V warp wrote: its item, this
+        // row's query (original ID) and position, the first union entries.  Warpgroup 0 writes
+        // the Q operand for the non-bf16 types (E4M3: quantised per row from the staged bf16
+        // rows; fp32: from global memory) once every S of the previous bundle has completed;
+        // E4M3 warpgroup 1 then reads its rows' score scales.  Releases the header.
+        auto take = [&](int ino) -> bool {
+            if (!warp_ok(mbar_wait(B.stfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
+            it.h = sinfo[1];
+            it.bi = sinfo[2];
+            it.ub = sinfo[3];
+            it.nU = sinfo[4];
+            it.nsteps = sinfo[5];
+            it.ok = sinfo[6] != 0;
+            qid = sinfo[kSinfoWords + r / g];
+            const int qpos = sinfo[kSinfoWords + MQ + r / g];
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             head = it.h * g + (r % g);
             vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
@@ -577,73 +658,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             cbase = 0;
             fetch(0, cpage, cmask);
             fetch(32, npage, nmask);
-            const uint32_t qcol = kColQ + (uint32_t)(ino & 1) * G::kQCols;
-            if constexpr (ES == 2) {
-                const uint8_t* row = smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
+            if constexpr (ES != 2) {
+                if (w == 0) {
+                    if (ino > 0 &&
+                        !warp_ok(mbar_wait(B.qfree(), (ino - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim)))
+                        return false;
+                    uint8_t* qt = smem + L.q;
+                    if constexpr (ES == 4) {
+                        const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t qv[32];
+                        for (int c = 0; c < 32; ++c) {
+                            const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
+                        }
+                    } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
+                        const uint8_t* row =
+                            smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
+                        uint4 raw[16];
+                        float amax = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v =
-                            qid >= 0 ? *reinterpret_cast<const uint4*>(row + half * 128 + c * 16) : make_uint4(0, 0, 0, 0);
-                        qv[4 * c] = v.x;
-                        qv[4 * c + 1] = v.y;
-                        qv[4 * c + 2] = v.z;
-                        qv[4 * c + 3] = v.w;
+                        for (int c = 0; c < 16; ++c) {
+                            raw[c] = qid >= 0 ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0, 0, 0, 0);
+                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                                         fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+                        }
+                        const float inv = amax > 0.f ? 448.f / amax : 0.f;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {  // 16 bf16 -> 16 E4M3 (one 16-byte chunk)
+                            uint32_t qv[4];
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint4 v = raw[2 * c + hh];
+                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                                float x[8];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
+                                    x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
+                                }
+                                qv[2 * hh] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                                qv[2 * hh + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                            }
+                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) =
+                                make_uint4(qv[0], qv[1], qv[2], qv[3]);
+                        }
+                        cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
+                        qsc[r] = cs;
                     }
-                    tmem_st_x32(tmem + lane_base + qcol + 32u * half, qv);
+                    fence_proxy_async_smem();  // generic-proxy writes of Q -> the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(B.qfull());
+                } else if constexpr (ES == 1) {
+                    if (!warp_ok(mbar_wait(B.qfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
+                    cs = qsc[r];
                 }
-            } else if constexpr (ES == 4) {
-                uint8_t* qt = smem + L.q;
-                const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
-                const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
-                }
-                fence_proxy_async_smem();
-            } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
-                const uint8_t* row = smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
-                uint4 raw[16];
-                float amax = 0.f;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    raw[c] = qid >= 0 ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0, 0, 0, 0);
-                    const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
-                                                 fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
-                }
-                const float inv = amax > 0.f ? 448.f / amax : 0.f;
-                uint32_t qv[32];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {  // 8 bf16 -> 8 E4M3 (2 columns)
-                    const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
-                        x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
-                    }
-                    qv[2 * c] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-                    qv[2 * c + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
-                }
-                tmem_st_x32(tmem + lane_base + qcol, qv);
-                cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
             }
-            if constexpr (G::kQTmem) tmem_wait_st();
             // a Q row of zeros (E4M3 scale 0) keeps a positive score scale: its scores are 0 anyway
             cs = fmaxf(cs, 1e-30f);
             cs2 = f2{cs, cs};
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(B.qfull());
-                if constexpr (ES != 4) mbar_arrive(B.stempty());
-            }
+            if (lane == 0) mbar_arrive(B.stempty());
             return true;
         };
         // the walk of bundles: -1 past the end; order entries that are bad are reported and skipped
@@ -659,14 +737,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // and their sum
         uint32_t sv[kST];
         uint32_t pk[ES == 4 ? 1 : G::kPCols];
-        auto exps = [&](const int (&lim)[PPS]) -> float {
+        auto exps = [&](const int (&lim_q)[PPS]) -> float {
             const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
             f2 part[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
             f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token column
 #pragma unroll
             for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
                 // a page the row did not select gets an infinite offset: 2^-inf = 0
-                const float off = lim[q] == 0 ? kPosInf : mb;
+                const float off = lim_q[q] == 0 ? kPosInf : mb;
                 const f2 noff{-off, -off};
 #pragma unroll
                 for (int j = q * T; j < (q + 1) * T; j += 2) {
@@ -698,23 +776,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         int rnd = 0, item_no = 0;
         int f = walk(rnd);
-        if (f >= 0) ok = take(f, 0);
+        if (f >= 0) ok = take(0);
         while (f >= 0 && ok) {
             // the next bundle's flat index: loaded now, used after this bundle's steps
             int rnd2 = rnd + 1;
             const int f2raw = item_at(p, rnd2, n_items);
             m_used = kNegInf;
             lsum = 0.f;
-            for (int s = 0; s < it.nsteps; ++s) {
-                const int gstep = gs + s, b = gstep & 1, slot = vs;
-                const int vphase = vph;
-                if (++vs == NSV) {
-                    vs = 0;
-                    vph ^= 1;
-                }
+            for (int s = w; s < it.nsteps; s += 2) {
+                const int k = use++;
                 // this step's pages and mask words (PPS divides 32: a step never spans two batches)
                 const int e0 = s * PPS;
-                if (e0 >= cbase + 32) {
+                while (e0 >= cbase + 32) {
                     cbase += 32;
                     cpage = npage;
                     cmask = nmask;
@@ -722,7 +795,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // row r sees token t of page q iff the page is in its own TopK row (its bit of the
                 // page's mask) and the token's position is < vis_end; a page that reaches kv_len
-                // may hold non-finite bytes past it (a tail step)
+                // may hold non-finite bytes past it (a tail step: its scores there become -inf
+                // here, its V rows there are zeroed by the PV warp)
                 int lim_q[PPS];
                 bool live = false, partial = false, tail = false;
 #pragma unroll
@@ -735,25 +809,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     partial |= lim_q[q] > 0 && lim_q[q] < T;
                     tail |= pg >= 0 && pg * T + T > p.kv_len;
                 }
-                if (ok) ok = warp_ok(mbar_wait(B.sfull(b), (gstep >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-                if (ok && tail) ok = warp_ok(mbar_wait(B.vfull(slot), vphase, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-                if (!ok) continue;
+                ok = warp_ok(mbar_wait(B.sfull(w), k & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t s_addr = tmem + lane_base + kColS + 128u * b;
+                const uint32_t s_addr = tmem + lane_base + colS;
                 tmem_ld128_wait(s_addr, sv);
-                if (tail) {  // thread r zeroes V token row r of the step if it lies past kv_len
-                    const int q = r / T;
-                    const int pg = __shfl_sync(0xffffffffu, cpage, e0 - cbase + q);
-                    if (pg >= 0 && pg * T + (r - q * T) >= p.kv_len) {
-                        uint8_t* vt = smem + L.vst + (uint32_t)slot * G::kTile;
-#pragma unroll
-                        for (int c = 0; c < G::kNChunk; ++c)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                *reinterpret_cast<uint4*>(vt + c * G::kChunkBytes + r * 128 + e * 16) =
-                                    make_uint4(0, 0, 0, 0);
-                    }
-                }
                 const bool warp_live = __any_sync(0xffffffffu, live);
                 // Raw scores of unseen tokens (past the row's causal limit or kv_len inside a page
                 // it selected) become -inf; pages the row did not select get an infinite offset in
@@ -775,8 +835,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int j = q * T; j < (q + 1) * T; j += 8) {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                mx[k] = max3f(mx[k], __uint_as_float(sv[j + 2 * k]), __uint_as_float(sv[j + 2 * k + 1]));
+                            for (int kk = 0; kk < 4; ++kk)
+                                mx[kk] = max3f(mx[kk], __uint_as_float(sv[j + 2 * kk]), __uint_as_float(sv[j + 2 * kk + 1]));
                         }
                         const float mq = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                         if (lim_q[q] > 0) mloc = fmaxf(mloc, mq * cs);
@@ -798,19 +858,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
                     }
                 }
-                // O is rescaled only after every earlier O update has finished (rare)
-                if (s > 0 && __any_sync(0xffffffffu, need)) {
-                    const int pg = gstep - 1;
-                    ok = warp_ok(mbar_wait(B.pvdone(pg & 1), (pg >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-                    if (!ok) continue;
+                // O_w is rescaled only after its previous update has finished (rare); the first
+                // update of O_w in a bundle overwrites it
+                if (s >= 2 && __any_sync(0xffffffffu, need)) {
+                    ok = warp_ok(mbar_wait(B.pvdone(w), (k - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+                    if (!ok) break;
                     tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t ov[32];
-                        tmem_ld32_wait(tmem + lane_base + kColO + 32u * c, ov);
+                        tmem_ld32_wait(tmem + lane_base + colO + 32u * c, ov);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        tmem_st_x32(tmem + lane_base + kColO + 32u * c, ov);
+                        tmem_st_x32(tmem + lane_base + colO + 32u * c, ov);
                     }
                 }
                 // P over the S buffer it came from (every column of S is in registers)
@@ -820,68 +880,92 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_n<G::kPCols>(s_addr, pk);
                 }
                 tmem_wait_st();
-                if (tail) fence_proxy_async_smem();  // zeroed V rows -> async proxy
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(B.pfull(b));
+                if (lane == 0) mbar_arrive(B.pfull(w));
             }
-            gs += it.nsteps;
+            if (!ok) break;
             const Item it_cur = it;
             const int qid_cur = qid, head_cur = head;
             const float lsum_cur = lsum, m_cur = m_used;
-            // The next bundle takes the other Q buffer before this bundle's epilogue, so its first
-            // S = Q K^T runs while the epilogue reads O.
-            int f2 = f2raw;
-            while (f2 == -2) {
+            const int k_last = use - 1;
+            const int n0 = (it_cur.nsteps + 1) / 2, n1 = it_cur.nsteps / 2;  // steps of each warpgroup
+            // The next bundle's header (and Q operand) is taken before this bundle's epilogue, so
+            // its first S = Q K^T runs while the epilogue reads O.
+            int fn = f2raw;
+            while (fn == -2) {
                 if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
-                f2 = item_at(p, ++rnd2, n_items);
+                fn = item_at(p, ++rnd2, n_items);
             }
-            if (ok && f2 >= 0) ok = take(f2, item_no + 1);
-            // ---- epilogue: O / l -> O[qid][head][:]
-            if (ok && it_cur.nsteps > 0) {
-                const int last = gs - 1;
-                ok = warp_ok(mbar_wait(B.pvdone(last & 1), (last >> 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
-            }
+            if (fn >= 0) ok = take(item_no + 1);
+            if (!ok) break;
+            // ---- epilogue: merge the two warpgroups' partial rows, O / l -> O[qid][head][:]
+            if ((w == 0 ? n0 : n1) > 0)
+                ok = warp_ok(mbar_wait(B.pvdone(w), k_last & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+            if (!ok) break;
+            mrg[w * kRows + r] = make_float2(m_cur, lsum_cur);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(B.ep1());
+            ok = warp_ok(mbar_wait(B.ep1(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
             if (!ok) break;
             tc_fence_after();
+            const float2 other = mrg[(1 - w) * kRows + r];
+            const float m0 = w == 0 ? m_cur : other.x, l0 = w == 0 ? lsum_cur : other.y;
+            const float m1 = w == 0 ? other.x : m_cur, l1 = w == 0 ? other.y : lsum_cur;
+            const float mm = fmaxf(l0 > 0.f ? m0 : kNegInf, l1 > 0.f ? m1 : kNegInf);
+            const float f0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, f1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+            const float ltot = l0 * f0 + l1 * f1;
             float vsc = 1.f;
             if constexpr (ES == 1) vsc = p.v_scale[it_cur.h];
-            const float inv = lsum_cur > 0.f ? vsc / lsum_cur : 0.f;
+            const float inv = ltot > 0.f ? vsc / ltot : 0.f;
+            const float a0 = f0 * inv, a1 = f1 * inv;
             const size_t oi = ((size_t)(qid_cur >= 0 ? qid_cur : 0) * p.Hq + head_cur) * kD;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t ov[32];
-                if (it_cur.nsteps > 0) {
-                    tmem_ld32_wait(tmem + lane_base + kColO + 32u * c, ov);
+            for (int c = 0; c < 2; ++c) {  // this warpgroup's half of the columns
+                const uint32_t col = 64u * w + 32u * c;
+                uint32_t o0[32], o1[32];
+                if (n0 > 0) {
+                    tmem_ld32_wait(tmem + lane_base + kColO + col, o0);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = 0u;
+                    for (int e = 0; e < 32; ++e) o0[e] = 0u;
                 }
+                if (n1 > 0) {
+                    tmem_ld32_wait(tmem + lane_base + kColO + 128u + col, o1);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o1[e] = 0u;
+                }
+                float ov[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o0[e]) * a0 + __uint_as_float(o1[e]) * a1;
                 if (qid_cur >= 0) {
                     if constexpr (ES == 4) {
-                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi + 32 * c);
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi + col);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                                 __uint_as_float(ov[4 * e + 2]) * inv,
-                                                 __uint_as_float(ov[4 * e + 3]) * inv);
+                        for (int e = 0; e < 8; ++e) dst[e] = make_float4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
                     } else {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + oi + 32 * c);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.O) + oi + col);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(
-                                pack_bf16x2(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
+                            dst[e] = make_uint4(pack_bf16x2(ov[8 * e], ov[8 * e + 1]), pack_bf16x2(ov[8 * e + 2], ov[8 * e + 3]),
+                                                pack_bf16x2(ov[8 * e + 4], ov[8 * e + 5]),
+                                                pack_bf16x2(ov[8 * e + 6], ov[8 * e + 7]));
                     }
                 }
             }
-            if (qid_cur >= 0 && p.lse != nullptr)
+            if (w == 0 && qid_cur >= 0 && p.lse != nullptr)
                 p.lse[(size_t)qid_cur * p.Hq + head_cur] =
-                    lsum_cur > 0.f ? (m_cur + __log2f(lsum_cur) - G::kPLog2) * 0.69314718055994531f : kNegInf;
+                    ltot > 0.f ? (mm + __log2f(ltot) - G::kPLog2) * 0.69314718055994531f : kNegInf;
+            // neither accumulator is overwritten by the next bundle before both warpgroups read it
             tc_fence_before();
-            f = f2;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(B.ep2());
+            ok = warp_ok(mbar_wait(B.ep2(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
+            if (!ok) break;
+            tc_fence_after();
+            f = fn;
             rnd = rnd2;
             ++item_no;
         }
@@ -899,11 +983,19 @@ size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g) { return smem_l
 size_t attn_tile_bytes(int es) { return (size_t)kST * kD * es; }
 
 template <int ES, int T>
-static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p, int grid,
-                            size_t smem, cudaStream_t stream) {
+static cudaError_t launch_t(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                            const AttnParams& p, int grid, size_t smem, cudaStream_t stream) {
+    // The register split (setmaxnreg) is sized for kLaunchRegs per thread at launch: a kernel
+    // built with another count is not launched (an increase beyond the launch's registers would
+    // never be granted).
+    static const int regs = [] {
+        cudaFuncAttributes a;
+        return cudaFuncGetAttributes(&a, (const void*)union_attn_kernel<ES, T>) == cudaSuccess ? a.numRegs : -1;
+    }();
+    if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     cudaError_t e = ensure_smem_attr((const void*)union_attn_kernel<ES, T>, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(union_attn_kernel<ES, T>, dim3(grid), dim3(kThreads), smem, stream, tmK, tmV, p);
+    return launch_pdl(union_attn_kernel<ES, T>, dim3(grid), dim3(kThreads), smem, stream, tmK, tmV, tmQ, p);
 }
 
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
@@ -921,16 +1013,16 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t strea
     return cudaGetLastError();
 }
 
-cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p,
-                              int grid, size_t smem, cudaStream_t stream) {
-    if (es == 2 && T == 16) return launch_t<2, 16>(tmK, tmV, p, grid, smem, stream);
-    if (es == 2 && T == 32) return launch_t<2, 32>(tmK, tmV, p, grid, smem, stream);
-    if (es == 2 && T == 64) return launch_t<2, 64>(tmK, tmV, p, grid, smem, stream);
-    if (es == 2 && T == 128) return launch_t<2, 128>(tmK, tmV, p, grid, smem, stream);
-    if (es == 1 && T == 64) return launch_t<1, 64>(tmK, tmV, p, grid, smem, stream);
-    if (es == 1 && T == 128) return launch_t<1, 128>(tmK, tmV, p, grid, smem, stream);
-    if (es == 4 && T == 32) return launch_t<4, 32>(tmK, tmV, p, grid, smem, stream);
-    if (es == 4 && T == 64) return launch_t<4, 64>(tmK, tmV, p, grid, smem, stream);
+cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                              const AttnParams& p, int grid, size_t smem, cudaStream_t stream) {
+    if (es == 2 && T == 16) return launch_t<2, 16>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 2 && T == 32) return launch_t<2, 32>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 2 && T == 64) return launch_t<2, 64>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 2 && T == 128) return launch_t<2, 128>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 1 && T == 64) return launch_t<1, 64>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 1 && T == 128) return launch_t<1, 128>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 4 && T == 32) return launch_t<4, 32>(tmK, tmV, tmQ, p, grid, smem, stream);
+    if (es == 4 && T == 64) return launch_t<4, 64>(tmK, tmV, tmQ, p, grid, smem, stream);
     return cudaErrorInvalidValue;
 }
 
