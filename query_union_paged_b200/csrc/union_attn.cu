@@ -82,8 +82,8 @@ constexpr int kKProducerWarp = 8, kSWarp = 9, kVProducerWarp = 10, kPvWarp = 11;
 constexpr uint32_t kColO = 0, kColS = 256;  // O_w at kColO + 128 w, S_w at kColS + 128 w
 // Register split: the launch gives every thread kLaunchRegs (384 x 168 = 64,512 of the SM's
 // 65,536); the producer and issuer warpgroup gives back down to kOtherRegs and the two softmax
-// warpgroups take kSoftmaxRegs: 256 x 224 + 128 x 56 = 64,512, exactly the launch's total.
-constexpr int kLaunchRegs = 168, kSoftmaxRegs = 224, kOtherRegs = 56;
+// warpgroups take kSoftmaxRegs: 256 x 208 + 128 x 88 = 64,512, exactly the launch's total.
+constexpr int kLaunchRegs = 168, kSoftmaxRegs = 208, kOtherRegs = 88;
 static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs, "register split");
 
 template <int ES, int T>
@@ -102,9 +102,14 @@ struct Geo {
     static constexpr int kNumMmaPV = kST * ES / 32;     // MMAs per O update (K = 128 tokens)
     static constexpr int kPCols = kST * ES / 4;         // TMEM columns of P
     static_assert(kPCols <= 128, "P fits in its S buffer");
-    // exponentials on the FMA pipe by a polynomial: pairs (j / 2) % 8 < kPolyPairs of every 16
-    // columns; the rest go to the MUFU unit
-    static constexpr int kPolyPairs = 2;
+    // E4M3: P goes to shared memory (one 16 KB K-major tile per warpgroup), so S_w is free as
+    // soon as the softmax has loaded it; the other types write P over S in TMEM
+    static constexpr bool kPSmem = ES == 1;
+    static constexpr int kPBytes = kRows * kST * ES;    // one warpgroup's P tile in shared memory
+    // exponentials on the FMA pipe by a polynomial for pairs (j / 2) % 8 < kPolyPairs of every 16
+    // columns, the rest on the MUFU unit (measured on this part per 128-score step of a warp: E4M3
+    // pack 809 cycles with 3 pairs, 832 with 2, 1,040 with none; bf16 pack 887 with 2)
+    static constexpr int kPolyPairs = ES == 1 ? 3 : 2;
     static_assert(PPS <= kMaxPPS, "pages per step");
     static constexpr uint32_t kFmt = (ES == 2) ? 1u : (ES == 4 ? 2u : 0u);
     static constexpr int kKind = (ES == 2) ? 0 : (ES == 4 ? 1 : 2);
@@ -116,14 +121,14 @@ struct Geo {
 };
 
 struct SmemLayout {
-    uint32_t kst, vst, q, qst, sinfo, mrg, qsc, bars, misc, total;
+    uint32_t kst, vst, q, p, qst, sinfo, mrg, bars, misc, total;
 };
 
 // Stage of the next bundle (E4M3: its bf16 Q rows): query slot m holds the g rows of its query,
 // 256 bytes each, at m * qstage_stride(g); the 16-byte pad keeps row reads free of bank conflicts.
 __host__ __device__ inline uint32_t qstage_stride(int g) { return (uint32_t)g * 256u + 16u; }
 constexpr int kSinfoWords = 8;  // bundle header: flat bundle, h, bi, ub, nU, nsteps, ok
-constexpr int kFixedBars = 14;
+constexpr int kFixedBars = 16;
 
 __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv, int g) {
     SmemLayout L;
@@ -135,14 +140,14 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     off += (uint32_t)nsv * kST * kD * es;
     L.q = off;  // 1024-aligned: every tile above is a multiple of 16 KB
     off += (uint32_t)kRows * kD * es;
+    L.p = off;  // E4M3: the two warpgroups' P tiles (1024-aligned)
+    if (es == 1) off += 2u * kRows * kST;
     L.qst = off;
     if (es == 1) off += MQ * qstage_stride(g);
     L.sinfo = off;
     off += 4u * (kSinfoWords + 2u * MQ);  // header, qid[MQ], q_pos[MQ]
     L.mrg = off;
     off += 2u * kRows * 8u;  // per warpgroup and row: running max and sum (float2)
-    L.qsc = off;
-    if (es == 1) off += 4u * kRows;  // E4M3: per-row score scale of the quantised Q
     off = (off + 7u) & ~7u;
     L.bars = off;
     off += 8u * (2u * (nsk + nsv) + kFixedBars);
@@ -170,8 +175,9 @@ struct Bars {
     __device__ __forceinline__ uint32_t stempty() const { return fixed(9); } // header read by every softmax warp
     __device__ __forceinline__ uint32_t ep1() const { return fixed(10); }    // both row states published
     __device__ __forceinline__ uint32_t ep2() const { return fixed(11); }    // both halves of O read
-    __device__ __forceinline__ uint32_t drain() const { return fixed(12); }
-    __device__ __forceinline__ uint32_t drain2() const { return fixed(13); }
+    __device__ __forceinline__ uint32_t sfree(int w) const { return fixed(12 + w); }  // S_w loaded (P in smem)
+    __device__ __forceinline__ uint32_t drain() const { return fixed(14); }
+    __device__ __forceinline__ uint32_t drain2() const { return fixed(15); }
 };
 
 struct Item {
@@ -267,7 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(B.pfull(w), 4);  // one arrive per warp of softmax warpgroup w
             mbar_init(B.pvdone(w), 1);
         }
-        mbar_init(B.qfull(), ES == 2 ? 1 : 4);  // bf16: the TMA transactions; else warpgroup 0's warps
+        mbar_init(B.qfull(), ES == 2 ? 1 : kSoftmaxWarps);  // bf16: the TMA transactions; else the softmax warps
+        for (int w = 0; w < 2; ++w) mbar_init(B.sfree(w), 4);
         mbar_init(B.qfree(), 1);
         mbar_init(B.stfull(), 1);
         mbar_init(B.stempty(), kSoftmaxWarps);
@@ -496,9 +503,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     for (int s = 0; s < it.nsteps; ++s) {
                         const int w = s & 1, k = use[w];
+                        // S_w is free once its previous use has been read: by the softmax (P in
+                        // shared memory) or by the O update (P over S in TMEM)
                         ok = warp_ok(mbar_wait_idle(B.kfull(ks), kph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
-                                     (k < 1 || mbar_wait_idle(B.pvdone(w), (k - 1) & 1, abort_flag, p.err,
-                                                              QUP_ERR_TIMEOUT, lim)));
+                                     (k < 1 || mbar_wait_idle(G::kPSmem ? B.sfree(w) : B.pvdone(w), (k - 1) & 1,
+                                                              abort_flag, p.err, QUP_ERR_TIMEOUT, lim)));
                         if (!ok) break;
                         tc_fence_after();
                         const uint64_t kdesc = smem_desc(sbase + L.kst + (uint32_t)ks * G::kTile, 16, 1024, 2);
@@ -566,12 +575,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         const uint64_t vdesc = smem_desc(sbase + L.vst + (uint32_t)vs * G::kTile,
                                                          (uint32_t)G::kChunkBytes, vsbo, vlayout);
+                        const uint64_t pdesc = smem_desc(sbase + L.p + (uint32_t)w * G::kPBytes, 16, 1024, 2);
                         if (elect_one_sync()) {
 #pragma unroll
                             for (int kk = 0; kk < G::kNumMmaPV; ++kk) {
-                                // K step = kMmaK tokens: 8 TMEM columns of P, kMmaK rows of V
-                                tc_mma_ts<G::kKind>(tmem + kColO + 128u * w, tmem + kColS + 128u * w + 8u * kk,
-                                                    vdesc + ((kk * G::kMmaK * 128) >> 4), idesc_o, s >= 2 || kk > 0);
+                                // K step = kMmaK tokens: 32 bytes of each P row, kMmaK rows of V
+                                if constexpr (G::kPSmem)
+                                    tc_mma<G::kKind>(tmem + kColO + 128u * w, pdesc + ((kk * 32) >> 4),
+                                                     vdesc + ((kk * G::kMmaK * 128) >> 4), idesc_o, s >= 2 || kk > 0);
+                                else
+                                    tc_mma_ts<G::kKind>(tmem + kColO + 128u * w, tmem + kColS + 128u * w + 8u * kk,
+                                                        vdesc + ((kk * G::kMmaK * 128) >> 4), idesc_o, s >= 2 || kk > 0);
                             }
                             tc_commit(B.pvdone(w));
                             tc_commit(B.vempty(vs));
@@ -605,13 +619,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float kPosInf = __int_as_float(0x7f800000);
         const int* sinfo = reinterpret_cast<const int*>(smem + L.sinfo);
         float2* mrg = reinterpret_cast<float2*>(smem + L.mrg);  // [2][kRows]
-        float* qsc = reinterpret_cast<float*>(smem + L.qsc);
         int use = 0;  // this warpgroup's uses of S_w and O_w so far
         bool ok = true;
         // the row's bundle state: item, query (original ID), Q head, visible positions, score scale
         Item it{};
         int qid = -1, head = 0, vis_end = 0;
-        float cs = p.scale_log2;
+        float cs = p.scale_log2, vscale = 1.f;
         float m_used = kNegInf, lsum = 0.f;
         f2 cs2{cs, cs};
         // The bundle's union entries, 32 at a time: lane j holds entry base + j, its logical
@@ -637,10 +650,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         // Take over the ino-th bundle of this CTA from the header the V warp wrote: its item, this
-        // row's query (original ID) and position, the first union entries.  Warpgroup 0 writes
-        // the Q operand for the non-bf16 types (E4M3: quantised per row from the staged bf16
-        // rows; fp32: from global memory) once every S of the previous bundle has completed;
-        // E4M3 warpgroup 1 then reads its rows' score scales.  Releases the header.
+        // row's query (original ID) and position, the first union entries.  For the non-bf16
+        // types both warpgroups write the Q operand (E4M3: quantised per row from the staged bf16
+        // rows; fp32: from global memory), half of each row each, once every S of the previous
+        // bundle has completed.  Releases the header.
         auto take = [&](int ino) -> bool {
             if (!warp_ok(mbar_wait(B.stfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
             it.h = sinfo[1];
@@ -658,64 +671,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             cbase = 0;
             fetch(0, cpage, cmask);
             fetch(32, npage, nmask);
+            if constexpr (ES == 1) vscale = p.v_scale[it.h];
             if constexpr (ES != 2) {
-                if (w == 0) {
-                    if (ino > 0 &&
-                        !warp_ok(mbar_wait(B.qfree(), (ino - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim)))
-                        return false;
-                    uint8_t* qt = smem + L.q;
-                    if constexpr (ES == 4) {
-                        const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
-                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
+                // the Q operand, once every S of the previous bundle has completed: each warpgroup
+                // writes half of every row's 128-byte chunks
+                if (ino > 0 && !warp_ok(mbar_wait(B.qfree(), (ino - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim)))
+                    return false;
+                uint8_t* qt = smem + L.q;
+                if constexpr (ES == 4) {
+                    const size_t row_off = ((size_t)(qid >= 0 ? qid : 0) * p.Hq + head) * kD;
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.Q) + row_off);
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
-                        }
-                    } else {  // the whole row: bf16 -> E4M3 with the row's scale amax / 448
-                        const uint8_t* row =
-                            smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
-                        uint4 raw[16];
-                        float amax = 0.f;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            raw[c] = qid >= 0 ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0, 0, 0, 0);
-                            const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
-                                                         fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
-                        }
-                        const float inv = amax > 0.f ? 448.f / amax : 0.f;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {  // 16 bf16 -> 16 E4M3 (one 16-byte chunk)
-                            uint32_t qv[4];
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const uint4 v = raw[2 * c + hh];
-                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                                float x[8];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
-                                    x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
-                                }
-                                qv[2 * hh] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
-                                qv[2 * hh + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
-                            }
-                            *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) =
-                                make_uint4(qv[0], qv[1], qv[2], qv[3]);
-                        }
-                        cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
-                        qsc[r] = cs;
+                    for (int c = 16 * w; c < 16 * w + 16; ++c) {
+                        const uint4 v = qid >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = v;
                     }
-                    fence_proxy_async_smem();  // generic-proxy writes of Q -> the tensor core
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(B.qfull());
-                } else if constexpr (ES == 1) {
-                    if (!warp_ok(mbar_wait(B.qfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
-                    cs = qsc[r];
+                } else {  // the whole row's amax, then this half: bf16 -> E4M3 with the row's scale amax / 448
+                    const uint8_t* row = smem + L.qst + (uint32_t)(r / g) * qstage_stride(g) + (uint32_t)(r % g) * 256u;
+                    uint4 raw[16];
+                    float amax = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        raw[c] = qid >= 0 ? *reinterpret_cast<const uint4*>(row + c * 16) : make_uint4(0, 0, 0, 0);
+                        const uint32_t w4[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                                     fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+                    }
+                    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {  // 16 bf16 -> 16 E4M3 (one 16-byte chunk)
+                        if ((c >> 2) != w) continue;
+                        uint32_t qv[4];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint4 v = raw[2 * c + hh];
+                            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                x[2 * e] = __uint_as_float(w4[e] << 16) * inv;
+                                x[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u) * inv;
+                            }
+                            qv[2 * hh] = pack_e4m3x4(x[0], x[1], x[2], x[3]);
+                            qv[2 * hh + 1] = pack_e4m3x4(x[4], x[5], x[6], x[7]);
+                        }
+                        *reinterpret_cast<uint4*>(qt + kmajor_sw128(r, c, kRows)) = make_uint4(qv[0], qv[1], qv[2], qv[3]);
+                    }
+                    cs = amax * (1.f / 448.f) * p.k_scale[it.h] * p.scale_log2;
                 }
+                fence_proxy_async_smem();  // generic-proxy writes of Q -> the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(B.qfull());
             }
             // a Q row of zeros (E4M3 scale 0) keeps a positive score scale: its scores are 0 anyway
             cs = fmaxf(cs, 1e-30f);
@@ -733,14 +741,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return ff;
         };
-        // exponentials of one step: p = 2^(s*cs - m_used + kPLog2) into pk (or sv for fp32),
-        // and their sum
+        // exponentials of one step: p = 2^(s*cs - m_used + kPLog2), their sum returned.  P leaves
+        // every 16 tokens as it is made (E4M3: one 16-byte chunk of row r of this warpgroup's
+        // shared-memory P tile; bf16: 8 TMEM columns over S_w), so no more than a chunk of it is
+        // ever held in registers; fp32 P is written over sv and stored by the caller.
         uint32_t sv[kST];
-        uint32_t pk[ES == 4 ? 1 : G::kPCols];
-        auto exps = [&](const int (&lim_q)[PPS]) -> float {
+        uint8_t* const ptile = smem + L.p + (uint32_t)w * G::kPBytes;
+        auto exps = [&](const int (&lim_q)[PPS], uint32_t s_addr) -> float {
             const float mb = (m_used == kNegInf ? 0.f : m_used) - G::kPLog2;
             f2 part[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-            f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token column
+            f2 e_prev{0.f, 0.f};  // E4M3: the first pair of a 4-token word
+            uint32_t ck[8];       // the current 16-token chunk of P (bf16: 8 words, E4M3: 4)
 #pragma unroll
             for (int q = 0; q < PPS; ++q) {  // one page (T tokens) at a time
                 // a page the row did not select gets an infinite offset: 2^-inf = 0
@@ -758,20 +769,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     part[(j >> 1) & 3] = add2(part[(j >> 1) & 3], e);
                     if constexpr (ES == 2) {
-                        pk[j / 2] = pack_bf16x2(e.x, e.y);
+                        ck[(j & 15) >> 1] = pack_bf16x2(e.x, e.y);
+                        if ((j & 15) == 14) tmem_st_x8(s_addr + (uint32_t)(j >> 1) - 7u, ck);
                     } else if constexpr (ES == 4) {
                         sv[j] = __float_as_uint(e.x);
                         sv[j + 1] = __float_as_uint(e.y);
-                    } else {  // E4M3: four tokens per 32-bit column
+                    } else {  // E4M3: four tokens per 32-bit word, four words per chunk
                         if (j & 2)
-                            pk[j / 4] = pack_e4m3x4(e_prev.x, e_prev.y, e.x, e.y);
+                            ck[(j & 15) >> 2] = pack_e4m3x4(e_prev.x, e_prev.y, e.x, e.y);
                         else
                             e_prev = e;
+                        if ((j & 15) == 14)
+                            *reinterpret_cast<uint4*>(ptile + kmajor_sw128(r, j >> 4, kRows)) =
+                                make_uint4(ck[0], ck[1], ck[2], ck[3]);
                     }
                 }
             }
             const f2 ps = add2(add2(part[0], part[1]), add2(part[2], part[3]));
             return ps.x + ps.y;
+        };
+        // P of zeros (a warp whose rows selected none of the step's pages)
+        auto zero_p = [&](uint32_t s_addr) {
+            if constexpr (ES == 1) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(ptile + kmajor_sw128(r, c, kRows)) = make_uint4(0, 0, 0, 0);
+            } else {
+                uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int c = 0; c < G::kPCols; c += 8) tmem_st_x8(s_addr + (uint32_t)c, z);
+            }
         };
 
         int rnd = 0, item_no = 0;
@@ -814,6 +841,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_base + colS;
                 tmem_ld128_wait(s_addr, sv);
+                if constexpr (G::kPSmem) {  // S_w is in registers: the next S may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(B.sfree(w));
+                }
                 const bool warp_live = __any_sync(0xffffffffu, live);
                 // Raw scores of unseen tokens (past the row's causal limit or kv_len inside a page
                 // it selected) become -inf; pages the row did not select get an infinite offset in
@@ -848,22 +880,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         m_used = mloc;
                         lsum *= alpha;
                     }
-                    lsum += exps(lim_q);
-                } else {
-                    if constexpr (ES == 4) {
-#pragma unroll
-                        for (int j = 0; j < kST; ++j) sv[j] = 0u;
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < G::kPCols; ++j) pk[j] = 0u;
-                    }
                 }
                 // O_w is rescaled only after its previous update has finished (rare); the first
-                // update of O_w in a bundle overwrites it
-                if (s >= 2 && __any_sync(0xffffffffu, need)) {
+                // update of O_w in a bundle overwrites it.  The shared-memory P tile (E4M3) is
+                // rewritten only after that update has read it.
+                const bool rescale = s >= 2 && __any_sync(0xffffffffu, need);
+                if (rescale || (G::kPSmem && k >= 1)) {
                     ok = warp_ok(mbar_wait(B.pvdone(w), (k - 1) & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                     if (!ok) break;
                     tc_fence_after();
+                }
+                if (rescale) {
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t ov[32];
@@ -873,12 +900,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st_x32(tmem + lane_base + colO + 32u * c, ov);
                     }
                 }
-                // P over the S buffer it came from (every column of S is in registers)
-                if constexpr (ES == 4) {
-                    tmem_st_n<kST>(s_addr, sv);
+                // P of this step: over S_w (bf16, fp32) or into row r of this warpgroup's shared-memory
+                // P tile (E4M3, K-major, swizzled), as it is made
+                if (warp_live) {
+                    lsum += exps(lim_q, s_addr);
+                    if constexpr (ES == 4) tmem_st_n<kST>(s_addr, sv);
                 } else {
-                    tmem_st_n<G::kPCols>(s_addr, pk);
+                    zero_p(s_addr);
                 }
+                if constexpr (G::kPSmem) fence_proxy_async_smem();
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -887,6 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const Item it_cur = it;
             const int qid_cur = qid, head_cur = head;
+            const float vsc = vscale;
             const float lsum_cur = lsum, m_cur = m_used;
             const int k_last = use - 1;
             const int n0 = (it_cur.nsteps + 1) / 2, n1 = it_cur.nsteps / 2;  // steps of each warpgroup
@@ -916,8 +947,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mm = fmaxf(l0 > 0.f ? m0 : kNegInf, l1 > 0.f ? m1 : kNegInf);
             const float f0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, f1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
             const float ltot = l0 * f0 + l1 * f1;
-            float vsc = 1.f;
-            if constexpr (ES == 1) vsc = p.v_scale[it_cur.h];
             const float inv = ltot > 0.f ? vsc / ltot : 0.f;
             const float a0 = f0 * inv, a1 = f1 * inv;
             const size_t oi = ((size_t)(qid_cur >= 0 ? qid_cur : 0) * p.Hq + head_cur) * kD;
