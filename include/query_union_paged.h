@@ -226,6 +226,53 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                             const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq, int d,
                             float softmax_scale, void* O, float* lse, void* stream);
 
+/*
+ * Batched requests (varlen chunks; chunked prefill of several sequences over
+ * one paged cache, as in CompactAttention: Approach).  R sequences, each with
+ * its own page table, cache length and chunk of queries, go through one
+ * grouping call and one attention call.  The requests are laid end to end:
+ *   q_ptr     device int32 [R+1], ascending: the queries of request r are the
+ *             batch rows q_ptr[r] .. q_ptr[r+1) (rows of Q, O, q_pos, topk)
+ *   page_ptr  device int32 [R+1], ascending: request r's logical pages are
+ *             page_table[page_ptr[r] .. page_ptr[r+1]) of the concatenated
+ *             page table (total_pages = page_ptr[R] entries, into one
+ *             physical K/V cache)
+ *   kv_len    device int32 [R]: tokens in request r's cache (at most its
+ *             pages x T); q_pos and topk hold request-local positions and
+ *             request-local logical page IDs (-1 = padding)
+ * qup_batch_prepare writes, on the stream:
+ *   topk_global device int32 [Hq][Nq][Ksel]: the TopK IDs rebased to the
+ *             concatenated page space (page_ptr[r] + local ID; -1 kept), for
+ *             qup_sparse_group(topk_global, ..., num_logical_pages = total_pages, ...)
+ *   q_end     device int32 [Nq]: page_ptr[r]*T + min(q_pos + 1, kv_len[r]),
+ *             the end of the query's visible positions (token slot o of
+ *             concatenated page u has position u*T + o)
+ *   page_len  device int32 [total_pages]: valid tokens of each page (0..T)
+ * Device errors: a local page ID outside its request's pages raises
+ * QUP_ERR_PAGE_ID (entry dropped); a row in no request or a kv_len beyond its
+ * pages raises QUP_ERR_GROUP (the row attends nothing).  QUP_ERR_ARG for bad
+ * sizes, T not in {16, 32, 64, 128}, total_pages*T >= 2^31 or missing
+ * pointers.  Each query attends exactly the tokens the one-sequence call
+ * would give it inside its own request.
+ */
+int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq, int Ksel, int T, int R,
+                      const int32_t* q_ptr, const int32_t* page_ptr, const int32_t* kv_len, int total_pages,
+                      int32_t* topk_global, int32_t* q_end, int32_t* page_len, void* stream);
+
+/*
+ * qup_sparse_prefill_attn for batched requests: the arguments of
+ * qup_sparse_prefill_attn with (q_pos, kv_len) replaced by the q_end and
+ * page_len arrays of qup_batch_prepare, page_table the concatenated table of
+ * total_pages entries, and groups from qup_sparse_group on topk_global.
+ * topk_global is read only in checked mode (and may be NULL).
+ */
+int qup_sparse_prefill_attn_batch(const void* Q, int q_dtype, const void* K_cache, const void* V_cache,
+                                  int kv_dtype, const float* k_scale, const float* v_scale,
+                                  const int32_t* page_table, int total_pages, int P_phys, int T,
+                                  const int32_t* topk_global, int Ksel, const qup_groups* groups,
+                                  const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq, int d,
+                                  float softmax_scale, void* O, float* lse, void* stream);
+
 /* Synchronizes `stream`, then reads and clears this device's error word. */
 int qup_get_error(int* code, void* stream);
 

@@ -20,6 +20,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host", "union_support",
+           "Batch", "batch_prepare", "sparse_prefill_attn_batch",
            "get_error", "set_debug", "set_checked", "load",
            "QupError", "F32", "BF16", "E4M3", "ERR"]
 
@@ -72,9 +73,13 @@ def load():
     lib.qup_exp2_poly.argtypes = [P, P, I, P]
     lib.qup_union_support.argtypes = [ctypes.POINTER(_Groups), I, I, I, I, I, P, SZ, P]
     lib.qup_set_checked.argtypes = [I]
+    lib.qup_batch_prepare.argtypes = [P, P, I, I, I, I, I, P, P, P, I, P, P, P, P]
+    lib.qup_sparse_prefill_attn_batch.argtypes = [P, I, P, P, I, P, P, P, I, I, I, P, I,
+                                                  ctypes.POINTER(_Groups), P, P, I, I, I, I,
+                                                  ctypes.c_float, P, P, P]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
                "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support",
-               "qup_set_checked"):
+               "qup_set_checked", "qup_batch_prepare", "qup_sparse_prefill_attn_batch"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -274,6 +279,61 @@ def sparse_prefill_attn(Q, K_cache, V_cache, page_table, groups: Groups, q_pos, 
                                        _p(q_pos), kv_len, Hq, Hkv, Nq, d, float(softmax_scale),
                                        _p(out), _p(lse), _stream_ptr(stream)),
            "qup_sparse_prefill_attn")
+    return out
+
+
+@dataclasses.dataclass
+class Batch:
+    """Device arrays of batched requests after batch_prepare (see qup_batch_prepare)."""
+    q_ptr: "torch.Tensor"
+    page_ptr: "torch.Tensor"
+    kv_len: "torch.Tensor"
+    topk_global: "torch.Tensor"
+    q_end: "torch.Tensor"
+    page_len: "torch.Tensor"
+    total_pages: int
+
+
+def batch_prepare(topk, q_pos, q_ptr, page_ptr, kv_len, total_pages: int, T: int, stream=None) -> Batch:
+    """Rebase request-local TopK rows and positions to the concatenated page space of a batch
+    (qup_batch_prepare).  topk int32 [Hq][Nq][Ksel], q_pos int32 [Nq]; q_ptr, page_ptr int32 [R+1];
+    kv_len int32 [R]; all CUDA tensors."""
+    import torch
+    Hq, Nq, Ksel = topk.shape
+    R = q_ptr.numel() - 1
+    dev = topk.device
+    b = Batch(q_ptr=q_ptr, page_ptr=page_ptr, kv_len=kv_len,
+              topk_global=torch.empty_like(topk), q_end=torch.empty(Nq, dtype=torch.int32, device=dev),
+              page_len=torch.empty(max(total_pages, 1), dtype=torch.int32, device=dev), total_pages=total_pages)
+    _check(load().qup_batch_prepare(_p(topk), _p(q_pos), Hq, Nq, Ksel, T, R, _p(q_ptr), _p(page_ptr), _p(kv_len),
+                                    total_pages, _p(b.topk_global), _p(b.q_end), _p(b.page_len),
+                                    _stream_ptr(stream)), "qup_batch_prepare")
+    return b
+
+
+def sparse_prefill_attn_batch(Q, K_cache, V_cache, page_table, groups: Groups, batch: Batch, k_scale=None,
+                              v_scale=None, softmax_scale: Optional[float] = None, out=None, lse=None,
+                              checked_topk: bool = False, stream=None):
+    """Union attention over batched requests (qup_sparse_prefill_attn_batch): page_table is the
+    concatenated table of batch.total_pages entries; groups come from sparse_group on
+    batch.topk_global."""
+    import torch
+    lib = load()
+    Nq, Hq, d = Q.shape
+    P_phys, Hkv, T, d2 = K_cache.shape
+    assert d2 == d and V_cache.shape == K_cache.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    cs = groups.c_struct()
+    tk = batch.topk_global if checked_topk else None
+    _check(lib.qup_sparse_prefill_attn_batch(_p(Q), _dtype_code(Q), _p(K_cache), _p(V_cache), _dtype_code(K_cache),
+                                             _p(k_scale), _p(v_scale), _p(page_table), batch.total_pages, P_phys, T,
+                                             _p(tk), tk.shape[-1] if tk is not None else 0, ctypes.byref(cs),
+                                             _p(batch.q_end), _p(batch.page_len), Hq, Hkv, Nq, d,
+                                             float(softmax_scale), _p(out), _p(lse), _stream_ptr(stream)),
+           "qup_sparse_prefill_attn_batch")
     return out
 
 

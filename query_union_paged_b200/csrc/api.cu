@@ -14,6 +14,11 @@
 #include "query_union_paged.h"
 
 namespace qup {
+// batch.cu: request-local TopK IDs -> global IDs, per-query visible ends, per-page valid tokens
+cudaError_t launch_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq, int K, int T, int R,
+                                 const int32_t* q_ptr, const int32_t* page_ptr, const int32_t* kv_len, int total_pages,
+                                 int32_t* topk_global, int32_t* q_end, int32_t* page_len, unsigned* err,
+                                 cudaStream_t stream);
 // group.cu: every row of each group sees every page of the group's union (row masks set to the
 // group's rows)
 cudaError_t launch_union_support(const int32_t* n_groups, const int32_t* group_ptr, const int32_t* union_ptr,
@@ -349,11 +354,16 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
     return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st);
 }
 
-int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
-                            const float* k_scale, const float* v_scale, const int32_t* page_table,
-                            int num_logical_pages, int P_phys, int T, const int32_t* topk, int Ksel,
-                            const qup_groups* groups, const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq,
-                            int d, float softmax_scale, void* O, float* lse, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The attention call for one sequence (q_pos, kv_len) or for batched requests (q_end, page_len).
+int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
+              const float* k_scale, const float* v_scale, const int32_t* page_table, int num_logical_pages,
+              int P_phys, int T, const int32_t* topk, int Ksel, const qup_groups* groups, const int32_t* q_pos,
+              int kv_len, const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq, int d,
+              float softmax_scale, void* O, float* lse, void* stream) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || d != qup::kHeadDim) return QUP_ERR_ARG;
     if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
     // supported (dtype, page size) pairs: bf16 16/32/64/128, E4M3 64/128, fp32 32/64
@@ -367,8 +377,10 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     if (es == 1 && (!k_scale || !v_scale)) return QUP_ERR_ARG;
     if ((es == 1 && T < 64) || (es == 4 && (T < 32 || T > 64))) return QUP_ERR_ARG;
     if (!groups || !bundle_fields_ok(groups) || groups->rows_per_group < 1) return QUP_ERR_ARG;
+    if ((int64_t)num_logical_pages * T >= ((int64_t)1 << 31)) return QUP_ERR_ARG;  // token positions are int32
     if (Nq == 0) return QUP_OK;
-    if (!Q || !K_cache || !V_cache || !page_table || !q_pos || !O) return QUP_ERR_ARG;
+    if (!Q || !K_cache || !V_cache || !page_table || !O) return QUP_ERR_ARG;
+    if (!q_end && !q_pos) return QUP_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(K_cache) | reinterpret_cast<uintptr_t>(V_cache)) & 15) return QUP_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(groups->bunion_mask)) & 15) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
@@ -436,6 +448,8 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     p.bundle_qid = groups->bundle_qid;
     p.bundle_order = groups->bundle_order;
     p.q_pos = q_pos;
+    p.q_end = q_end;
+    p.page_len = page_len;
     p.O = O;
     p.lse = lse;
     p.err = ds->err;
@@ -457,6 +471,53 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
     const cudaError_t e =
         qup::launch_union_attn(es, T, tm[0], tm[1], tmq, p, ds->sms, smem, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
+                            const float* k_scale, const float* v_scale, const int32_t* page_table,
+                            int num_logical_pages, int P_phys, int T, const int32_t* topk, int Ksel,
+                            const qup_groups* groups, const int32_t* q_pos, int kv_len, int Hq, int Hkv, int Nq,
+                            int d, float softmax_scale, void* O, float* lse, void* stream) {
+    if (Nq > 0 && !q_pos) return QUP_ERR_ARG;
+    return attn_impl(Q, q_dtype, K_cache, V_cache, kv_dtype, k_scale, v_scale, page_table, num_logical_pages,
+                     P_phys, T, topk, Ksel, groups, q_pos, kv_len, nullptr, nullptr, Hq, Hkv, Nq, d, softmax_scale,
+                     O, lse, stream);
+}
+
+int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq, int Ksel, int T, int R,
+                      const int32_t* q_ptr, const int32_t* page_ptr, const int32_t* kv_len, int total_pages,
+                      int32_t* topk_global, int32_t* q_end, int32_t* page_len, void* stream) {
+    if (Hq <= 0 || Nq < 0 || Ksel < 0 || R < 0 || total_pages < 0) return QUP_ERR_ARG;
+    if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
+    if ((int64_t)total_pages * T >= ((int64_t)1 << 31)) return QUP_ERR_ARG;
+    if (Nq > 0 && (!q_pos || !q_end || !q_ptr || !page_ptr || !kv_len || R == 0 ||
+                   (Ksel > 0 && (!topk || !topk_global))))
+        return QUP_ERR_ARG;
+    if (total_pages > 0 && (!page_len || !page_ptr || !kv_len || R == 0)) return QUP_ERR_ARG;
+    DevState* ds = nullptr;
+    int rc = device_state(&ds);
+    if (rc) return rc;
+    return qup::launch_batch_prepare(topk, q_pos, Hq, Nq, Ksel, T, R, q_ptr, page_ptr, kv_len, total_pages,
+                                     topk_global, q_end, page_len, ds->err,
+                                     static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QUP_OK
+               : QUP_ERR_CUDA;
+}
+
+int qup_sparse_prefill_attn_batch(const void* Q, int q_dtype, const void* K_cache, const void* V_cache,
+                                  int kv_dtype, const float* k_scale, const float* v_scale,
+                                  const int32_t* page_table, int total_pages, int P_phys, int T,
+                                  const int32_t* topk_global, int Ksel, const qup_groups* groups,
+                                  const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq, int d,
+                                  float softmax_scale, void* O, float* lse, void* stream) {
+    if (Nq > 0 && (!q_end || !page_len)) return QUP_ERR_ARG;
+    return attn_impl(Q, q_dtype, K_cache, V_cache, kv_dtype, k_scale, v_scale, page_table, total_pages, P_phys, T,
+                     topk_global, Ksel, groups, nullptr, 0, q_end, page_len, Hq, Hkv, Nq, d, softmax_scale, O, lse,
+                     stream);
 }
 
 int qup_get_error(int* code, void* stream) {

@@ -55,6 +55,8 @@ struct AttnParams {
     const int32_t* bundle_qid;   // [Hkv][Nq][128/g]
     const int32_t* bundle_order; // [n_items] flat bundle indices, largest union first
     const int32_t* q_pos;
+    const int32_t* q_end;     // batched requests: [Nq] end of each query's visible positions, else null
+    const int32_t* page_len;  // batched requests: [num_logical_pages] valid tokens per page, else null
     void* O;
     float* lse;
     unsigned* err;

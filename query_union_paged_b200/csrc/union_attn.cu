@@ -145,7 +145,7 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     L.qst = off;
     if (es == 1) off += MQ * qstage_stride(g);
     L.sinfo = off;
-    off += 4u * (kSinfoWords + 2u * MQ);  // header, qid[MQ], q_pos[MQ]
+    off += 4u * (kSinfoWords + 2u * MQ);  // header, qid[MQ], visible-position end[MQ]
     L.mrg = off;
     off += 2u * kRows * 8u;  // per warpgroup and row: running max and sum (float2)
     off = (off + 7u) & ~7u;
@@ -222,6 +222,12 @@ __device__ __forceinline__ uint32_t kmajor_sw128(int r, int c, int rows) {
 }
 
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// Valid tokens of logical page u (0..T): tokens past the end of its sequence are never attended
+// and may hold any bytes.  One sequence: kv_len; batched requests: the per-page count.
+__device__ __forceinline__ int page_valid(const AttnParams& p, int u, int T) {
+    return p.page_len ? p.page_len[u] : max(0, min(T, p.kv_len - u * T));
+}
 
 template <int N>
 __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
@@ -354,7 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             qid = max(qid, -1);
                             sinfo[kSinfoWords + m] = qid;
-                            sinfo[kSinfoWords + MQ + m] = qid >= 0 ? p.q_pos[qid] : -1;
+                            // positions < this end are visible to the query (batched requests: its
+                            // precomputed end in the global token space)
+                            sinfo[kSinfoWords + MQ + m] =
+                                qid < 0 ? 0 : (p.q_end ? p.q_end[qid] : min(p.q_pos[qid] + 1, p.kv_len));
                         }
                         nvalid += __popc(__ballot_sync(0xffffffffu, qid >= 0));
                     }
@@ -549,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int q = 0; q < PPS; ++q) {
                             const int pg = __shfl_sync(0xffffffffu, cpg, e0 - cb + q);
-                            tail |= pg >= 0 && pg * T + T > p.kv_len;
+                            tail |= pg >= 0 && page_valid(p, pg, T) < T;
                         }
                         ok = warp_ok(mbar_wait_idle(B.pfull(w), k & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim) &&
                                      mbar_wait_idle(B.vfull(vs), vph, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
@@ -559,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                             for (int q = 0; q < PPS; ++q) {
                                 const int pg = __shfl_sync(0xffffffffu, cpg, e0 - cb + q);
-                                if (pg < 0 || pg * T + T <= p.kv_len) continue;
-                                const int t0 = max(0, p.kv_len - pg * T);  // first token row past kv_len
+                                const int t0 = pg < 0 ? T : page_valid(p, pg, T);  // first token row past kv_len
+                                if (t0 >= T) continue;
                                 const int nwords = (T - t0) * G::kNChunk * 8;  // 16-byte words to clear
                                 for (int i = lane; i < nwords; i += 32) {
                                     const int row = q * T + t0 + i / (G::kNChunk * 8);
@@ -630,13 +639,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The bundle's union entries, 32 at a time: lane j holds entry base + j, its logical
         // page (-1 for padding or an entry the producers reject) and this warp's 32-bit word
         // of the page's row mask.  The next 32 are loaded one batch ahead.
+        // A page whose tokens reach past the end of its sequence (a tail page) may hold non-finite
+        // bytes there: its entry carries a tail flag.
         int cpage = -1, npage = -1;
         uint32_t cmask = 0u, nmask = 0u;
+        bool ctail = false, ntail = false;
         int cbase = 0;
-        auto fetch = [&](int base, int& pg, uint32_t& mk) {
+        auto fetch = [&](int base, int& pg, uint32_t& mk, bool& tl) {
             const int e = base + lane;
             pg = -1;
             mk = 0u;
+            tl = false;
             if (e < it.nU) {
                 const int u = p.union_pages[it.ub + e];
                 const uint32_t m = p.row_mask[(size_t)(it.ub + e) * 4 + wq];
@@ -645,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ph >= 0 && ph < p.P_phys) {
                         pg = u;
                         mk = m;
+                        tl = page_valid(p, u, T) < T;
                     }
                 }
             }
@@ -663,14 +677,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             it.nsteps = sinfo[5];
             it.ok = sinfo[6] != 0;
             qid = sinfo[kSinfoWords + r / g];
-            const int qpos = sinfo[kSinfoWords + MQ + r / g];
+            const int qend = sinfo[kSinfoWords + MQ + r / g];
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             head = it.h * g + (r % g);
-            vis_end = min(qpos + 1, p.kv_len);  // positions < vis_end are visible
+            vis_end = qend;  // positions < vis_end are visible
             cs = p.scale_log2;                  // score scale (log2 domain) of this row
             cbase = 0;
-            fetch(0, cpage, cmask);
-            fetch(32, npage, nmask);
+            fetch(0, cpage, cmask, ctail);
+            fetch(32, npage, nmask, ntail);
             if constexpr (ES == 1) vscale = p.v_scale[it.h];
             if constexpr (ES != 2) {
                 // the Q operand, once every S of the previous bundle has completed: each warpgroup
@@ -818,7 +832,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cbase += 32;
                     cpage = npage;
                     cmask = nmask;
-                    fetch(cbase + 32, npage, nmask);
+                    ctail = ntail;
+                    fetch(cbase + 32, npage, nmask, ntail);
                 }
                 // row r sees token t of page q iff the page is in its own TopK row (its bit of the
                 // page's mask) and the token's position is < vis_end; a page that reaches kv_len
@@ -834,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     lim_q[q] = mine ? max(0, min(T, vis_end - pg * T)) : 0;
                     live |= lim_q[q] > 0;
                     partial |= lim_q[q] > 0 && lim_q[q] < T;
-                    tail |= pg >= 0 && pg * T + T > p.kv_len;
+                    tail |= __shfl_sync(0xffffffffu, ctail, e0 - cbase + q);
                 }
                 ok = warp_ok(mbar_wait(B.sfull(w), k & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
                 if (!ok) break;

@@ -167,14 +167,19 @@ def _community_chunk(name, seed, kv_dtype, T, prefix, Nq, n_comm, comm_size, com
     Hq, Hkv, d, K = 32, 8, 128, 16
     g = Hq // Hkv
     sel = np.empty((Hkv, Nq, K), np.int32)
+    own = (prefix + np.arange(Nq)) // T
     for h in range(Hkv):
         pool = rng.choice(np.arange(comm_lo, comm_hi + 1), size=n_comm * comm_size, replace=False)
         comms = pool.reshape(n_comm, comm_size)
         cid = rng.integers(0, n_comm, size=Nq)
-        for i in range(Nq):
-            own = (prefix + i) // T
-            picks = rng.choice(comms[cid[i]], size=K - 3, replace=False)
-            sel[h, i] = np.concatenate([[0, own, own - 1], picks])
+        # 13 distinct members of the query's community: the first 13 of a random permutation
+        # of its comm_size members (one independent permutation per query)
+        keys = rng.random((Nq, comm_size))
+        picks = np.take_along_axis(comms[cid], np.argsort(keys, axis=1)[:, :K - 3], axis=1)
+        sel[h, :, 0] = 0
+        sel[h, :, 1] = own
+        sel[h, :, 2] = own - 1
+        sel[h, :, 3:] = picks
     q_dtype = DT_BF16
     return _finish(name, rng, Hq, Hkv, Nq, d, T, prefix, q_dtype, kv_dtype,
                    _replicate_kv_groups(sel, g), identity_pages=identity_pages, window=window)
@@ -198,6 +203,16 @@ def gqa_chunk_fp8(seed: int = 2, identity_pages: bool = False) -> Workload:
     the wider window's tighter groups save more attention time than they cost.
     """
     return _community_chunk("gqa_chunk_fp8_16k+2k", seed, DT_E4M3, 128, 16384, 2048,
+                            8, 15, 1, 126, identity_pages, window=128)
+
+
+def chunk16k_fp8(seed: int = 5, identity_pages: bool = False) -> Workload:
+    """A 16K-query chunk after a 16K prefix (the pages' base captures: 16K-query chunks, Top16,
+    FP8 KV): 32/8 heads, E4M3 KV (per-KV-head scale), 128-token pages, TopK 16 = {sink, own,
+    own-1} + 13 from the query's community (8 disjoint communities of 15 pages in 1..126 per KV
+    head, one per query iid).  Grouping window 128, as for the other E4M3 community workloads.
+    """
+    return _community_chunk("chunk16k_fp8_16k+16k", seed, DT_E4M3, 128, 16384, 16384,
                             8, 15, 1, 126, identity_pages, window=128)
 
 
@@ -295,6 +310,7 @@ CONFIGS = {
     "4b": lambda **kw: ctx64k_fp8("b", **kw),
     "4c": lambda **kw: ctx64k_fp8("c", **kw),
     "5": block_union_128k,
+    "6": chunk16k_fp8,
 }
 
 

@@ -140,6 +140,22 @@ def test_full_size_every_element(cfg):
     check_close(O, ref, w.kv_dtype, w.name, report=True)
 
 
+def test_chunk16k_rows_of_every_block():
+    """The 16K-query chunk (the pages' base capture shape): one row per (Q head, 32-query block),
+    so every bundle of the grouping is compared, in the launch configuration the bench times.
+    (The oracle needs minutes for the whole output of this workload.)"""
+    w = workload("6")
+    dev = to_device(w)
+    O = out_to_f64(_attn(w, dev, _gpu_groups(w, dev)))
+    assert np.all(np.isfinite(O))
+    rng = np.random.default_rng(66)
+    blocks = np.arange(w.Hq * w.Nq // 32, dtype=np.int64)
+    rows = blocks * 32 + rng.integers(0, 32, size=blocks.size)
+    ref = oracle.sparse_attn_workload(w, rows=rows)
+    hq, i = rows // w.Nq, rows % w.Nq
+    check_close(O[i, hq], ref, w.kv_dtype, w.name + " (one row per head and 32-query block)", report=True)
+
+
 def _shuffled_positions(w, seed, max_back):
     """Query IDs in random order, and each position moved back by up to max_back tokens (gaps,
     repeats, out of order): rows may then hold pages past their query, which the causal limit

@@ -48,6 +48,15 @@ def test_workload_bitexact(cfg, window):
     assert_bundles_equal(got, oracle.bundle(ref, w.Hq, w.Hkv, w.Nq, 8))
 
 
+def test_chunk16k_bitexact():
+    """The 16K-query chunk: grouping workspace, groups and the 16,384-query bundle walk bit-exact."""
+    w = workload("6")
+    got = _run(w.topk, w.Hq, w.Hkv, w.num_logical_pages, 8, w.window)
+    ref = oracle.group(w.topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, 8, w.window)
+    assert_groups_equal(got, ref)
+    assert_bundles_equal(got, oracle.bundle(ref, w.Hq, w.Hkv, w.Nq, 8))
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_large_windows_small_universe_bitexact(seed):
     """Windows of 65..256 queries whose pages fit 8 words: the whole-CTA greedy."""
