@@ -250,6 +250,8 @@ def main():
     ap.add_argument("--bundle-window", type=int, default=None)
     ap.add_argument("--union-support", action="store_true",
                     help="every row of a group attends to its group's whole union (qup_union_support)")
+    ap.add_argument("--page-major", action="store_true",
+                    help="direct KV-page union: page-major items and partial results merged by lse")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -288,7 +290,22 @@ def main():
     O = torch.empty_like(dev["Q"])
     stream = torch.cuda.current_stream()
 
+    items = None
+    if args.page_major:
+        items = qup.page_major_items(topk, w.Hq, w.Hkv, w.num_logical_pages, w.T)
+
     def step(ev=None):
+        if args.page_major:  # items (timed as the grouping call), then attention and the merge
+            if ev is not None:
+                ev[0].record(stream)
+            qup.page_major_items(topk, w.Hq, w.Hkv, w.num_logical_pages, w.T, out=items)
+            if ev is not None:
+                ev[1].record(stream)
+            qup.page_major_attn(dev["Q"], dev["K"], dev["V"], page_table, items, q_pos, w.kv_len, k_scale=ks,
+                                v_scale=vs, out=O, num_logical_pages=w.num_logical_pages)
+            if ev is not None:
+                ev[2].record(stream)
+            return
         if ev is not None:
             ev[0].record(stream)
         qup.sparse_group(topk, w.Hq, w.Hkv, w.num_logical_pages, max_group, window, out=groups)
@@ -335,6 +352,8 @@ def main():
     flop = 4.0 * w.d * E
     n_uniq = unique_kv_pages(w)
     uniq_bytes = n_uniq * w.kv_page_bytes()
+    if args.page_major:  # the grouping counters of the same selection, for the work accounting
+        qup.sparse_group(topk, w.Hq, w.Hkv, w.num_logical_pages, max_group, window, out=groups)
     ctr = groups.counters.cpu().numpy().sum(axis=0)
     bctr = groups.bcounters.cpu().numpy().sum(axis=0)
     ms_per_step = total_ms / args.steps
@@ -347,7 +366,7 @@ def main():
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
 
     # ---- end to end through host buffers (pinned), copies inside the timed region
-    e2e = run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O, flop)
+    e2e = None if args.page_major else run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O, flop)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -358,7 +377,10 @@ def main():
         "config": {"workload": w.name, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "d": w.d,
                    "page_tokens": w.T, "topk": w.K, "kv_len": w.kv_len, "max_group": max_group,
                    "window": window, "bundle_window": bundle_window,
-                   "support": "group union" if args.union_support else "own TopK row", "l2": "flushed before every timed step (2x L2 write)",
+                   "support": "group union" if args.union_support else "own TopK row",
+                   "execution": "page-major items, partial results merged by lse" if args.page_major
+                   else "query unions (bundles of page-affine groups)",
+                   "l2": "flushed before every timed step (2x L2 write)",
                    "parallelism": f"replicas x{world} (independent chunks)"},
         "us_per_call": {"group": round(statistics.median(t_group) * 1e3, 2),
                         "attn": round(statistics.median(t_attn) * 1e3, 2),
@@ -370,6 +392,12 @@ def main():
                  "page_edges": int(ctr[3]), "bundles": int(bctr[1]),
                  "bundle_page_visits": int(bctr[0]),
                  "streamed_kv_bytes": int(bctr[0]) * w.kv_page_bytes()},
+        **({"page_major": {"items": int(items.arrays["n_items"].sum().item()), "tile_pages": items.tile_pages,
+                           "streamed_kv_bytes": int(items.arrays["n_items"].sum().item()) * items.tile_pages *
+                           w.kv_page_bytes(),
+                           "partial_results": int(items.arrays["row_off"][-1].item()),
+                           "partial_bytes_written_and_read": 2 * int(items.arrays["row_off"][-1].item()) * 4 * (w.d + 1)}}
+           if args.page_major else {}),
         "roofline": {"kernel": "union_attn_kernel", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": round(mma_peak, 1), "unit": "TFLOP/s",
                      "frac": round(attn_tflops / mma_peak, 4),

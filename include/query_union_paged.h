@@ -273,6 +273,63 @@ int qup_sparse_prefill_attn_batch(const void* Q, int q_dtype, const void* K_cach
                                   const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq, int d,
                                   float softmax_scale, void* O, float* lse, void* stream);
 
+/*
+ * Direct KV-page union (PageWeaver, Abstract; Figure 5): the page-major
+ * alternative to query unions.  Work is organised by KV page instead of by
+ * query group: the pages of each KV head are cut into tiles of 256 tokens
+ * (tile_pages = 256 / T pages), and an item is one tile with up to 128 / g
+ * queries whose page set (over the g Q heads of the KV group) meets it.  Each
+ * tile is streamed once per item by the same tensor-core union kernel; every
+ * row (query, Q head) keeps its own page mask and gets one partial result per
+ * tile its own TopK row touches (O_t / l_t in fp32 and lse_t in log2 units),
+ * which a merge then reduces per row by lse.  The result equals
+ * qup_sparse_prefill_attn's (the same per-query supports) up to rounding.
+ *
+ * Sizes (qup_page_major_workspace): ws_bytes of scratch for the item builder,
+ * item_cap items per KV head and slot_cap partial slots that always suffice,
+ * tile_pages.  QUP_ERR_ARG for unsupported sizes (g > 32, too many pages for
+ * the builder's shared-memory bitsets, capacities past 2^31).
+ */
+typedef struct {
+    int32_t* n_items;      /* [Hkv] items of each KV head */
+    int32_t* item_ptr;     /* [Hkv][item_cap+1] first union entry of each item (item i: tile_pages entries) */
+    int32_t* item_pages;   /* [Hkv*item_cap*tile_pages] logical pages of each item's tile */
+    uint32_t* item_mask;   /* [Hkv*item_cap*tile_pages][4] 128-bit row masks, as bunion_mask */
+    int32_t* item_qid;     /* [Hkv][item_cap][128/g] query of each query slot, -1 if empty */
+    int32_t* item_slot;    /* [Hkv*item_cap][128] partial slot of each row, -1 if the row has none */
+    int32_t* item_order;   /* [Hkv*item_cap] order in which the kernel deals items */
+    int64_t* row_off;      /* [Hq*Nq+1] partial slots of row (h', i) = h'*Nq + i: row_off[..] .. row_off[..+1] */
+    int64_t item_cap;      /* items per KV head the arrays hold */
+    int64_t slot_cap;      /* partial slots the caller's part_o / part_lse hold */
+    int32_t tile_pages;    /* set by qup_page_major_items */
+} qup_page_items;
+
+int qup_page_major_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int T, size_t* ws_bytes,
+                             int64_t* item_cap, int64_t* slot_cap, int32_t* tile_pages);
+
+/*
+ * Builds the page-major items of topk (device int32 [Hq][Nq][Ksel], -1 =
+ * padding) on the stream: five small kernels; a query's place inside the items
+ * of a tile comes from an atomic counter (run-to-run order varies, results do
+ * not).  Device errors: QUP_ERR_PAGE_ID for IDs out of range (dropped),
+ * QUP_ERR_CAPACITY if the items or slots exceed the caps.
+ */
+int qup_page_major_items(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int T,
+                         qup_page_items* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Page-major attention: the union kernel over the items, writing each row's
+ * partial results to part_o (device fp32 [slot_cap][d], 16-byte aligned) and
+ * part_lse (device fp32 [slot_cap]), then the merge into O [Nq][Hq][d] and lse
+ * (fp32 [Nq][Hq] natural log, or NULL).  Other arguments as for
+ * qup_sparse_prefill_attn.
+ */
+int qup_page_major_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
+                        const float* k_scale, const float* v_scale, const int32_t* page_table, int num_logical_pages,
+                        int P_phys, int T, const qup_page_items* items, const int32_t* q_pos, int kv_len, int Hq,
+                        int Hkv, int Nq, int d, float softmax_scale, float* part_o, float* part_lse, void* O,
+                        float* lse, void* stream);
+
 /* Synchronizes `stream`, then reads and clears this device's error word. */
 int qup_get_error(int* code, void* stream);
 

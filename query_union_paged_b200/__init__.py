@@ -20,7 +20,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = ["Groups", "sparse_group", "sparse_prefill_attn", "build_bundles", "groups_from_host", "union_support",
-           "Batch", "batch_prepare", "sparse_prefill_attn_batch",
+           "Batch", "batch_prepare", "sparse_prefill_attn_batch", "PageItems", "page_major_items", "page_major_attn",
            "get_error", "set_debug", "set_checked", "load",
            "QupError", "F32", "BF16", "E4M3", "ERR"]
 
@@ -74,12 +74,18 @@ def load():
     lib.qup_union_support.argtypes = [ctypes.POINTER(_Groups), I, I, I, I, I, P, SZ, P]
     lib.qup_set_checked.argtypes = [I]
     lib.qup_batch_prepare.argtypes = [P, P, I, I, I, I, I, P, P, P, I, P, P, P, P]
+    lib.qup_page_major_workspace.argtypes = [I, I, I, I, I, I, ctypes.POINTER(SZ), ctypes.POINTER(I64),
+                                             ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_int32)]
+    lib.qup_page_major_items.argtypes = [P, I, I, I, I, I, I, ctypes.POINTER(_PageItems), P, SZ, P]
+    lib.qup_page_major_attn.argtypes = [P, I, P, P, I, P, P, P, I, I, I, ctypes.POINTER(_PageItems), P, I, I, I, I,
+                                        I, ctypes.c_float, P, P, P, P, P]
     lib.qup_sparse_prefill_attn_batch.argtypes = [P, I, P, P, I, P, P, P, I, I, I, P, I,
                                                   ctypes.POINTER(_Groups), P, P, I, I, I, I,
                                                   ctypes.c_float, P, P, P]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
                "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support",
-               "qup_set_checked", "qup_batch_prepare", "qup_sparse_prefill_attn_batch"):
+               "qup_set_checked", "qup_batch_prepare", "qup_sparse_prefill_attn_batch", "qup_page_major_workspace",
+               "qup_page_major_items", "qup_page_major_attn"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -279,6 +285,86 @@ def sparse_prefill_attn(Q, K_cache, V_cache, page_table, groups: Groups, q_pos, 
                                        _p(q_pos), kv_len, Hq, Hkv, Nq, d, float(softmax_scale),
                                        _p(out), _p(lse), _stream_ptr(stream)),
            "qup_sparse_prefill_attn")
+    return out
+
+
+class _PageItems(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("n_items", "item_ptr", "item_pages", "item_mask", "item_qid",
+                                               "item_slot", "item_order", "row_off")] + \
+               [("item_cap", ctypes.c_int64), ("slot_cap", ctypes.c_int64), ("tile_pages", ctypes.c_int32)]
+
+
+@dataclasses.dataclass
+class PageItems:
+    """Device arrays of page-major items (see qup_page_items) and the partial-result buffers."""
+    arrays: dict
+    item_cap: int
+    slot_cap: int
+    tile_pages: int
+    workspace: "torch.Tensor"
+    part_o: "torch.Tensor"
+    part_lse: "torch.Tensor"
+
+    def c_struct(self) -> _PageItems:
+        a = self.arrays
+        return _PageItems(*[a[k].data_ptr() for k in ("n_items", "item_ptr", "item_pages", "item_mask", "item_qid",
+                                                      "item_slot", "item_order", "row_off")],
+                          self.item_cap, self.slot_cap, self.tile_pages)
+
+
+def page_major_items(topk, Hq: int, Hkv: int, num_logical_pages: int, T: int, out: Optional[PageItems] = None,
+                     stream=None) -> PageItems:
+    """Page-major items of the TopK rows (qup_page_major_items): tiles of 256 tokens and the
+    queries that meet them, with per-row partial slots."""
+    import torch
+    lib = load()
+    Hq_, Nq, Ksel = topk.shape
+    ws, icap, scap, tp = ctypes.c_size_t(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int32(0)
+    _check(lib.qup_page_major_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, T, ctypes.byref(ws), ctypes.byref(icap),
+                                        ctypes.byref(scap), ctypes.byref(tp)), "qup_page_major_workspace")
+    if out is None:
+        dev = topk.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        g = Hq // Hkv
+        n = Hkv * icap.value
+        arrays = dict(n_items=torch.empty(Hkv, **i32), item_ptr=torch.empty(Hkv, icap.value + 1, **i32),
+                      item_pages=torch.empty(n * tp.value, **i32), item_mask=torch.empty(n * tp.value, 4, **i32),
+                      item_qid=torch.empty(Hkv, icap.value, 128 // g, **i32), item_slot=torch.empty(n, 128, **i32),
+                      item_order=torch.empty(n, **i32),
+                      row_off=torch.empty(Hq * Nq + 1, dtype=torch.int64, device=dev))
+        out = PageItems(arrays=arrays, item_cap=icap.value, slot_cap=scap.value, tile_pages=tp.value,
+                        workspace=torch.empty(max(ws.value, 1), dtype=torch.uint8, device=dev),
+                        part_o=torch.empty(scap.value, 128, dtype=torch.float32, device=dev),
+                        part_lse=torch.empty(scap.value, dtype=torch.float32, device=dev))
+    cs = out.c_struct()
+    _check(lib.qup_page_major_items(_p(topk), Hq, Hkv, Nq, Ksel, num_logical_pages, T, ctypes.byref(cs),
+                                    _p(out.workspace), out.workspace.numel(), _stream_ptr(stream)),
+           "qup_page_major_items")
+    out.tile_pages = cs.tile_pages
+    return out
+
+
+def page_major_attn(Q, K_cache, V_cache, page_table, items: PageItems, q_pos, kv_len: int, k_scale=None,
+                    v_scale=None, softmax_scale: Optional[float] = None, out=None, lse=None,
+                    num_logical_pages: Optional[int] = None, stream=None):
+    """Page-major attention over the items (qup_page_major_attn): partial results per row and
+    tile, then their merge.  Returns O [Nq][Hq][d] in Q's dtype."""
+    import torch
+    lib = load()
+    Nq, Hq, d = Q.shape
+    P_phys, Hkv, T, d2 = K_cache.shape
+    if out is None:
+        out = torch.empty_like(Q)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if num_logical_pages is None:
+        num_logical_pages = page_table.numel()
+    cs = items.c_struct()
+    _check(lib.qup_page_major_attn(_p(Q), _dtype_code(Q), _p(K_cache), _p(V_cache), _dtype_code(K_cache),
+                                   _p(k_scale), _p(v_scale), _p(page_table), num_logical_pages, P_phys, T,
+                                   ctypes.byref(cs), _p(q_pos), kv_len, Hq, Hkv, Nq, d, float(softmax_scale),
+                                   _p(items.part_o), _p(items.part_lse), _p(out), _p(lse), _stream_ptr(stream)),
+           "qup_page_major_attn")
     return out
 
 

@@ -358,12 +358,45 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
 
 namespace {
 
-// The attention call for one sequence (q_pos, kv_len) or for batched requests (q_end, page_len).
+// The attention kernel's work list: bundles of query unions (qup_groups), or page-major items
+// whose rows write partial results.
+struct Work {
+    const int32_t* n_bundles;
+    const int32_t* union_ptr;
+    const int32_t* union_pages;
+    const uint32_t* row_mask;
+    const int32_t* bundle_qid;
+    const int32_t* bundle_order;
+    long long cap_union;
+    int bstride;           // bundles per KV head in the layout of union_ptr and bundle_qid
+    float* part_o;         // page-major: partial results, else null
+    float* part_lse;
+    const int32_t* item_slot;
+};
+
+Work work_of(const qup_groups* g, int Nq) {
+    Work w;
+    w.n_bundles = g->n_bundles;
+    w.union_ptr = g->bunion_ptr;
+    w.union_pages = g->bunion_pages;
+    w.row_mask = g->bunion_mask;
+    w.bundle_qid = g->bundle_qid;
+    w.bundle_order = g->bundle_order;
+    w.cap_union = g->cap_union;
+    w.bstride = Nq;
+    w.part_o = nullptr;
+    w.part_lse = nullptr;
+    w.item_slot = nullptr;
+    return w;
+}
+
+// The attention call for one sequence (q_pos, kv_len) or for batched requests (q_end, page_len),
+// on the bundles of `groups` (checked mode may validate them against topk) or on a work list.
 int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
               const float* k_scale, const float* v_scale, const int32_t* page_table, int num_logical_pages,
-              int P_phys, int T, const int32_t* topk, int Ksel, const qup_groups* groups, const int32_t* q_pos,
-              int kv_len, const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq, int d,
-              float softmax_scale, void* O, float* lse, void* stream) {
+              int P_phys, int T, const int32_t* topk, int Ksel, const qup_groups* groups, const Work* work,
+              const int32_t* q_pos, int kv_len, const int32_t* q_end, const int32_t* page_len, int Hq, int Hkv, int Nq,
+              int d, float softmax_scale, void* O, float* lse, void* stream) {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || d != qup::kHeadDim) return QUP_ERR_ARG;
     if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
     // supported (dtype, page size) pairs: bf16 16/32/64/128, E4M3 64/128, fp32 32/64
@@ -376,16 +409,18 @@ int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cac
     else return QUP_ERR_ARG;
     if (es == 1 && (!k_scale || !v_scale)) return QUP_ERR_ARG;
     if ((es == 1 && T < 64) || (es == 4 && (T < 32 || T > 64))) return QUP_ERR_ARG;
-    if (!groups || !bundle_fields_ok(groups) || groups->rows_per_group < 1) return QUP_ERR_ARG;
+    if (groups && (!bundle_fields_ok(groups) || groups->rows_per_group < 1)) return QUP_ERR_ARG;
+    if (!groups && !work) return QUP_ERR_ARG;
     if ((int64_t)num_logical_pages * T >= ((int64_t)1 << 31)) return QUP_ERR_ARG;  // token positions are int32
     if (Nq == 0) return QUP_OK;
     if (!Q || !K_cache || !V_cache || !page_table || !O) return QUP_ERR_ARG;
     if (!q_end && !q_pos) return QUP_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(K_cache) | reinterpret_cast<uintptr_t>(V_cache)) & 15) return QUP_ERR_ARG;
-    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(groups->bunion_mask)) & 15) return QUP_ERR_ARG;
+    const Work wk = groups ? work_of(groups, Nq) : *work;
+    if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(wk.row_mask)) & 15) return QUP_ERR_ARG;
     const int g = Hq / Hkv;
-    if (128 % g != 0 || groups->rows_per_group % g != 0) return QUP_ERR_ARG;
-    const bool checked = g_checked.load() != 0 && topk != nullptr;
+    if (128 % g != 0 || (groups && groups->rows_per_group % g != 0)) return QUP_ERR_ARG;
+    const bool checked = g_checked.load() != 0 && topk != nullptr && groups != nullptr;
     if (checked && Ksel < 0) return QUP_ERR_ARG;
     DevState* ds = nullptr;
     int rc = device_state(&ds);
@@ -441,19 +476,22 @@ int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cac
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.page_table = page_table;
-    p.n_bundles = groups->n_bundles;
-    p.union_ptr = groups->bunion_ptr;
-    p.union_pages = groups->bunion_pages;
-    p.row_mask = groups->bunion_mask;
-    p.bundle_qid = groups->bundle_qid;
-    p.bundle_order = groups->bundle_order;
+    p.n_bundles = wk.n_bundles;
+    p.union_ptr = wk.union_ptr;
+    p.union_pages = wk.union_pages;
+    p.row_mask = wk.row_mask;
+    p.bundle_qid = wk.bundle_qid;
+    p.bundle_order = wk.bundle_order;
+    p.part_o = wk.part_o;
+    p.part_lse = wk.part_lse;
+    p.item_slot = wk.item_slot;
     p.q_pos = q_pos;
     p.q_end = q_end;
     p.page_len = page_len;
     p.O = O;
     p.lse = lse;
     p.err = ds->err;
-    p.cap_union = groups->cap_union;
+    p.cap_union = wk.cap_union;
     p.num_logical_pages = num_logical_pages;
     p.P_phys = P_phys;
     p.T = T;
@@ -463,6 +501,7 @@ int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cac
     p.Nq = Nq;
     p.g = g;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.bstride = wk.bstride;
     p.nsk = nsk;
     p.nsv = nsv;
     const int wait_ms = g_wait_limit_ms.load();
@@ -484,8 +523,8 @@ int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, con
                             int d, float softmax_scale, void* O, float* lse, void* stream) {
     if (Nq > 0 && !q_pos) return QUP_ERR_ARG;
     return attn_impl(Q, q_dtype, K_cache, V_cache, kv_dtype, k_scale, v_scale, page_table, num_logical_pages,
-                     P_phys, T, topk, Ksel, groups, q_pos, kv_len, nullptr, nullptr, Hq, Hkv, Nq, d, softmax_scale,
-                     O, lse, stream);
+                     P_phys, T, topk, Ksel, groups, nullptr, q_pos, kv_len, nullptr, nullptr, Hq, Hkv, Nq, d,
+                     softmax_scale, O, lse, stream);
 }
 
 int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq, int Ksel, int T, int R,
@@ -516,8 +555,113 @@ int qup_sparse_prefill_attn_batch(const void* Q, int q_dtype, const void* K_cach
                                   float softmax_scale, void* O, float* lse, void* stream) {
     if (Nq > 0 && (!q_end || !page_len)) return QUP_ERR_ARG;
     return attn_impl(Q, q_dtype, K_cache, V_cache, kv_dtype, k_scale, v_scale, page_table, total_pages, P_phys, T,
-                     topk_global, Ksel, groups, nullptr, 0, q_end, page_len, Hq, Hkv, Nq, d, softmax_scale, O, lse,
-                     stream);
+                     topk_global, Ksel, groups, nullptr, nullptr, 0, q_end, page_len, Hq, Hkv, Nq, d, softmax_scale, O,
+                     lse, stream);
+}
+
+int qup_page_major_workspace(int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int T, size_t* ws_bytes,
+                              int64_t* item_cap, int64_t* slot_cap, int32_t* tile_pages) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq < 0 || Ksel < 0 || num_logical_pages <= 0) return QUP_ERR_ARG;
+    if (!(T == 16 || T == 32 || T == 64 || T == 128)) return QUP_ERR_ARG;
+    const int g = Hq / Hkv;
+    if (g > 32 || 128 % g != 0) return QUP_ERR_ARG;
+    const int NW = (num_logical_pages + 31) / 32;
+    if (qup::page_major_build_smem(g, NW) > 227u * 1024u) return QUP_ERR_ARG;
+    const int Pt = 256 / T, ntiles = (num_logical_pages + Pt - 1) / Pt, MQ = 128 / g;
+    // items of one KV head: sum over tiles of ceil(queries meeting the tile / MQ)
+    const int64_t touch = (int64_t)Nq * std::min<int64_t>(ntiles, (int64_t)g * Ksel);
+    const int64_t icap = std::max<int64_t>((touch + MQ - 1) / MQ + ntiles, 1);
+    const int64_t scap = std::max<int64_t>((int64_t)Hq * Nq * std::min<int64_t>(ntiles, Ksel), 1);
+    if (icap * Hkv * Pt >= ((int64_t)1 << 31) || scap >= ((int64_t)1 << 31)) return QUP_ERR_ARG;
+    size_t off = 0;
+    off = align256(off + sizeof(int32_t) * (size_t)Hkv * ntiles);      // tile counts
+    off = align256(off + sizeof(int32_t) * (size_t)Hkv * ntiles);      // tile fill cursors
+    off = align256(off + sizeof(int32_t) * (size_t)Hq * Nq);           // row tile counts
+    off = align256(off + sizeof(int64_t) * (size_t)Hkv * ntiles);      // tile item bases
+    off = align256(off + sizeof(int64_t) * (size_t)(2 + Hkv));         // totals
+    if (ws_bytes) *ws_bytes = off;
+    if (item_cap) *item_cap = icap;
+    if (slot_cap) *slot_cap = scap;
+    if (tile_pages) *tile_pages = Pt;
+    return QUP_OK;
+}
+
+int qup_page_major_items(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int num_logical_pages, int T,
+                         qup_page_items* out, void* ws, size_t ws_bytes, void* stream) {
+    size_t need = 0;
+    int64_t icap = 0, scap = 0;
+    int32_t Pt = 0;
+    int rc = qup_page_major_workspace(Hq, Hkv, Nq, Ksel, num_logical_pages, T, &need, &icap, &scap, &Pt);
+    if (rc) return rc;
+    if (!out || !out->n_items || !out->item_ptr || !out->item_pages || !out->item_mask || !out->item_qid ||
+        !out->item_slot || !out->item_order || !out->row_off)
+        return QUP_ERR_ARG;
+    if ((Nq > 0 && Ksel > 0 && !topk) || !ws) return QUP_ERR_ARG;
+    if (ws_bytes < need || out->item_cap < icap || out->slot_cap < scap) return QUP_ERR_CAPACITY;
+    DevState* ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    out->tile_pages = Pt;
+    if (Nq == 0) return QUP_OK;
+    const int g = Hq / Hkv, NW = (num_logical_pages + 31) / 32, ntiles = (num_logical_pages + Pt - 1) / Pt;
+    char* base = static_cast<char*>(ws);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char* q = base + off;
+        off = align256(off + bytes);
+        return q;
+    };
+    int32_t* tile_cnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)Hkv * ntiles));
+    int32_t* tile_fill = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)Hkv * ntiles));
+    int32_t* row_cnt = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)Hq * Nq));
+    int64_t* tile_base = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)Hkv * ntiles));
+    int64_t* totals = reinterpret_cast<int64_t*>(take(sizeof(int64_t) * (size_t)(2 + Hkv)));
+    if (Ksel == 0) {
+        if (cudaMemsetAsync(out->n_items, 0, sizeof(int32_t) * Hkv, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+            cudaMemsetAsync(out->row_off, 0, sizeof(int64_t) * ((size_t)Hq * Nq + 1),
+                            static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return QUP_ERR_CUDA;
+        return QUP_OK;
+    }
+    return qup::launch_page_major_build(topk, Hq, Hkv, Nq, Ksel, num_logical_pages, NW, Pt, ntiles, 128 / g,
+                                        out->item_cap, out->slot_cap, tile_cnt, tile_fill, row_cnt, tile_base,
+                                        out->row_off, totals, out->n_items, out->item_ptr, out->item_pages,
+                                        out->item_mask, out->item_qid, out->item_slot, out->item_order, ds->err,
+                                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QUP_OK
+               : QUP_ERR_CUDA;
+}
+
+int qup_page_major_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache, int kv_dtype,
+                        const float* k_scale, const float* v_scale, const int32_t* page_table, int num_logical_pages,
+                        int P_phys, int T, const qup_page_items* items, const int32_t* q_pos, int kv_len, int Hq,
+                        int Hkv, int Nq, int d, float softmax_scale, float* part_o, float* part_lse, void* O,
+                        float* lse, void* stream) {
+    if (!items || !items->n_items || !items->item_ptr || !items->item_pages || !items->item_mask ||
+        !items->item_qid || !items->item_slot || !items->item_order || !items->row_off || items->item_cap < 1 ||
+        items->tile_pages != 256 / T)
+        return QUP_ERR_ARG;
+    if (Nq > 0 && (!q_pos || !part_o || !part_lse || !O)) return QUP_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(part_o) & 15) return QUP_ERR_ARG;
+    Work wk;
+    wk.n_bundles = items->n_items;
+    wk.union_ptr = items->item_ptr;
+    wk.union_pages = items->item_pages;
+    wk.row_mask = items->item_mask;
+    wk.bundle_qid = items->item_qid;
+    wk.bundle_order = items->item_order;
+    wk.cap_union = items->item_cap * Hkv * items->tile_pages;
+    wk.bstride = (int)items->item_cap;
+    wk.part_o = part_o;
+    wk.part_lse = part_lse;
+    wk.item_slot = items->item_slot;
+    int rc = attn_impl(Q, q_dtype, K_cache, V_cache, kv_dtype, k_scale, v_scale, page_table, num_logical_pages, P_phys,
+                       T, nullptr, 0, nullptr, &wk, q_pos, kv_len, nullptr, nullptr, Hq, Hkv, Nq, d, softmax_scale, O,
+                       lse, stream);
+    if (rc || Nq == 0) return rc;
+    return qup::launch_page_major_merge(part_o, part_lse, items->row_off, Hq, Nq, q_dtype == QUP_BF16 ? 1 : 0, O, lse,
+                                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QUP_OK
+               : QUP_ERR_CUDA;
 }
 
 int qup_get_error(int* code, void* stream) {

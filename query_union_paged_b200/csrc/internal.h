@@ -63,6 +63,12 @@ struct AttnParams {
     long long cap_union;
     int num_logical_pages, P_phys, T, kv_len, Hq, Hkv, Nq, g;
     float scale_log2;  // softmax_scale * log2(e)
+    int bstride;       // bundles per KV head in the bundle arrays' layout (Nq for groups)
+    // page-major items: every row's partial result (O / l in fp32, log2-domain lse) goes to
+    // part_o[slot][d], part_lse[slot], slot = item_slot[flat item][row] (-1: none); null otherwise
+    float* part_o;
+    float* part_lse;
+    const int32_t* item_slot;
     int nsk, nsv;  // slots of the K ring and of the V ring
     unsigned long long wait_limit_ns;
     int dbg_skip_stage;
@@ -77,6 +83,18 @@ size_t attn_tile_bytes(int es);
 // (read by the bf16 kernel only)
 cudaError_t launch_union_attn(int es, int T, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                               const AttnParams& p, int grid, size_t smem, cudaStream_t stream);
+
+// page-major items (page_major.cu): shared memory of the count and fill kernels, the item
+// builder (count, scan, clear, fill) and the merge of partial results
+size_t page_major_build_smem(int g, int NW);
+cudaError_t launch_page_major_build(const int32_t* topk, int Hq, int Hkv, int Nq, int K, int P, int NW, int Pt,
+                                    int ntiles, int MQ, long long item_cap, long long slot_cap, int32_t* tile_cnt,
+                                    int32_t* tile_fill, int32_t* row_cnt, int64_t* tile_base, int64_t* row_off,
+                                    int64_t* totals, int32_t* n_items, int32_t* item_ptr, int32_t* item_pages,
+                                    uint32_t* item_mask, int32_t* item_qid, int32_t* item_slot, int32_t* item_order,
+                                    unsigned* err, cudaStream_t st);
+cudaError_t launch_page_major_merge(const float* part_o, const float* part_lse, const int64_t* row_off, int Hq, int Nq,
+                                    int q_bf16, void* O, float* lse, cudaStream_t st);
 
 // checked mode: every bundle row's page mask against its own TopK row (QUP_ERR_GROUP on a mismatch)
 cudaError_t launch_check_support(const int32_t* topk, int K, int Hkv, int Nq, int g, int P, const int32_t* n_bundles,

@@ -193,7 +193,7 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_pre
     while (h + 1 < p.Hkv && nb_prefix[h + 1] <= f) ++h;
     it.h = h;
     it.bi = f - nb_prefix[h];
-    const size_t bp = (size_t)h * (p.Nq + 1) + it.bi;
+    const size_t bp = (size_t)h * (p.bstride + 1) + it.bi;
     it.ub = p.union_ptr[bp];
     it.nU = p.union_ptr[bp + 1] - it.ub;
     it.ok = it.ub >= 0 && it.nU >= 0 && (long long)it.ub + it.nU <= p.cap_union;
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < p.Hkv; ++h) {
             nb_prefix[h] = acc;
             int n = p.n_bundles[h];
-            if (n < 0 || n > p.Nq) {
+            if (n < 0 || n > p.bstride) {
                 atomicOr(p.err, QUP_ERR_GROUP);
                 n = 0;
             }
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int m = m0 + lane;
                         int qid = -1;
                         if (m < MQ) {
-                            qid = p.bundle_qid[((size_t)it.h * p.Nq + it.bi) * MQ + m];
+                            qid = p.bundle_qid[((size_t)it.h * p.bstride + it.bi) * MQ + m];
                             if (qid >= p.Nq) {
                                 atomicOr(p.err, QUP_ERR_GROUP);
                                 qid = -1;
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         // the row's bundle state: item, query (original ID), Q head, visible positions, score scale
         Item it{};
-        int qid = -1, head = 0, vis_end = 0;
+        int qid = -1, head = 0, vis_end = 0, fl = 0;
         float cs = p.scale_log2, vscale = 1.f;
         float m_used = kNegInf, lsum = 0.f;
         f2 cs2{cs, cs};
@@ -670,6 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // bundle has completed.  Releases the header.
         auto take = [&](int ino) -> bool {
             if (!warp_ok(mbar_wait(B.stfull(), ino & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim))) return false;
+            fl = sinfo[0];
             it.h = sinfo[1];
             it.bi = sinfo[2];
             it.ub = sinfo[3];
@@ -931,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             const Item it_cur = it;
-            const int qid_cur = qid, head_cur = head;
+            const int qid_cur = qid, head_cur = head, f_cur = fl;
             const float vsc = vscale;
             const float lsum_cur = lsum, m_cur = m_used;
             const int k_last = use - 1;
@@ -965,6 +966,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float inv = ltot > 0.f ? vsc / ltot : 0.f;
             const float a0 = f0 * inv, a1 = f1 * inv;
             const size_t oi = ((size_t)(qid_cur >= 0 ? qid_cur : 0) * p.Hq + head_cur) * kD;
+            // page-major items: this row's partial result goes to its slot (none: -1)
+            const long long pslot = p.part_o ? p.item_slot[(size_t)f_cur * kRows + r] : -1;
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {  // this warpgroup's half of the columns
                 const uint32_t col = 64u * w + 32u * c;
@@ -984,7 +987,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float ov[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o0[e]) * a0 + __uint_as_float(o1[e]) * a1;
-                if (qid_cur >= 0) {
+                if (p.part_o) {
+                    if (pslot >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(p.part_o + (size_t)pslot * kD + col);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dst[e] = make_float4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
+                    }
+                } else if (qid_cur >= 0) {
                     if constexpr (ES == 4) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.O) + oi + col);
 #pragma unroll
@@ -999,7 +1008,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (w == 0 && qid_cur >= 0 && p.lse != nullptr)
+            if (w == 0 && p.part_o && pslot >= 0)  // log2 domain, merged by the page-major reduction
+                p.part_lse[pslot] = ltot > 0.f ? mm + __log2f(ltot) - G::kPLog2 : kNegInf;
+            if (w == 0 && !p.part_o && qid_cur >= 0 && p.lse != nullptr)
                 p.lse[(size_t)qid_cur * p.Hq + head_cur] =
                     ltot > 0.f ? (mm + __log2f(ltot) - G::kPLog2) * 0.69314718055994531f : kNegInf;
             // neither accumulator is overwritten by the next bundle before both warpgroups read it
