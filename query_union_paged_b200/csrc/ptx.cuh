@@ -4,7 +4,6 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
-#include <cuda_fp16.h>
 
 namespace qup {
 
@@ -482,32 +481,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-
-// packed fp16 pair from two fp32 (round to nearest): lo in the low half
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-// 2^x of both fp16 halves in one MUFU instruction
-__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
-    uint32_t r;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
-    return r;
-}
-__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-// both fp16 halves -> E4M3 (saturating), the low half in the low byte
-__device__ __forceinline__ uint32_t e4m3x2_from_f16x2(uint32_t x) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(x));
-    return (uint32_t)r;
-}
-__device__ __forceinline__ float f16_lo(uint32_t x) { return __half2float(__ushort_as_half((unsigned short)(x & 0xffffu))); }
-__device__ __forceinline__ float f16_hi(uint32_t x) { return __half2float(__ushort_as_half((unsigned short)(x >> 16))); }
 
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
     uint16_t lo, hi;

@@ -23,19 +23,22 @@
 // is rare.  A warp whose 32 rows selected none of a step's pages skips that
 // step's exponentials.  Each softmax warp reads the bundle's page numbers and
 // its own 32-bit word of every page's row mask straight from the bundle
-// arrays, 32 entries at a time, one batch ahead; it waits for a V tile only on
-// a step whose page reaches kv_len (whose V rows past kv_len it zeroes).  A
-// quarter of the exponentials come from a polynomial on the FMA pipe
-// (exp2_poly2) and the rest from the MUFU unit.
+// arrays, 32 entries at a time, one batch ahead.  On a page that reaches past
+// the end of its sequence the scores there become -inf and the PV warp zeroes
+// the V rows there (they may hold non-finite bytes).  Two (bf16) or three (E4M3) pairs in eight of the exponentials come
+// from a polynomial on the FMA pipe (exp2_poly2), the rest from the MUFU unit.
+// E4M3 P goes to a shared-memory tile of the warpgroup (its S buffer is then
+// free as soon as the scores are in registers); bf16 and fp32 P go over S.
 //
 // Q: the bundle's rows, gathered by original query ID (no reordered Q tensor),
 // sit in shared memory as the A operand of S in the 128-byte-swizzled K-major
 // layout.  bf16: the V producer loads them by TMA (one box of g heads x 64
 // elements per query and half of d; empty query slots read zeros from outside
 // the tensor) once every S of the previous bundle has completed.  E4M3: the V
-// producer bulk-copies the bf16 rows into a stage, and softmax warpgroup 0
-// quantises each row to E4M3 with its own scale into the operand.  fp32: the
-// same warpgroup copies the rows from global memory.
+// producer bulk-copies the bf16 rows into a stage, and the softmax warpgroups
+// quantise each row to E4M3 with its own scale into the operand (each writes
+// half of every row).  fp32: the two warpgroups copy the rows from global
+// memory, half each.
 //
 // Warp roles (384 threads; warp w runs on SM sub-partition w % 4):
 //   warps 0-3   softmax warpgroup 0 (even steps), warps 4-7 warpgroup 1 (odd
