@@ -101,7 +101,7 @@ GroupWs group_ws_layout(int Hq, int Hkv, int Nq, int NW, int nwin) {
     w.fwcnt = off;
     off = align256(off + sizeof(int32_t) * 5 * (size_t)Hkv * std::max(Nq, 1));
     w.fstatus = off;
-    off = align256(off + sizeof(uint64_t) * 2 * (size_t)Hkv * std::max(Nq, 1) + 16);
+    off = align256(off + sizeof(uint64_t) * 2 * (size_t)Hkv * std::max(Nq, 1) + 16);  // + done word, 2 tickets
     w.total = off;
     return w;
 }
@@ -218,18 +218,19 @@ int run_bundles(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pages, i
     a.err = ds->err;
     a.sms = ds->sms;
     if (fused_bundle_ok(NW, WB, Hkv, ds)) {
-        // status words of the bundle windows (after those of the group windows, if any) and
-        // the completion count start at zero
+        // status words of the bundle windows (after those of the group windows, if any), then
+        // the completion count and the two window tickets (group kernel, bundle kernel), all
+        // starting at zero
         uint64_t* status = reinterpret_cast<uint64_t*>(base + L.fstatus) + fused_status_offset;
         unsigned* done = reinterpret_cast<unsigned*>(status + (size_t)Hkv * a.nwin);
         int32_t* wcnt = reinterpret_cast<int32_t*>(base + L.fwcnt) + 4 * (size_t)Hkv * std::max(Nq, 1);
         if (!gbits_ready) {
-            if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * a.nwin + sizeof(unsigned), st) !=
+            if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * a.nwin + 3 * sizeof(unsigned), st) !=
                 cudaSuccess)
                 return QUP_ERR_CUDA;
         }
         if (!gbits_ready && qup::launch_gbits(a, st) != cudaSuccess) return QUP_ERR_CUDA;
-        return qup::launch_bundles_fused(a, wcnt, status, done, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
+        return qup::launch_bundles_fused(a, wcnt, status, done, done + 2, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
     }
     return qup::launch_bundles(a, st) == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;
 }
@@ -341,10 +342,11 @@ int qup_sparse_group(const int32_t* topk, int Hq, int Hkv, int Nq, int Ksel, int
         const int max_groups = std::min(Nq, nwin * ((window + max_group - 1) / max_group));
         const int nwinB = (max_groups + WB - 1) / WB;
         uint64_t* status = reinterpret_cast<uint64_t*>(base + L.fstatus);
-        if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * (nwin + nwinB) + sizeof(unsigned), st) !=
+        unsigned* done = reinterpret_cast<unsigned*>(status + (size_t)Hkv * (nwin + nwinB));
+        if (cudaMemsetAsync(status, 0, sizeof(uint64_t) * (size_t)Hkv * (nwin + nwinB) + 3 * sizeof(unsigned), st) !=
             cudaSuccess)
             return QUP_ERR_CUDA;
-        if (qup::launch_group_fused(a, a.rowbits, reinterpret_cast<int32_t*>(base + L.fwcnt), status, st) !=
+        if (qup::launch_group_fused(a, a.rowbits, reinterpret_cast<int32_t*>(base + L.fwcnt), status, done + 1, st) !=
             cudaSuccess)
             return QUP_ERR_CUDA;
         return run_bundles(out, Hq, Hkv, Nq, num_logical_pages, max_group, ws, ds, st, true, (size_t)Hkv * nwin,

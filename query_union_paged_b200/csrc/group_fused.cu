@@ -28,10 +28,12 @@
 // Offsets: windows are numbered f = h * nwin + w (the order of the CSR
 // outputs).  Each CTA publishes its window's entry count, then walks back over
 // the windows before it (decoupled look-back) until it meets one that already
-// published its inclusive prefix.  CTAs take windows in increasing f and the
-// grid never exceeds the number of CTAs that can be resident at once, so every
-// window waited on is held by a running CTA.  Each wait is bounded; a wait
-// that runs out raises QUP_ERR_TIMEOUT.
+// published its inclusive prefix.  CTAs claim windows from an atomic ticket, in
+// increasing f: a window is only ever claimed by a CTA that is running, and
+// every window before it was claimed earlier by a running CTA that publishes it
+// without waiting on later windows, so the look-back always ends, however many
+// of the grid's CTAs the device holds at once (other kernels may share it).
+// Each wait is still bounded; a wait that runs out raises QUP_ERR_TIMEOUT.
 #include <algorithm>
 #include <cstdint>
 #include <mutex>
@@ -563,7 +565,8 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
     int nwin, int32_t* __restrict__ group_ptr, int32_t* __restrict__ members, int32_t* __restrict__ n_groups,
     int32_t* __restrict__ union_ptr, int32_t* __restrict__ union_pages, uint64_t* __restrict__ row_mask,
     int64_t* __restrict__ counters, uint32_t* __restrict__ gbits, int32_t* __restrict__ wcnt,
-    uint64_t* __restrict__ status, long long cap, unsigned* err, unsigned spin_limit) {
+    uint64_t* __restrict__ status, unsigned* __restrict__ ticket, long long cap, unsigned* err,
+    unsigned spin_limit) {
     extern __shared__ uint32_t sm_f1[];
     const int g = Hq / Hkv;
     uint32_t* rb = sm_f1;  // [W][g][NW] page bitset of every TopK row of the window
@@ -574,7 +577,12 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     grid_dep_launch();  // the bundle kernel may take free SMs now; it waits for this grid
     const int items = Hkv * nwin;
-    for (int f = blockIdx.x; f < items; f += gridDim.x) {
+    __shared__ int s_f;
+    for (;;) {
+        if (tid == 0) s_f = (int)atomicAdd(ticket, 1u);  // windows in claim order
+        __syncthreads();
+        const int f = s_f;
+        if (f >= items) break;
         const int h = f / nwin, w = f % nwin;
         const int w0 = w * W, nw = min(W, Nq - w0);
         // ---- TopK rows -> row bitsets (-1 is padding, out-of-range IDs are reported and dropped).
@@ -913,8 +921,8 @@ __global__ void __launch_bounds__(kFusedThreads, 2) bnd_fused_kernel(
     int32_t* __restrict__ n_bundles, int32_t* __restrict__ bundle_ptr, int32_t* __restrict__ bundle_groups,
     int32_t* __restrict__ bunion_ptr, int32_t* __restrict__ bunion_pages, uint32_t* __restrict__ bunion_mask,
     int32_t* __restrict__ bundle_qid, int64_t* __restrict__ bcounters, int32_t* __restrict__ bundle_order,
-    int32_t* __restrict__ wcnt, uint64_t* __restrict__ status, unsigned* __restrict__ done, long long cap,
-    unsigned* err, unsigned spin_limit, int order_kcap, int ecap) {
+    int32_t* __restrict__ wcnt, uint64_t* __restrict__ status, unsigned* __restrict__ done,
+    unsigned* __restrict__ ticket, long long cap, unsigned* err, unsigned spin_limit, int order_kcap, int ecap) {
     extern __shared__ uint32_t sm_f2[];
     const WinSmem s = carve(sm_f2, WB, NW);
     // per warp: the bundle's union bitset and its word prefix counts
@@ -934,7 +942,12 @@ __global__ void __launch_bounds__(kFusedThreads, 2) bnd_fused_kernel(
     grid_dep_launch();  // the attention kernel may start its prologue
     grid_dep_wait();    // the group kernel's outputs are complete and visible
     const int items = Hkv * nwinB;
-    for (int f = blockIdx.x; f < items; f += gridDim.x) {
+    __shared__ int s_f;
+    for (;;) {
+        if (tid == 0) s_f = (int)atomicAdd(ticket, 1u);  // windows in claim order
+        __syncthreads();
+        const int f = s_f;
+        if (f >= items) break;
         const int h = f / nwinB, wbi = f % nwinB;
         int ngh = n_groups[h];
         if (ngh < 0 || ngh > Nq) {
@@ -1168,7 +1181,7 @@ static int resident_ctas(Kern kernel, size_t smem, int sms, int threads = kFused
 }
 
 cudaError_t launch_group_fused(const GroupLaunch& a, uint32_t* gbits, int32_t* wcnt, uint64_t* status,
-                               cudaStream_t stream) {
+                               unsigned* ticket, cudaStream_t stream) {
     const int g = a.Hq / a.Hkv;
     const size_t smem = fused_group_smem(a.W, g, a.NW);
     const int items = a.Hkv * a.nwin;
@@ -1181,17 +1194,17 @@ cudaError_t launch_group_fused(const GroupLaunch& a, uint32_t* gbits, int32_t* w
         grid = std::min(items, resident_ctas(grp_fused_kernel<128>, smem, a.sms, 128));
         grp_fused_kernel<128><<<grid, 128, smem, stream>>>(
             a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW, a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
-            a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, a.cap, a.err, 1u << 22);
+            a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, ticket, a.cap, a.err, 1u << 22);
         return cudaGetLastError();
     }
     grp_fused_kernel<256><<<grid, 256, smem, stream>>>(
         a.topk, a.Hq, a.Hkv, a.Nq, a.K, a.P, a.NW, a.max_group, a.W, a.nwin, a.group_ptr, a.members, a.n_groups,
-        a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, a.cap, a.err, 1u << 22);
+        a.union_ptr, a.union_pages, a.row_mask, a.counters, gbits, wcnt, status, ticket, a.cap, a.err, 1u << 22);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bundles_fused(const BundleLaunch& a, int32_t* wcnt, uint64_t* status, unsigned* done,
-                                 cudaStream_t stream) {
+                                 unsigned* ticket, cudaStream_t stream) {
     const size_t smem = fused_bundle_smem(a.WB, a.NW, a.Hkv);
     cudaError_t e = ensure_smem_attr((const void*)bnd_fused_kernel, smem);
     if (e != cudaSuccess) return e;
@@ -1200,7 +1213,7 @@ cudaError_t launch_bundles_fused(const BundleLaunch& a, int32_t* wcnt, uint64_t*
     return launch_pdl(bnd_fused_kernel, dim3(grid), dim3(kFusedThreads), smem, stream,
         (const uint32_t*)a.gbits, a.Hkv, a.Nq, a.NW, a.g, a.RS, a.slots, a.WB, a.nwin, a.n_groups, a.group_ptr, a.members,
         a.union_ptr, a.union_pages, a.row_mask, a.n_bundles, a.bundle_ptr, a.bundle_groups, a.bunion_ptr,
-        a.bunion_pages, a.bunion_mask, a.bundle_qid, a.bcounters, a.bundle_order, wcnt, status, done, a.cap, a.err,
+        a.bunion_pages, a.bunion_mask, a.bundle_qid, a.bcounters, a.bundle_order, wcnt, status, done, ticket, a.cap, a.err,
         1u << 22, (int)((smem - 64) / 4 - (kOrderBuckets2 + 64 + a.Hkv + 1)), kBundleEntryCap);
 }
 

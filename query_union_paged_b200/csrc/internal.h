@@ -167,13 +167,14 @@ cudaError_t launch_bundles(const BundleLaunch& a, cudaStream_t stream);
 
 // Fused grouping path (group_fused.cu): dynamic shared memory of each kernel,
 // and the launches.  wcnt / status are workspace arrays sized for Hkv * Nq
-// windows; status (and the bundle kernel's `done` word) must be zero at launch.
+// windows; status, the bundle kernel's `done` word and each kernel's window
+// ticket must be zero at launch.
 size_t fused_group_smem(int W, int g, int NW);
 size_t fused_bundle_smem(int WB, int NW, int Hkv);
 cudaError_t launch_group_fused(const GroupLaunch& a, uint32_t* gbits, int32_t* wcnt, uint64_t* status,
-                               cudaStream_t stream);
+                               unsigned* ticket, cudaStream_t stream);
 cudaError_t launch_bundles_fused(const BundleLaunch& a, int32_t* wcnt, uint64_t* status, unsigned* done,
-                                 cudaStream_t stream);
+                                 unsigned* ticket, cudaStream_t stream);
 // group union lists -> group bitsets (a.gbits), for bundles of a caller-given partition
 cudaError_t launch_gbits(const BundleLaunch& a, cudaStream_t stream);
 
