@@ -339,9 +339,9 @@ const char* qup_error_string(int code);
 /*
  * Pipeline-wait limit and host-side fault injection (for tests of the bounded
  * waits; both reset with wait_limit_ms <= 0 and skip_stage < 0).  With
- * skip_stage >= 0 the attention kernel's first CTA does not load that ring
- * stage, so the consumer's wait runs out after wait_limit_ms, QUP_ERR_TIMEOUT
- * is raised and every CTA exits cleanly.
+ * skip_stage >= 0 no CTA of the attention kernel loads that stage of its K
+ * and V rings, so the consumers' waits run out after wait_limit_ms,
+ * QUP_ERR_TIMEOUT is raised and every CTA exits cleanly.
  */
 int qup_set_debug(int wait_limit_ms, int skip_stage);
 

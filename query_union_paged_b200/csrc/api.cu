@@ -44,6 +44,7 @@ DevState g_dev[kMaxDevices];
 std::atomic<int> g_wait_limit_ms{0};  // 0: default
 std::atomic<int> g_skip_stage{-1};
 std::atomic<int> g_checked{0};  // checked mode: attention validates the row masks against topk
+std::atomic<unsigned> g_walk_slot{0};  // the next launch slot of the attention kernel's bundle counter
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -509,6 +510,7 @@ int attn_impl(const void* Q, int q_dtype, const void* K_cache, const void* V_cac
     const int wait_ms = g_wait_limit_ms.load();
     p.wait_limit_ns = (unsigned long long)(wait_ms > 0 ? wait_ms : 2000) * 1000000ull;
     p.dbg_skip_stage = g_skip_stage.load();
+    p.walk_slot = (int)(g_walk_slot.fetch_add(1u) % (unsigned)qup::kWalkSlots);
     const cudaError_t e =
         qup::launch_union_attn(es, T, tm[0], tm[1], tmq, p, ds->sms, smem, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QUP_OK : QUP_ERR_CUDA;

@@ -13,6 +13,9 @@ constexpr int kStepTok = 128;   // union tokens per pipeline step (MMA M of S^T,
 constexpr int kHeadDim = 128;
 constexpr int kMaxPPS = 8;      // pages per 128-token step at T = 16
 constexpr int kMaxStages = 16;
+// Launch slots of the attention kernel's run-time bundle counter: launches that run at the
+// same time must hold different slots (the host hands them out in turn).
+constexpr int kWalkSlots = 64;
 
 // Raises a kernel's dynamic shared-memory limit to `smem` once per device context (the
 // attribute is a maximum: later launches with less need no call).
@@ -72,6 +75,7 @@ struct AttnParams {
     int nsk, nsv;  // slots of the K ring and of the V ring
     unsigned long long wait_limit_ns;
     int dbg_skip_stage;
+    int walk_slot;  // 0 .. kWalkSlots-1: this launch's bundle counter
 };
 
 // dynamic shared memory of the attention kernel for (element size, K slots, V slots, KV heads),

@@ -124,13 +124,15 @@ struct Geo {
 };
 
 struct SmemLayout {
-    uint32_t kst, vst, q, p, qst, sinfo, mrg, bars, misc, total;
+    uint32_t kst, vst, q, p, qst, sinfo, mrg, bars, misc, walk, total;
 };
 
 // Stage of the next bundle (E4M3: its bf16 Q rows): query slot m holds the g rows of its query,
 // 256 bytes each, at m * qstage_stride(g); the 16-byte pad keeps row reads free of bank conflicts.
 __host__ __device__ inline uint32_t qstage_stride(int g) { return (uint32_t)g * 256u + 16u; }
 constexpr int kSinfoWords = 8;  // bundle header: flat bundle, h, bi, ub, nU, nsteps, ok
+constexpr int kWalkRing = 64;    // entries of the walk's shared-memory ring (a power of two)
+constexpr int kWalkReaders = 11; // roles that read the walk: softmax warps 0-7, V, S and PV warps
 constexpr int kFixedBars = 16;
 
 __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int Hkv, int g) {
@@ -148,7 +150,7 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     L.qst = off;
     if (es == 1) off += MQ * qstage_stride(g);
     L.sinfo = off;
-    off += 4u * (kSinfoWords + 2u * MQ);  // header, qid[MQ], visible-position end[MQ]
+    off += 4u * (kSinfoWords + MQ);  // header, qid[MQ]
     L.mrg = off;
     off += 2u * kRows * 8u;  // per warpgroup and row: running max and sum (float2)
     off = (off + 7u) & ~7u;
@@ -156,6 +158,9 @@ __host__ __device__ inline SmemLayout smem_layout(int es, int nsk, int nsv, int 
     off += 8u * (2u * (nsk + nsv) + kFixedBars);
     L.misc = off;
     off += 16u + 4u * (uint32_t)(Hkv + 1);
+    off = (off + 15u) & ~15u;
+    L.walk = off;  // the walk: ring, published count, readers' progress
+    off += 4u * (kWalkRing + 1 + kWalkReaders);
     L.total = off + 1024u;  // slack for aligning the dynamic base to 1024
     return L;
 }
@@ -205,18 +210,93 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, const int* nb_pre
     return it;
 }
 
-// Flat bundle index of this CTA's r-th work item, -1 past the end, -2 for a bad
-// order entry (skipped; QUP_ERR_GROUP).  The bundle order (largest unions first)
-// is dealt out in a snake: round r gives CTA b the position r*G + b when r is
-// even and r*G + G-1-b when r is odd, so each CTA's total work stays near the
-// mean.  Positions only grow with r, so the first position past the end ends
-// the walk.  Every role calls this and reaches the same verdict.
-__device__ __forceinline__ int item_at(const AttnParams& p, int r, int n_items) {
-    const long long G = gridDim.x;
-    const long long pos = (long long)r * G + ((r & 1) ? G - 1 - blockIdx.x : (long long)blockIdx.x);
-    if (pos >= n_items) return -1;
-    const int f = p.bundle_order[pos];
-    return (f >= 0 && f < n_items) ? f : -2;
+// ------------------------------------------------------------------ the walk of bundles
+// Bundles are handed out at run time: the K warp of each CTA takes the next position of
+// the bundle order (largest unions first) from a counter shared by the whole grid, so a
+// CTA on a slower SM simply takes fewer bundles.  It publishes the claimed bundles, in
+// order, in a ring in shared memory (-1 ends the walk); every other role reads the
+// same sequence from the ring and records how far it has read, and the K warp does not
+// overwrite an entry before every reader has read it.
+//
+// One counter pair per launch slot: [0] claims, [1] CTAs done.  The last CTA to finish
+// resets both, so the next launch given the same slot starts from zero; the host hands
+// out the slots in turn, so up to kWalkSlots launches may run at once.
+__device__ unsigned g_walk_ticket[kWalkSlots][2];
+
+constexpr int kReaderV = 8, kReaderS = 9, kReaderPV = 10;  // walk readers after the softmax warps
+
+struct Walk {
+    int* ring;           // [kWalkRing] flat bundle indices, -1: end of the walk
+    volatile int* pub;   // entries published so far
+    volatile int* prog;  // [kWalkReaders] entries each reader has read
+};
+
+// Bounded spin of one thread until cond() holds; false (and the abort flag and
+// QUP_ERR_TIMEOUT set) when it runs out, false without an error when another role aborted.
+template <class F>
+__device__ __forceinline__ bool spin_until(F cond, volatile int* abort_flag, unsigned* err, uint64_t limit_ns) {
+    if (cond()) return true;
+    const uint64_t t0 = cycles();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (cond()) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (cycles() - t0 > limit_ns * kCyclesPerNs) {
+                *abort_flag = 1;
+                atomicOr(err, QUP_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Entry j of the walk for reader `reader` (warp-collective; lane 0 waits): the flat bundle
+// index, -1 at the end of the walk or when the wait gave up.
+__device__ __forceinline__ int walk_get(const Walk& wk, int j, int reader, volatile int* abort_flag, unsigned* err,
+                                        uint64_t limit_ns, int lane) {
+    int f = -1;
+    if (lane == 0) {
+        if (spin_until([&] { return *wk.pub > j; }, abort_flag, err, limit_ns)) {
+            __threadfence_block();
+            f = *reinterpret_cast<volatile int*>(wk.ring + (j & (kWalkRing - 1)));
+        }
+        __threadfence_block();  // the entry is read before the K warp may reuse it
+        wk.prog[reader] = j + 1;
+    }
+    return __shfl_sync(0xffffffffu, f, 0);
+}
+
+// K warp, lane 0: claim and publish entry j (once every reader has read entry j - kWalkRing).
+// Bad order entries are reported and skipped.  Returns the published value.
+__device__ __forceinline__ int walk_publish(const Walk& wk, int j, const AttnParams& p, unsigned* ticket, int n_items,
+                                            volatile int* abort_flag, uint64_t limit_ns) {
+    int f = -1;
+    const bool room = spin_until(
+        [&] {
+            int lo = 0x7fffffff;
+#pragma unroll
+            for (int r = 0; r < kWalkReaders; ++r) lo = min(lo, wk.prog[r]);
+            return lo > j - kWalkRing;
+        },
+        abort_flag, p.err, limit_ns);
+    __threadfence_block();  // the readers' progress is seen before the entry is rewritten
+    if (room) {
+        for (;;) {
+            const unsigned t = atomicAdd(ticket, 1u);
+            if (t >= (unsigned)n_items) break;
+            const int ff = p.bundle_order[t];
+            if (ff >= 0 && ff < n_items) {
+                f = ff;
+                break;
+            }
+            atomicOr(p.err, QUP_ERR_GROUP);
+        }
+    }
+    wk.ring[j & (kWalkRing - 1)] = f;
+    __threadfence_block();
+    *wk.pub = j + 1;
+    return f;
 }
 
 // byte offset of 16-byte chunk c of row r inside a K-major SW128 operand tile of `rows` rows
@@ -261,6 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
     int* nb_prefix = reinterpret_cast<int*>(smem + L.misc + 16);
+    const Walk wk{reinterpret_cast<int*>(smem + L.walk), reinterpret_cast<volatile int*>(smem + L.walk) + kWalkRing,
+                  reinterpret_cast<volatile int*>(smem + L.walk) + kWalkRing + 1};
+    unsigned* const ticket = g_walk_ticket[(unsigned)p.walk_slot < (unsigned)kWalkSlots ? p.walk_slot : 0];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t lim = p.wait_limit_ns;
     const int g = p.g, MQ = kRows / g;
@@ -293,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(B.drain2(), 1);
         fence_mbar_init();
         *abort_flag = 0;
+        *wk.pub = 0;
+        for (int r = 0; r < kWalkReaders; ++r) wk.prog[r] = 0;
     }
     if (threadIdx.x == kKProducerWarp * 32) prefetch_tensormap(&tmK);
     if (threadIdx.x == kVProducerWarp * 32) {
@@ -335,10 +420,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ring = sbase + (isV ? L.vst : L.kst);
             int gs = 0, n_done = 0;
             bool ok = true;
-            for (int rnd = 0; ok; ++rnd) {
-                const int f = item_at(p, rnd, n_items);
-                if (f == -1) break;
-                if (f < 0) continue;
+            for (int j = 0; ok; ++j) {
+                // the K warp claims the CTA's next bundle once it has issued every K tile of the
+                // previous one; the V warp reads the same entry of the walk
+                int f = -1;
+                if (!isV) {
+                    if (lane == 0) f = walk_publish(wk, j, p, ticket, n_items, abort_flag, lim);
+                    f = __shfl_sync(0xffffffffu, f, 0);
+                } else {
+                    f = walk_get(wk, j, kReaderV, abort_flag, p.err, lim, lane);
+                }
+                if (f < 0) break;
                 const Item it = load_item<PPS>(p, nb_prefix, f);
                 if (isV) {
                     // the header, once every softmax warp has read the previous bundle's
@@ -363,10 +455,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             qid = max(qid, -1);
                             sinfo[kSinfoWords + m] = qid;
-                            // positions < this end are visible to the query (batched requests: its
-                            // precomputed end in the global token space)
-                            sinfo[kSinfoWords + MQ + m] =
-                                qid < 0 ? 0 : (p.q_end ? p.q_end[qid] : min(p.q_pos[qid] + 1, p.kv_len));
                         }
                         nvalid += __popc(__ballot_sync(0xffffffffu, qid >= 0));
                     }
@@ -446,8 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                  abort_flag, p.err, QUP_ERR_TIMEOUT, lim);
                         ok = __shfl_sync(0xffffffffu, okv, 0) != 0;
                         if (!ok) break;
-                        const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && blockIdx.x == 0 &&
-                                                          gs == p.dbg_skip_stage);
+                        const bool issue = lane == 0 && !(p.dbg_skip_stage >= 0 && gs == p.dbg_skip_stage);
                         int ph[PPS];
 #pragma unroll
                         for (int q = 0; q < PPS; ++q) ph[q] = __shfl_sync(0xffffffffu, phys, k * PPS + q);
@@ -480,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (ES == 2) mbar_wait_drain(B.qfull(), (n_done - 1) & 1, lim);
                 }
                 for (int i = max(0, gs - NR); i < gs; ++i) {
-                    if (p.dbg_skip_stage >= 0 && blockIdx.x == 0 && i == p.dbg_skip_stage) continue;
+                    if (p.dbg_skip_stage >= 0 && i == p.dbg_skip_stage) continue;
                     mbar_wait_drain(isV ? B.vfull(i % NR) : B.kfull(i % NR), (i / NR) & 1, lim);
                 }
             }
@@ -505,9 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int ks = 0, kph = 0, vs = 0, vph = 0;  // ring slot and phase of the next step
             bool ok = true;
             for (int rnd = 0; ok; ++rnd) {
-                const int f = item_at(p, rnd, n_items);
-                if (f == -1) break;
-                if (f < 0) continue;
+                const int f = walk_get(wk, rnd, isS ? kReaderS : kReaderPV, abort_flag, p.err, lim, lane);
+                if (f < 0) break;
                 const Item it = load_item<PPS>(p, nb_prefix, f);
                 if (isS) {
                     ok = warp_ok(mbar_wait_idle(B.qfull(), item_no & 1, abort_flag, p.err, QUP_ERR_TIMEOUT, lim));
@@ -681,7 +767,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             it.nsteps = sinfo[5];
             it.ok = sinfo[6] != 0;
             qid = sinfo[kSinfoWords + r / g];
-            const int qend = sinfo[kSinfoWords + MQ + r / g];
+            // positions < this end are visible to the query (batched requests: its precomputed end
+            // in the global token space); loaded alongside the first union entries
+            const int qend = qid < 0 ? 0 : (p.q_end ? p.q_end[qid] : min(p.q_pos[qid] + 1, p.kv_len));
             if (!it.ok && threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
             head = it.h * g + (r % g);
             vis_end = qend;  // positions < vis_end are visible
@@ -750,15 +838,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(B.stempty());
             return true;
         };
-        // the walk of bundles: -1 past the end; order entries that are bad are reported and skipped
-        auto walk = [&](int& rr) -> int {
-            int ff = item_at(p, rr, n_items);
-            while (ff == -2) {
-                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
-                ff = item_at(p, ++rr, n_items);
-            }
-            return ff;
-        };
+        // entry rr of the CTA's walk of bundles: -1 past the end
+        auto walk = [&](int rr) -> int { return walk_get(wk, rr, warp, abort_flag, p.err, lim, lane); };
         // exponentials of one step: p = 2^(s*cs - m_used + kPLog2), their sum returned.  P leaves
         // every 16 tokens as it is made (E4M3: one 16-byte chunk of row r of this warpgroup's
         // shared-memory P tile; bf16: 8 TMEM columns over S_w), so no more than a chunk of it is
@@ -823,9 +904,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         int f = walk(rnd);
         if (f >= 0) ok = take(0);
         while (f >= 0 && ok) {
-            // the next bundle's flat index: loaded now, used after this bundle's steps
-            int rnd2 = rnd + 1;
-            const int f2raw = item_at(p, rnd2, n_items);
             m_used = kNegInf;
             lsum = 0.f;
             for (int s = w; s < it.nsteps; s += 2) {
@@ -941,12 +1019,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int k_last = use - 1;
             const int n0 = (it_cur.nsteps + 1) / 2, n1 = it_cur.nsteps / 2;  // steps of each warpgroup
             // The next bundle's header (and Q operand) is taken before this bundle's epilogue, so
-            // its first S = Q K^T runs while the epilogue reads O.
-            int fn = f2raw;
-            while (fn == -2) {
-                if (threadIdx.x == 0) atomicOr(p.err, QUP_ERR_GROUP);
-                fn = item_at(p, ++rnd2, n_items);
-            }
+            // its first S = Q K^T runs while the epilogue reads O.  Its entry of the walk is read
+            // only now: the K warp claims it once this bundle's K tiles are all issued.
+            const int rnd2 = rnd + 1;
+            const int fn = walk(rnd2);
             if (fn >= 0) ok = take(item_no + 1);
             if (!ok) break;
             // ---- epilogue: merge the two warpgroups' partial rows, O / l -> O[qid][head][:]
@@ -1034,6 +1110,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == kSWarp) tmem_dealloc(tmem, kTmemCols);
+    // the last CTA out resets this launch slot's bundle counter (every claim has been made)
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(ticket + 1, 1u) == gridDim.x - 1) {
+            atomicExch(ticket, 0u);
+            atomicExch(ticket + 1, 0u);
+        }
+    }
 }
 
 size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g) { return smem_layout(es, nsk, nsv, Hkv, g).total; }
