@@ -236,6 +236,42 @@ def oracle_sample(w, target_s: float = 12.0, seed: int = 0):
     return tflops, threads, f"{n} of {w.Hq * w.Nq} (query head, query) rows, {edges} selected edges, {dt:.1f} s"
 
 
+def group_reference_sample(w, max_group: int, window: int, repeats: int = 3):
+    """Time the CPU grouping reference (oracle.group, plain C) on the whole workload: one thread,
+    and one call per query window spread over a thread pool (groups never cross a window, so the
+    windows are independent calls; ctypes releases the GIL during each).  Median of `repeats`.
+    The counters of the windowed calls are checked against the single call's."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    topk = np.ascontiguousarray(w.topk)
+    starts = list(range(0, w.Nq, window))
+    slices = [np.ascontiguousarray(topk[:, a:a + window, :]) for a in starts]
+    threads = os.cpu_count() or 1
+
+    def one():
+        return oracle.group(topk, w.Hq, w.Hkv, w.Nq, w.num_logical_pages, max_group, window)
+
+    def windowed(pool):
+        return list(pool.map(lambda t: oracle.group(t, w.Hq, w.Hkv, t.shape[1], w.num_logical_pages,
+                                                     max_group, window), slices))
+
+    t1 = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        ref = one()
+        t1.append(time.perf_counter() - t0)
+    tn = []
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            parts = windowed(pool)
+            tn.append(time.perf_counter() - t0)
+    match = bool(np.array_equal(sum(pt["counters"] for pt in parts), ref["counters"]))
+    return {"single_thread_us": round(statistics.median(t1) * 1e6, 1),
+            "threads_over_windows_us": round(statistics.median(tn) * 1e6, 1),
+            "threads": threads, "windows": len(starts), "counters_match": match}
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -342,6 +378,13 @@ def main():
     code = qup.get_error()
     if code:
         raise RuntimeError(f"device error {code} during the timed steps")
+    # the same steps with a warm L2 (no flush between them), reported beside the cold numbers
+    wevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        step(wevs[k])
+    torch.cuda.synchronize()
+    w_group = [wevs[k][0].elapsed_time(wevs[k][1]) for k in range(args.steps)]
+    w_attn = [wevs[k][1].elapsed_time(wevs[k][2]) for k in range(args.steps)]
     t_group = [evs[k][0].elapsed_time(evs[k][1]) for k in range(args.steps)]
     t_attn = [evs[k][1].elapsed_time(evs[k][2]) for k in range(args.steps)]
     t_step = [a + b for a, b in zip(t_group, t_attn)]
@@ -386,6 +429,9 @@ def main():
                         "attn": round(statistics.median(t_attn) * 1e3, 2),
                         "complete": round(statistics.median(t_step) * 1e3, 2),
                         "attn_min": round(min(t_attn) * 1e3, 2), "attn_max": round(max(t_attn) * 1e3, 2)},
+        "warm_l2_us_per_call": {"group": round(statistics.median(w_group) * 1e3, 2),
+                                "attn": round(statistics.median(w_attn) * 1e3, 2),
+                                "complete": round(statistics.median([a + b for a, b in zip(w_group, w_attn)]) * 1e3, 2)},
         "work": {"selected_edges": E, "flop": flop, "unique_kv_pages": n_uniq,
                  "unique_kv_bytes": uniq_bytes, "logical_page_visits": int(ctr[0]),
                  "masked_row_slots": int(ctr[1]), "masked_query_slots": int(ctr[2]),
@@ -414,7 +460,8 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             tf, cores, desc = oracle_sample(w)
             line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                    "sample": desc}
+                                    "sample": desc,
+                                    "group_reference": group_reference_sample(w, max_group, window)}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

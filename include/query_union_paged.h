@@ -92,8 +92,8 @@ extern "C" {
  *            the pages the attention kernel streams), number of bundles.
  *   bundle_order[0 .. total bundles) = flat bundle indices (f = bundles of
  *            earlier KV heads + b) sorted by union size, largest first, equal
- *            sizes by index: the order in which the attention kernel deals
- *            bundles to its CTAs.
+ *            sizes by index: the order in which the attention kernel's CTAs
+ *            claim bundles at run time.
  */
 typedef struct {
     int32_t* n_groups;     /* [Hkv] */
@@ -218,6 +218,11 @@ int qup_union_support(qup_groups* g, int Hq, int Hkv, int Nq, int num_logical_pa
  *   lse               device fp32 [Nq][Hq] natural-log sum of exponentials of
  *                     the scaled scores, or NULL; empty support gives O = 0,
  *                     lse = -inf
+ * The CTAs claim bundles at run time from a device counter; each launch takes
+ * the next of 64 counters per device in turn, so at most 64 launches of the
+ * attention kernel (this call, the batched and page-major calls) may run at
+ * the same time, and a captured CUDA graph holding one must not be replayed
+ * while a replay of the same graph is still running.
  */
 int qup_sparse_prefill_attn(const void* Q, int q_dtype, const void* K_cache, const void* V_cache,
                             int kv_dtype, const float* k_scale, const float* v_scale,
@@ -297,7 +302,7 @@ typedef struct {
     uint32_t* item_mask;   /* [Hkv*item_cap*tile_pages][4] 128-bit row masks, as bunion_mask */
     int32_t* item_qid;     /* [Hkv][item_cap][128/g] query of each query slot, -1 if empty */
     int32_t* item_slot;    /* [Hkv*item_cap][128] partial slot of each row, -1 if the row has none */
-    int32_t* item_order;   /* [Hkv*item_cap] order in which the kernel deals items */
+    int32_t* item_order;   /* [Hkv*item_cap] order in which the kernel's CTAs claim items */
     int64_t* row_off;      /* [Hq*Nq+1] partial slots of row (h', i) = h'*Nq + i: row_off[..] .. row_off[..+1] */
     int64_t item_cap;      /* items per KV head the arrays hold */
     int64_t slot_cap;      /* partial slots the caller's part_o / part_lse hold */

@@ -720,8 +720,8 @@ cudaError_t launch_group(const GroupLaunch& a, cudaStream_t stream) {
 // Work order of the attention kernel: the flat bundle indices (KV heads in
 // order, then bundles) sorted by union size, largest first, equal sizes by
 // index (a stable counting sort; sizes above kOrderBuckets-1 share the top
-// bucket).  The attention kernel deals this order out to its CTAs in a snake,
-// which keeps the per-CTA sums of union pages close to the mean.
+// bucket).  The attention kernel's CTAs claim bundles in this order at run
+// time, so the largest go first and the smallest fill the end.
 constexpr int kOrderBuckets = 4096;
 
 __global__ void __launch_bounds__(1024) bnd_order_kernel(const int32_t* __restrict__ n_bundles,

@@ -43,3 +43,13 @@ def test_tiny_workload_edge_count_is_exact():
     E = bench.selected_edges_per_row(w)
     own_part = (w.q_pos % w.T) + 1
     assert np.array_equal(E[0], 7 * w.T + own_part)
+
+
+def test_grouping_reference_over_windows_matches_the_single_call():
+    """The windowed timing of the CPU grouping reference runs one call per query window; groups
+    never cross a window, so the summed counters equal those of the single whole-workload call."""
+    w = W.tiny_ref()
+    r = bench.group_reference_sample(w, w.max_group, w.window, repeats=1)
+    assert r["counters_match"]
+    assert r["windows"] == -(-w.Nq // w.window)
+    assert r["single_thread_us"] > 0 and r["threads_over_windows_us"] > 0
