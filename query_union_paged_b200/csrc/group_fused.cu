@@ -111,20 +111,43 @@ __device__ inline WinSmem carve(uint32_t* base, int W, int NW) {
     return s;
 }
 
+// 32 x 32 bit matrix held one row per lane (bit k of lane i = element (i, k)) transposed in
+// place: afterwards bit i of lane k = element (i, k).  Five block swaps: at width j, the rows
+// with bit j clear take the left-hand columns of row i + j into their right-hand half, and
+// rows with bit j set take the right-hand columns of row i - j into their left-hand half.
+__device__ __forceinline__ void transpose32(uint32_t& x, int lane) {
+    const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int j = 16 >> i;
+        const uint32_t m = masks[i];  // columns k with (k & j) == 0
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+        x = (lane & j) ? ((x & ~m) | ((y & ~m) >> j)) : ((x & m) | ((y & m) << j));
+    }
+}
+
 // Universe, its prefix counts, set sizes and compact sets of items [0, n).
 // Whole CTA; ends with the compact sets ready (a barrier inside).
 __device__ void compact_window(const WinSmem& s, int n, int NW) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int wd = tid; wd < NW; wd += blockDim.x) s.UW[wd] = 0u;
-    for (int a = tid; a < n; a += blockDim.x) s.ssize[a] = 0;
     __syncthreads();
-    for (int x = tid; x < n * NW; x += blockDim.x) {
-        const uint32_t v = s.S[x];
-        if (v) {
-            const int a = x / NW;
-            atomicOr(&s.UW[x - a * NW], v);
-            atomicAdd(&s.ssize[a], __popc(v));
-        }
+    // universe words: each thread ORs one word over a run of items, then one atomic per run
+    // (atomics of every item on the same few words would serialise)
+    const int runs = max(1, (int)blockDim.x / max(NW, 1));
+    const int per = (n + runs - 1) / runs;
+    for (int x = tid; x < NW * runs; x += blockDim.x) {
+        const int wd = x % NW, c = x / NW;
+        const int a1 = min(n, (c + 1) * per);
+        uint32_t acc = 0u;
+        for (int a = c * per; a < a1; ++a) acc |= s.S[(size_t)a * NW + wd];
+        if (acc) atomicOr(&s.UW[wd], acc);
+    }
+    // set sizes: one thread per item
+    for (int a = tid; a < n; a += blockDim.x) {
+        int c = 0;
+        for (int wd = 0; wd < NW; ++wd) c += __popc(s.S[(size_t)a * NW + wd]);
+        s.ssize[a] = c;
     }
     __syncthreads();
     if (warp == 0) {  // exclusive prefix of popc(UW) over words
@@ -148,23 +171,29 @@ __device__ void compact_window(const WinSmem& s, int n, int NW) {
         }
     }
     __syncthreads();
-    const int NWC = s.misc[1], NWCp = NW | 1;
+    const int NWCp = NW | 1;
     for (int x = tid; x < n * NWCp; x += blockDim.x) s.cs[x] = 0u;
     __syncthreads();
+    // compact sets (bit c = the c-th page of the universe): one thread per (item, word); the
+    // word's bits land at ranks p0 .. p0 + popc(universe word) - 1, in at most two compact words,
+    // so a word costs at most two atomics however many bits it has
     for (int x = tid; x < n * NW; x += blockDim.x) {
-        const int a = x / NW, wd = x % NW;
         uint32_t v = s.S[x];
         if (!v) continue;
+        const int a = x / NW, wd = x - a * NW;
         const uint32_t uw = s.UW[wd];
         const int p0 = s.pref[wd];
+        uint64_t acc = 0u;
         while (v) {
             const int b = __ffs(v) - 1;
             v &= v - 1;
-            const int c = p0 + __popc(uw & ((1u << b) - 1u));
-            atomicOr(&s.cs[(size_t)a * NWCp + (c >> 5)], 1u << (c & 31));
+            acc |= 1ull << __popc(uw & ((1u << b) - 1u));
         }
+        acc <<= (p0 & 31);
+        uint32_t* dst = s.cs + (size_t)a * NWCp + (p0 >> 5);
+        if ((uint32_t)acc) atomicOr(dst, (uint32_t)acc);
+        if ((uint32_t)(acc >> 32)) atomicOr(dst + 1, (uint32_t)(acc >> 32));
     }
-    (void)NWC;
     __syncthreads();
 }
 
@@ -617,8 +646,14 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
                         put(v[u].w);
                     }
                 }
-            } else {
-                for (int k = 0; k < K; ++k) put(src[k]);
+            } else {  // 16 loads in flight at a time (the stores to dst could alias src for the compiler)
+                for (int k0 = 0; k0 < K; k0 += 16) {
+                    int v[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) v[u] = k0 + u < K ? __ldg(src + k0 + u) : -1;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) put(v[u]);
+                }
             }
         }
         __syncthreads();
@@ -686,7 +721,9 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
         const bool fits = base + total <= cap;
         if (tid == 0 && !fits) atomicOr(err, QUP_ERR_CAPACITY);
         const int gbase = w * (W / max_group);
-        // ---- emit: one warp per group
+        // ---- emit: one warp per group; lane r holds row r of the group (row = member rank * g +
+        // head; max_group * g <= 32), so the union word is one OR reduction and each page's row
+        // mask one ballot
         for (int k = warp; k < ng; k += kWarps) {
             const int m0 = s.gstart[k], cnt = s.gstart[k + 1] - m0, R = cnt * g;
             const int gi = gbase + k;
@@ -695,44 +732,23 @@ __global__ void __launch_bounds__(NT, 65536 / (NT * 128)) grp_fused_kernel(
                 group_ptr[(size_t)h * (Nq + 1) + gi] = w0 + m0;
                 union_ptr[(size_t)h * (Nq + 1) + gi] = (int32_t)(base + s.goff[k]);
             }
-            // the group's union bitset (for the bundle pass) and its sorted pages
-            const int wpl = (NW + 31) >> 5;
-            const int wb = min(NW, lane * wpl), we = min(NW, wb + wpl);
-            int c = 0;
-            for (int wd = wb; wd < we; ++wd) {
-                uint32_t u = 0;
-                for (int m = 0; m < cnt; ++m) u |= s.S[(size_t)s.order[m0 + m] * NW + wd];
-                gbits[((size_t)h * Nq + gi) * NW + wd] = u;
-                c += __popc(u);
-            }
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            int rank = incl - c;
-            if (fits) {
-                const long long out0 = base + s.goff[k];
-                for (int wd = wb; wd < we; ++wd) {
-                    uint32_t u = 0;
-                    for (int m = 0; m < cnt; ++m) u |= s.S[(size_t)s.order[m0 + m] * NW + wd];
-                    if (!u) continue;
-                    uint32_t rw[32];  // row r = member rank * g + head: its bits of this word
-#pragma unroll
-                    for (int r = 0; r < 32; ++r)
-                        rw[r] = r < R ? rb[((size_t)s.order[m0 + r / g] * g + (r % g)) * NW + wd] : 0u;
-                    while (u) {
-                        const int b = __ffs(u) - 1;
-                        u &= u - 1;
-                        uint64_t mk = 0;
-#pragma unroll
-                        for (int r = 0; r < 32; ++r) mk |= (uint64_t)((rw[r] >> b) & 1u) << r;
-                        union_pages[out0 + rank] = wd * 32 + b;
-                        row_mask[out0 + rank] = mk;
-                        ++rank;
-                    }
+            const uint32_t* row0 =
+                lane < R ? rb + ((size_t)s.order[m0 + lane / g] * g + (lane % g)) * NW : nullptr;
+            long long out = base + s.goff[k];
+            for (int wd = 0; wd < NW; ++wd) {
+                // the 32 x 32 bit block (row = lane, page = bit) transposed: lane b ends with page
+                // wd * 32 + b's row mask
+                uint32_t x = row0 ? row0[wd] : 0u;
+                transpose32(x, lane);
+                const uint32_t u = __ballot_sync(0xffffffffu, x != 0u);
+                // the group's union bitset (for the bundle pass) and its pages in order
+                if (lane == 0) gbits[((size_t)h * Nq + gi) * NW + wd] = u;
+                if (fits && x != 0u) {
+                    const long long e = out + __popc(u & ((1u << lane) - 1u));
+                    union_pages[e] = wd * 32 + lane;
+                    row_mask[e] = (uint64_t)x;
                 }
+                out += __popc(u);
             }
         }
         if (tid == 0) {
