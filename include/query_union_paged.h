@@ -265,6 +265,36 @@ int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq,
                       int32_t* topk_global, int32_t* q_end, int32_t* page_len, void* stream);
 
 /*
+ * Proxy-query page selection, the step upstream of qup_sparse_group that
+ * produces each query's TopK pages (PIVOT: Efficient Query-Group Indexing for
+ * Token-Level Sparse Attention, Abstract: one shared full-prefix scan per
+ * group of nearby queries instead of one per query).  Queries are cut into
+ * groups of group_size consecutive IDs; per KV head and group the mean of the
+ * group's indexer queries (the proxy) scores every page the group's last
+ * query can see, and its n_cand best pages are the candidates.  Each query
+ * then takes Ksel of the candidates it can see (page p is visible to a query
+ * at position q iff p * T <= q): re-scored with its own indexer query
+ * (refine = 1, PIVOT-Refine) or in the proxy's order (refine = 0,
+ * PIVOT-Reuse).  A score is the dot product of an indexer query with a page's
+ * indexer key, computed in float32 with every product and sum rounded in
+ * element order (the proxy: queries summed in ID order, then divided by the
+ * group size); order = higher score first, equal scores by lower page ID.
+ *   q_idx      device [Nq][Hkv][d_idx], dtype QUP_BF16 or QUP_F32, 16-byte aligned
+ *   page_key   device [num_logical_pages][Hkv][d_idx], same dtype, 16-byte aligned
+ *   q_pos      device int32 [Nq], token positions (>= 0)
+ *   g          query heads per KV head (1..32): each KV head's selection is
+ *              written to its g query heads
+ *   topk       out: device int32 [Hkv*g][Nq][Ksel], -1 padded (the topk of
+ *              qup_sparse_group, with num_logical_pages pages)
+ * Limits (QUP_ERR_ARG otherwise): d_idx <= 512 and a multiple of 8 (bf16) or
+ * 4 (fp32); num_logical_pages <= 8192; 1 <= Ksel <= n_cand <= 256.  Nothing is
+ * allocated; the call is asynchronous on `stream`.
+ */
+int qup_pivot_select(const void* q_idx, const void* page_key, int dtype, const int32_t* q_pos, int Nq, int Hkv,
+                     int g, int d_idx, int num_logical_pages, int T, int group_size, int n_cand, int Ksel,
+                     int refine, int32_t* topk, void* stream);
+
+/*
  * qup_sparse_prefill_attn for batched requests: the arguments of
  * qup_sparse_prefill_attn with (q_pos, kv_len) replaced by the q_end and
  * page_len arrays of qup_batch_prepare, page_table the concatenated table of

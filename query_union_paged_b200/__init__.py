@@ -79,13 +79,14 @@ def load():
     lib.qup_page_major_items.argtypes = [P, I, I, I, I, I, I, ctypes.POINTER(_PageItems), P, SZ, P]
     lib.qup_page_major_attn.argtypes = [P, I, P, P, I, P, P, P, I, I, I, ctypes.POINTER(_PageItems), P, I, I, I, I,
                                         I, ctypes.c_float, P, P, P, P, P]
+    lib.qup_pivot_select.argtypes = [P, P, I, P, I, I, I, I, I, I, I, I, I, I, P, P]
     lib.qup_sparse_prefill_attn_batch.argtypes = [P, I, P, P, I, P, P, P, I, I, I, P, I,
                                                   ctypes.POINTER(_Groups), P, P, I, I, I, I,
                                                   ctypes.c_float, P, P, P]
     for fn in ("qup_group_workspace", "qup_sparse_group", "qup_build_bundles", "qup_sparse_prefill_attn",
                "qup_get_error", "qup_set_debug", "qup_num_sms", "qup_exp2_poly", "qup_union_support",
                "qup_set_checked", "qup_batch_prepare", "qup_sparse_prefill_attn_batch", "qup_page_major_workspace",
-               "qup_page_major_items", "qup_page_major_attn"):
+               "qup_page_major_items", "qup_page_major_attn", "qup_pivot_select"):
         getattr(lib, fn).restype = I
     _lib = lib
     return lib
@@ -395,6 +396,23 @@ def batch_prepare(topk, q_pos, q_ptr, page_ptr, kv_len, total_pages: int, T: int
                                     total_pages, _p(b.topk_global), _p(b.q_end), _p(b.page_len),
                                     _stream_ptr(stream)), "qup_batch_prepare")
     return b
+
+
+def pivot_select(q_idx, page_key, q_pos, g: int, T: int, group_size: int, n_cand: int, K: int,
+                 refine: bool = True, out=None, stream=None):
+    """Proxy-query page selection (qup_pivot_select): TopK page IDs per (query head, query) for
+    sparse_group.  q_idx [Nq][Hkv][d_idx] and page_key [P][Hkv][d_idx] bf16 or fp32 CUDA tensors,
+    q_pos int32 [Nq]; returns int32 [Hkv*g][Nq][K] (-1 padded)."""
+    import torch
+    Nq, Hkv, d = q_idx.shape
+    P = page_key.shape[0]
+    assert page_key.shape[1:] == (Hkv, d) and page_key.dtype == q_idx.dtype
+    if out is None:
+        out = torch.empty((Hkv * g, Nq, K), dtype=torch.int32, device=q_idx.device)
+    _check(load().qup_pivot_select(_p(q_idx), _p(page_key), _dtype_code(q_idx), _p(q_pos), Nq, Hkv, g, d, P, T,
+                                   group_size, n_cand, K, 1 if refine else 0, _p(out), _stream_ptr(stream)),
+           "qup_pivot_select")
+    return out
 
 
 def sparse_prefill_attn_batch(Q, K_cache, V_cache, page_table, groups: Groups, batch: Batch, k_scale=None,

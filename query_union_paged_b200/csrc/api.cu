@@ -551,6 +551,28 @@ int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq,
                : QUP_ERR_CUDA;
 }
 
+int qup_pivot_select(const void* q_idx, const void* page_key, int dtype, const int32_t* q_pos, int Nq, int Hkv,
+                     int g, int d_idx, int num_logical_pages, int T, int group_size, int n_cand, int Ksel,
+                     int refine, int32_t* topk, void* stream) {
+    if (Nq < 0 || Hkv <= 0 || g <= 0 || g > 32 || T <= 0 || group_size <= 0) return QUP_ERR_ARG;
+    if (dtype != QUP_BF16 && dtype != QUP_F32) return QUP_ERR_ARG;
+    if (d_idx <= 0 || d_idx > qup::kMaxSelDim || d_idx % (dtype == QUP_BF16 ? 8 : 4) != 0) return QUP_ERR_ARG;
+    if (num_logical_pages <= 0 || num_logical_pages > qup::kMaxSelPages) return QUP_ERR_ARG;
+    if (n_cand <= 0 || n_cand > qup::kMaxSelCand || Ksel <= 0 || Ksel > n_cand) return QUP_ERR_ARG;
+    if (refine != 0 && refine != 1) return QUP_ERR_ARG;
+    if (Nq > 0 && (!q_idx || !page_key || !q_pos || !topk)) return QUP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(q_idx) & 15) || (reinterpret_cast<uintptr_t>(page_key) & 15)) return QUP_ERR_ARG;
+    DevState* ds = nullptr;
+    int rc = device_state(&ds);
+    if (rc) return rc;
+    if (qup::pivot_select_smem(num_logical_pages, d_idx) > (size_t)ds->smem_optin) return QUP_ERR_ARG;
+    return qup::launch_pivot_select(q_idx, page_key, dtype == QUP_BF16, q_pos, Nq, Hkv, g, d_idx, num_logical_pages,
+                                    T, group_size, n_cand, Ksel, refine == 1, topk,
+                                    static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QUP_OK
+               : QUP_ERR_CUDA;
+}
+
 int qup_sparse_prefill_attn_batch(const void* Q, int q_dtype, const void* K_cache, const void* V_cache,
                                   int kv_dtype, const float* k_scale, const float* v_scale,
                                   const int32_t* page_table, int total_pages, int P_phys, int T,

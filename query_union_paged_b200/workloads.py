@@ -302,6 +302,44 @@ def random_small(seed: int, Hq=4, Hkv=2, Nq=100, d=128, T=64, prefix=960, K=6,
                    sel, max_group=max_group, window=window, identity_pages=identity_pages)
 
 
+@dataclasses.dataclass
+class IndexerInputs:
+    """Inputs of the proxy-query page selector: indexer queries q [Nq][Hkv][d] and page keys
+    k [P][Hkv][d] (float32 values that bf16 holds exactly when bf16, plus their bf16 bits),
+    positions q_pos [Nq]."""
+    q: np.ndarray
+    k: np.ndarray
+    q_bits: Optional[np.ndarray]
+    k_bits: Optional[np.ndarray]
+    q_pos: np.ndarray
+    T: int
+    num_logical_pages: int
+
+
+def indexer_inputs(seed: int, Nq: int, Hkv: int, d: int, prefix: int, T: int, bf16: bool = True,
+                   integer: bool = False, shuffle_positions: bool = False, extra_pages: int = 0) -> IndexerInputs:
+    """Seeded indexer queries and page keys: N(0, 1) (or small integers in -3..3, which make every
+    score exact and produce ties), for a chunk of Nq queries after `prefix` tokens.  The positions
+    are prefix + 0 .. Nq-1, optionally permuted; the page space covers them plus extra_pages."""
+    rng = np.random.default_rng(seed)
+    P = (prefix + Nq + T - 1) // T + extra_pages
+    if integer:
+        q = rng.integers(-3, 4, size=(Nq, Hkv, d)).astype(np.float32)
+        k = rng.integers(-3, 4, size=(P, Hkv, d)).astype(np.float32)
+    else:
+        q = rng.standard_normal((Nq, Hkv, d), dtype=np.float32)
+        k = rng.standard_normal((P, Hkv, d), dtype=np.float32)
+    qb = kb = None
+    if bf16:
+        qb, kb = f32_to_bf16_bits(q), f32_to_bf16_bits(k)
+        q = (qb.astype(np.uint32) << 16).view(np.float32)
+        k = (kb.astype(np.uint32) << 16).view(np.float32)
+    pos = prefix + np.arange(Nq, dtype=np.int32)
+    if shuffle_positions:
+        pos = rng.permutation(pos).astype(np.int32)
+    return IndexerInputs(q, k, qb, kb, pos, T, P)
+
+
 CONFIGS = {
     "1": tiny_ref,
     "2": gqa_chunk_bf16,

@@ -135,3 +135,25 @@ def test_checked_mode_argument_and_no_device_answer(lib):
                                           ctypes.c_void_p(0x70000), None, None)
     assert rc == qup.ERR["CUDA"], rc
 """)
+
+
+def test_pivot_select_rejects_bad_arguments_before_any_device_work(lib):
+    _run_without_devices("""
+    import ctypes
+    import query_union_paged_b200 as qup
+    qup.load()
+    f = qup._lib.qup_pivot_select
+    q, k, pos, out = (ctypes.c_void_p(a) for a in (0x10000, 0x20000, 0x30000, 0x40000))
+    good = dict(dtype=1, Nq=64, Hkv=2, g=4, d=128, P=100, T=64, G=16, C=32, K=8, refine=1)
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(q, k, a["dtype"], pos, a["Nq"], a["Hkv"], a["g"], a["d"], a["P"], a["T"], a["G"], a["C"],
+                 a["K"], a["refine"], out, None)
+    for bad in (dict(C=0), dict(C=257), dict(K=33), dict(K=0), dict(d=100), dict(d=1024), dict(P=9000),
+                dict(G=0), dict(g=33), dict(dtype=2), dict(refine=2)):
+        assert call(**bad) == qup.ERR["ARG"], bad
+    # fp32 index vectors need a multiple of 4 only
+    assert call(dtype=0, d=100) == qup.ERR["CUDA"]
+    # valid arguments reach the device lookup, which answers that there is no device
+    assert call() == qup.ERR["CUDA"]
+""")
