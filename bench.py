@@ -289,6 +289,9 @@ def main():
     ap.add_argument("--page-major", action="store_true",
                     help="direct KV-page union: page-major items and partial results merged by lse")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--select", choices=["refine", "reuse"], default=None,
+                    help="also time the proxy-query page selector (qup_pivot_select) on indexer inputs of the "
+                         "workload's shape (128-wide index vectors, groups of 16, 4 x TopK candidates)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -408,6 +411,36 @@ def main():
                 W.DT_E4M3: peaks["bf16_tflops"] * 2}[w.kv_dtype]
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
 
+    # ---- the upstream selector, timed alone (not part of the step or its metric)
+    select = None
+    if args.select:
+        prefix = int(w.q_pos.min())
+        base_p = (prefix + w.Nq + w.T - 1) // w.T
+        inp = W.indexer_inputs(7, w.Nq, w.Hkv, 128, prefix, w.T, extra_pages=max(0, w.num_logical_pages - base_p))
+        qi = torch.from_numpy(inp.q_bits).cuda().view(torch.bfloat16)
+        pk = torch.from_numpy(inp.k_bits).cuda().view(torch.bfloat16)
+        qp = torch.from_numpy(inp.q_pos).cuda()
+        G, C, Ks = 16, min(256, 4 * w.K), w.K
+        sel_out = torch.empty((w.Hq, w.Nq, Ks), dtype=torch.int32, device="cuda")
+        refine = args.select == "refine"
+        for _ in range(3):
+            qup.pivot_select(qi, pk, qp, w.Hq // w.Hkv, w.T, G, C, Ks, refine=refine, out=sel_out)
+        sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            sev[k][0].record(stream)
+            qup.pivot_select(qi, pk, qp, w.Hq // w.Hkv, w.T, G, C, Ks, refine=refine, out=sel_out)
+            sev[k][1].record(stream)
+        torch.cuda.synchronize()
+        assert qup.get_error() == 0
+        groups_n = (w.Nq + G - 1) // G
+        scan_macs = w.Hkv * sum(min(inp.num_logical_pages, int(inp.q_pos[g0:g0 + G].max()) // w.T + 1)
+                                for g0 in range(0, w.Nq, G)) * 128
+        select = {"variant": args.select, "group_size": G, "n_cand": C, "topk": Ks, "index_dim": 128,
+                  "us_per_call": round(statistics.median([a.elapsed_time(b) for a, b in sev]) * 1e3, 2),
+                  "proxy_scan_macs": int(scan_macs), "groups": groups_n * w.Hkv,
+                  "refine_macs": int(w.Hkv * w.Nq * C * 128) if refine else 0}
+
     # ---- end to end through host buffers (pinned), copies inside the timed region
     e2e = None if args.page_major else run_e2e(args, w, qup, dev, ks, vs, groups, max_group, window, stream, O, flop)
 
@@ -452,6 +485,7 @@ def main():
                      ("" if w.kv_dtype == W.DT_BF16 else " x nominal dtype ratio"),
                      "unique_kv_gbs": round(uniq_bytes / (attn_ms * 1e-3) / 1e9, 1),
                      "hbm_frac_unique_kv": round(uniq_bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        **({"select": select} if select else {}),
         "gpu_launches": (LAUNCHES_PER_STEP + (LAUNCHES_UNION_SUPPORT if args.union_support else 0)) * args.steps,
         "e2e": e2e,
     }

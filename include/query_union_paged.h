@@ -287,8 +287,10 @@ int qup_batch_prepare(const int32_t* topk, const int32_t* q_pos, int Hq, int Nq,
  *   topk       out: device int32 [Hkv*g][Nq][Ksel], -1 padded (the topk of
  *              qup_sparse_group, with num_logical_pages pages)
  * Limits (QUP_ERR_ARG otherwise): d_idx <= 512 and a multiple of 8 (bf16) or
- * 4 (fp32); num_logical_pages <= 8192; 1 <= Ksel <= n_cand <= 256.  Nothing is
- * allocated; the call is asynchronous on `stream`.
+ * 4 (fp32); num_logical_pages <= 8192; 1 <= Ksel <= n_cand <= 256; and one
+ * CTA's shared memory must hold num_logical_pages * 8 + n_cand * d_idx *
+ * (2 or 4) + 36 * d_idx + 2048 bytes (the candidates' key rows are staged
+ * there).  Nothing is allocated; the call is asynchronous on `stream`.
  */
 int qup_pivot_select(const void* q_idx, const void* page_key, int dtype, const int32_t* q_pos, int Nq, int Hkv,
                      int g, int d_idx, int num_logical_pages, int T, int group_size, int n_cand, int Ksel,

@@ -565,7 +565,8 @@ int qup_pivot_select(const void* q_idx, const void* page_key, int dtype, const i
     DevState* ds = nullptr;
     int rc = device_state(&ds);
     if (rc) return rc;
-    if (qup::pivot_select_smem(num_logical_pages, d_idx) > (size_t)ds->smem_optin) return QUP_ERR_ARG;
+    if (qup::pivot_select_smem(num_logical_pages, d_idx, dtype == QUP_BF16 ? 2 : 4, n_cand) > (size_t)ds->smem_optin)
+        return QUP_ERR_ARG;
     return qup::launch_pivot_select(q_idx, page_key, dtype == QUP_BF16, q_pos, Nq, Hkv, g, d_idx, num_logical_pages,
                                     T, group_size, n_cand, Ksel, refine == 1, topk,
                                     static_cast<cudaStream_t>(stream)) == cudaSuccess

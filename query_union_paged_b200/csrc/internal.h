@@ -83,7 +83,7 @@ struct AttnParams {
 constexpr int kMaxSelCand = 256;
 constexpr int kMaxSelPages = 8192;
 constexpr int kMaxSelDim = 512;
-size_t pivot_select_smem(int num_logical_pages, int d);
+size_t pivot_select_smem(int num_logical_pages, int d, int esize, int n_cand);
 cudaError_t launch_pivot_select(const void* q_idx, const void* page_key, bool bf16, const int32_t* q_pos, int Nq,
                                 int Hkv, int g, int d, int P, int T, int G, int n_cand, int K, bool refine,
                                 int32_t* topk, cudaStream_t stream);
