@@ -2,7 +2,8 @@
 // Abstract; Figure 1; Figure 3), re-designed for tcgen05 + TMEM.
 //
 // Work item: a bundle of up to 128 query rows (up to 128 / rows_per_group
-// page-affine groups of one KV head, see qup_groups).  Pages of the bundle
+// page-affine groups of one KV head, see qup_groups); each CTA claims its
+// bundles at run time, largest unions first (the walk, below).  Pages of the bundle
 // union are streamed once per bundle in steps of 128 tokens (one 128-token
 // page, or 128 / T smaller pages) through two TMA rings, one of K tiles and
 // one of V tiles.  Step s of a bundle belongs to softmax warpgroup w = s % 2,
@@ -43,11 +44,12 @@
 // Warp roles (384 threads; warp w runs on SM sub-partition w % 4):
 //   warps 0-3   softmax warpgroup 0 (even steps), warps 4-7 warpgroup 1 (odd
 //               steps); both run the epilogue, each for half of the columns.
-//   warp 8      K producer: walks the bundle's page list, resolves physical
-//               pages (warp-parallel) and TMA-loads the K tiles.
+//   warp 8      K producer: claims the CTA's bundles and publishes them to
+//               the other roles; walks each bundle's page list, resolves
+//               physical pages (warp-parallel) and TMA-loads the K tiles.
 //   warp 10     V producer: the same walk for the V tiles; writes each
-//               bundle's header (query IDs and positions of its rows) and
-//               loads or stages its Q rows.
+//               bundle's header (item and query IDs of its rows) and loads
+//               or stages its Q rows.
 //   warp 9      S issuer (one elected lane of a warp-uniform loop) and TMEM
 //               owner (512 columns): S(s) once K tile s has landed and the O
 //               update that last read P from S_w has finished.
