@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "select.h"
 #include "query_union_paged.h"
 
 namespace qup {

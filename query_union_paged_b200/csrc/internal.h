@@ -78,16 +78,6 @@ struct AttnParams {
     int walk_slot;  // 0 .. kWalkSlots-1: this launch's bundle counter
 };
 
-// Proxy-query page selection (select.cu): at most kMaxSelCand candidates per group, at most
-// kMaxSelPages logical pages (the block-wide sort holds them all), index width <= kMaxSelDim.
-constexpr int kMaxSelCand = 256;
-constexpr int kMaxSelPages = 8192;
-constexpr int kMaxSelDim = 512;
-size_t pivot_select_smem(int num_logical_pages, int d, int esize, int n_cand);
-cudaError_t launch_pivot_select(const void* q_idx, const void* page_key, bool bf16, const int32_t* q_pos, int Nq,
-                                int Hkv, int g, int d, int P, int T, int G, int n_cand, int K, bool refine,
-                                int32_t* topk, cudaStream_t stream);
-
 // dynamic shared memory of the attention kernel for (element size, K slots, V slots, KV heads),
 // and one K or V tile (one ring slot)
 size_t attn_smem_bytes(int es, int nsk, int nsv, int Hkv, int g);

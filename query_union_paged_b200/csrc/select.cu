@@ -20,6 +20,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "select.h"
 #include "query_union_paged.h"
 
 namespace qup {
